@@ -1,0 +1,186 @@
+"""CPU oracle for pyramid top-K block selection + causal block-sparse attention.
+
+TEST INFRASTRUCTURE ONLY. The tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may call it; the CUDA product path never does.
+
+The arithmetic lives in ``pyr_oracle.c`` (plain C, double accumulation, no
+code shared with the CUDA library). This wrapper only compiles it with gcc
+and marshals arguments. Every function follows the PISA abstract (pyramid of
+pooled keys, coarse-to-fine LogSumExp scoring of a bounded candidate set) and
+the PHBA summary (block centroids as mean key rows; routes to strictly
+preceding blocks, -1 padding; the current block always attended causally;
+output plus log-sum-exp). See the header of ``pyr_oracle.c`` for the readings
+taken where the pages are silent.
+
+Parity pins (tests/test_oracle_*.py) check this oracle against closed forms,
+library routines, brute force and invariants, never against the CUDA path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pyr_oracle.c")
+_OUT = os.path.join(_HERE, "_build", "liboracle.so")
+
+
+class OraShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "Hq", "Hkv", "N", "Nq", "q_offset", "d", "b", "topk", "cap",
+                                             "dtype")]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (gcc -O2, OpenMP over independent units)."""
+    if force or not os.path.exists(_OUT) or os.path.getmtime(_OUT) < os.path.getmtime(_SRC):
+        os.makedirs(os.path.dirname(_OUT), exist_ok=True)
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c11", _SRC, "-o",
+                               _OUT + ".tmp", "-lm"])
+        os.replace(_OUT + ".tmp", _OUT)
+    return _OUT
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        sp = ctypes.POINTER(OraShape)
+        lib.ora_num_levels.argtypes = [sp]
+        lib.ora_num_levels.restype = ctypes.c_int
+        lib.ora_num_nodes.argtypes = [sp]
+        lib.ora_num_nodes.restype = ctypes.c_int64
+        lib.ora_num_qblocks.argtypes = [sp]
+        lib.ora_num_qblocks.restype = ctypes.c_int64
+        lib.ora_first_qblock.argtypes = [sp]
+        lib.ora_first_qblock.restype = ctypes.c_int64
+        lib.ora_pyramid.argtypes = [sp, _P, ctypes.c_int, _P, _P]
+        lib.ora_pyramid.restype = ctypes.c_int
+        lib.ora_node_score.argtypes = [sp, _P, _P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+        lib.ora_node_score.restype = ctypes.c_int
+        lib.ora_select.argtypes = [sp, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P, _P]
+        lib.ora_select.restype = ctypes.c_int
+        lib.ora_attend.argtypes = [sp, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P]
+        lib.ora_attend.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def shape_of(w) -> OraShape:
+    """OraShape from any object with the workload fields (B, Hq, ..., dtype)."""
+    return OraShape(w.B, w.Hq, w.Hkv, w.N, w.Nq, w.q_offset, w.d, w.b, w.topk, w.cap, w.dtype)
+
+
+def _ptr(t):
+    if isinstance(t, torch.Tensor):
+        assert t.device.type == "cpu" and t.is_contiguous()
+        return t.data_ptr()
+    assert isinstance(t, np.ndarray) and t.flags["C_CONTIGUOUS"]
+    return t.ctypes.data
+
+
+def num_levels(w) -> int:
+    return _load().ora_num_levels(ctypes.byref(shape_of(w)))
+
+
+def num_nodes(w) -> int:
+    return _load().ora_num_nodes(ctypes.byref(shape_of(w)))
+
+
+def num_qblocks(w) -> int:
+    return _load().ora_num_qblocks(ctypes.byref(shape_of(w)))
+
+
+def level_offsets(w):
+    """(offset, count) of each pyramid level in the level-major node list."""
+    nb = (w.N + w.b - 1) // w.b
+    out, off, l = [], 0, 0
+    while True:
+        n = (nb + (1 << l) - 1) >> l
+        out.append((off, n))
+        off += n
+        if n == 1:
+            break
+        l += 1
+    return out
+
+
+def pyramid(w, K, units) -> np.ndarray:
+    """Pyramids of the listed (batch*Hkv + kv_head) units: [len(units), P, d] float64."""
+    units = np.ascontiguousarray(np.asarray(units, dtype=np.int32))
+    out = np.empty((len(units), num_nodes(w), w.d), dtype=np.float64)
+    rc = _load().ora_pyramid(ctypes.byref(shape_of(w)), _ptr(K), len(units), _ptr(units), _ptr(out))
+    if rc:
+        raise ValueError(f"ora_pyramid rc={rc}")
+    return out
+
+
+def node_score(w, Q, pyr_unit: np.ndarray, unit: int, qb: int, level: int, m: int):
+    """(score, n_valid) of node (level, m) for query block qb; (-inf, 0) if invalid."""
+    s, n = ctypes.c_double(), ctypes.c_double()
+    pyr_unit = np.ascontiguousarray(pyr_unit)
+    _load().ora_node_score(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(pyr_unit), unit, qb, level, m,
+                           ctypes.byref(s), ctypes.byref(n))
+    return s.value, n.value
+
+
+def select(w, Q, pyr: np.ndarray, units, items, start_level: int = -1):
+    """Selection for items [(slot, qb), ...]; slot indexes ``units`` / ``pyr``.
+
+    Returns (idx [n, topk] int32, gap [n] float64, ncand [n, L+1] int32).
+    """
+    units = np.ascontiguousarray(np.asarray(units, dtype=np.int32))
+    items = np.asarray(items, dtype=np.int64).reshape(-1, 2)
+    slot = np.ascontiguousarray(items[:, 0].astype(np.int32))
+    qb = np.ascontiguousarray(items[:, 1].astype(np.int64))
+    n = len(items)
+    idx = np.empty((n, max(w.topk, 1)), dtype=np.int32)
+    gap = np.empty(n, dtype=np.float64)
+    ncand = np.empty((n, num_levels(w)), dtype=np.int32)
+    pyr = np.ascontiguousarray(pyr)
+    rc = _load().ora_select(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(pyr), len(units), _ptr(units), n, _ptr(slot),
+                            _ptr(qb), start_level, _ptr(idx), _ptr(gap), _ptr(ncand))
+    if rc:
+        raise ValueError(f"ora_select rc={rc}")
+    return idx[:, :w.topk], gap, ncand
+
+
+def select_all(w, Q, K, units=None, start_level: int = -1):
+    """Full selection for the listed units (default: all): idx [U, nqb, topk], gap [U, nqb], ncand."""
+    if units is None:
+        units = list(range(w.B * w.Hkv))
+    pyr = pyramid(w, K, units)
+    nqb = num_qblocks(w)
+    items = [(s, q) for s in range(len(units)) for q in range(nqb)]
+    idx, gap, ncand = select(w, Q, pyr, units, items, start_level)
+    return idx.reshape(len(units), nqb, w.topk), gap.reshape(len(units), nqb), ncand.reshape(len(units), nqb, -1)
+
+
+def attend(w, Q, K, V, idx, rows, dense: bool = False):
+    """Attention for flat query rows ((b*Hq + hq)*Nq + t): (O [n, d], lse [n]) float64.
+
+    idx: [B, Hkv, nqb, topk] int32 (ignored when dense).
+    """
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = len(rows)
+    O = np.empty((n, w.d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    if idx is None:
+        idx_arr = np.zeros(1, dtype=np.int32)
+    else:
+        idx_arr = np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+    rc = _load().ora_attend(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(K), _ptr(V), _ptr(idx_arr), n, _ptr(rows),
+                            1 if dense else 0, _ptr(O), _ptr(lse))
+    if rc == 2:
+        raise ValueError("ora_attend: idx lists a block that is not strictly before the query block, or repeats")
+    if rc:
+        raise ValueError(f"ora_attend rc={rc}")
+    return O, lse
