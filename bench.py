@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""Forward throughput of pyramid selection + causal block-sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole path over one batch of synthetic input:
+pyr_build (key pyramid) -> pyr_select (coarse-to-fine LogSumExp top-K) ->
+bsa_forward (causal block-sparse attention), through the C ABI. The default
+workload is the 32K-token bf16 MHA prefill (B=1, H=16, N=32768, d=128, b=64,
+top-K=16 + diagonal, cap 32). Inputs (Q, K, V: 384 MiB) are larger than the
+126 MB L2, so consecutive steps do not run from cache.
+
+Prints ONE JSON line on rank 0. `value` is tokens/s = B*N per step, summed over
+ranks, divided by the max over ranks of the device time of the K timed steps.
+With N > 1 (torchrun, one process per GPU) every rank runs its own workload
+instance: the path shards by (batch, kv head) with no exchange step, so the
+scaling is weak and there is no collective on the data path.
+
+--impl reference times the CPU oracle (test infrastructure, plain C in double)
+on the host cores, on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "fwd tokens/s (select+attn) at 32K–1M ctx; % HBM & tensor roofline vs CPU oracle"
+DEFAULT_WORKLOAD = "mha_bf16_32k"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+CSRC = os.path.join(ROOT, "hierarchical_block_sparse_pyr_b200", "csrc")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+# ------------------------------------------------------------ work counts --
+
+def level_sizes(w):
+    nb = w.nb
+    out, l = [], 0
+    while True:
+        n = -(-nb // (1 << l))
+        out.append(n)
+        if n == 1:
+            break
+        l += 1
+    return out
+
+
+def work_counts(w):
+    """Algorithmic bytes / FLOPs of one step (exact counts from the method's definition)."""
+    elt = 4 if w.dtype == synth.F32 else 2
+    lv = level_sizes(w)
+    P = sum(lv)
+    U = w.B * w.Hkv
+    first = w.q_offset // w.b
+    nqb = (w.q_offset + w.Nq - 1) // w.b - first + 1
+    s0 = 0
+    while lv[s0] > w.cap:
+        s0 += 1
+    # selection: candidates scored per level (upper bound per level: all valid nodes at s0, then <= cap)
+    sel_flops = 0
+    sel_exps = 0
+    att_pairs = 0
+    for qb in range(nqb):
+        i = first + qb
+        p0, p1 = max(i * w.b, w.q_offset), min((i + 1) * w.b, w.q_offset + w.Nq)
+        rows = w.G * (p1 - p0)
+        nc = -(-i // (1 << s0))  # valid nodes at s0: those starting before block i
+        for l in range(s0, -1, -1):
+            sel_flops += 2 * rows * nc * w.d
+            sel_exps += rows * nc
+            keep = min(w.cap // 2 if l > 0 else w.topk, nc)
+            if l > 0:
+                # children of the kept nodes that start before i (at most 2 per kept node)
+                nc = min(2 * keep, -(-i // (1 << (l - 1))))
+        nsel = min(w.topk, i)
+        # selected blocks are strictly before i (full blocks); the diagonal is causal
+        n = p1 - p0
+        att_pairs += w.G * (n * nsel * w.b + (p0 - i * w.b + 1 + p1 - i * w.b) * n // 2)
+    sel_flops *= U
+    sel_exps *= U
+    att_pairs *= U
+    att_flops = 4 * w.d * att_pairs
+    pyr_bytes = U * (w.N * w.d * elt + P * w.d * 4)
+    q_bytes = w.B * w.Hq * w.Nq * w.d * elt
+    sel_bytes = q_bytes + U * P * w.d * 4 + U * nqb * w.topk * 4
+    # attention: Q + O once; K, V of the selected + diagonal blocks once per query block and kv head
+    kv_blocks = 0
+    for qb in range(nqb):
+        i = first + qb
+        kv_blocks += min(w.topk, i) + 1
+    att_bytes = 2 * q_bytes + U * kv_blocks * 2 * w.b * w.d * elt
+    return dict(pyr_bytes=pyr_bytes, sel_flops=sel_flops, sel_exps=sel_exps, sel_bytes=sel_bytes,
+                att_flops=att_flops, att_bytes=att_bytes, att_pairs=att_pairs, tokens=w.B * w.Nq)
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def src_hash(files):
+    h = hashlib.sha256()
+    for fn in files:
+        with open(os.path.join(CSRC, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {"pyramid": ["pyramid.cu"], "select": ["select.cu"], "attention": ["attn_simt.cu"]}
+
+
+def measured_traffic(kernel, workload):
+    """dram bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        t = json.load(f)
+    rec = t.get(workload, {}).get(kernel)
+    if not rec or rec.get("src_sha") != src_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, pw, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                pw.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        load = [s for s, p in zip(sm, pw) if p > 200] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(pw) if pw else None}
+
+
+# --------------------------------------------------------------- our arm --
+
+def count_launches(step):
+    """Kernels of libpyr launched by one step (profiled outside the timed region)."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+        ours = [n for n in names if any(k in n for k in ("pyr_", "select_kernel", "attn_", "bsa_", "dense_"))]
+        return len(ours), sorted(set(ours))
+    except Exception as ex:  # profiler unavailable: report unknown
+        return None, [f"profiler unavailable: {ex}"]
+
+
+def run_ours(args, w, rank, world, local_rank):
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = P.shape_of(w)
+    Qh, Kh, Vh, _ = synth.generate(w, pin=True)
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    buf = P.Buffers(s, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        P.pyr_build(s, K, buf.pyr, buf.status, stream)
+        if ev:
+            ev[1].record(stream)
+        P.pyr_select(s, Q, buf.pyr, buf.idx, buf.gap, buf.status, stream)
+        if ev:
+            ev[2].record(stream)
+        P.bsa_forward(s, Q, K, V, buf.idx, buf.O, buf.lse, buf.status, stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {buf.status.item()}: {P.strerror(int(buf.status.item()))}")
+    launches_per_step, kernel_names = count_launches(step)
+
+    # timed region: K steps, per-kernel events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    per = {"pyramid": [], "select": [], "attention": []}
+    for ev in evs:
+        per["pyramid"].append(ev[0].elapsed_time(ev[1]))
+        per["select"].append(ev[1].elapsed_time(ev[2]))
+        per["attention"].append(ev[2].elapsed_time(ev[3]))
+    ms_t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end to end through the binding: pinned host inputs -> device -> path -> O back to pinned host
+    O_host = torch.empty(buf.O.shape, dtype=buf.O.dtype, pin_memory=True)
+    h2d = Qh.numel() * Qh.element_size() + Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
+    d2h = O_host.numel() * O_host.element_size()
+
+    def e2e_step():
+        Q.copy_(Qh, non_blocking=True)
+        K.copy_(Kh, non_blocking=True)
+        V.copy_(Vh, non_blocking=True)
+        step()
+        O_host.copy_(buf.O, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {buf.status.item()}")
+
+    wc = work_counts(w)
+    peaks = load_peaks()
+    ms_step = ms_max / args.steps
+    value = world * wc["tokens"] / (ms_step * 1e-3)
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    sm_clock = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    kernels = {
+        "pyramid": dict(ms=avg["pyramid"], bound="hbm", achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9,
+                        peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["pyr_bytes"],
+                        traffic=measured_traffic("pyramid", w.name)),
+        "select": dict(ms=avg["select"], bound="alu",
+                       achieved=wc["sel_flops"] / (avg["select"] * 1e-3) / 1e12,
+                       peak=148 * 128 * 2 * sm_clock * 1e6 / 1e12, unit="TFLOP/s", algorithmic=wc["sel_flops"],
+                       hbm_gbs=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9,
+                       traffic=measured_traffic("select", w.name)),
+        "attention": dict(ms=avg["attention"], bound="alu",
+                          achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
+                          peak=148 * 128 * 2 * sm_clock * 1e6 / 1e12, unit="TFLOP/s", algorithmic=wc["att_flops"],
+                          traffic=measured_traffic("attention", w.name)),
+    }
+    for k in kernels.values():
+        k["frac"] = k["achieved"] / k["peak"]
+        k["share"] = k["ms"] / ms_step
+    dom_name = max(kernels, key=lambda k: kernels[k]["ms"])
+    dom = kernels[dom_name]
+    roofline = {"kernel": dom_name, "bound": dom["bound"], "achieved": round(dom["achieved"], 3),
+                "peak": round(dom["peak"], 3), "unit": dom["unit"], "frac": round(dom["frac"], 4),
+                "traffic": dom["traffic"],
+                "peak_source": ("measured" if dom["bound"] != "alu" and peaks["source"] == "measured" else
+                                "derived: 148 SMs x 128 FP32 lanes x 2 x median SM clock under load"
+                                if dom["bound"] == "alu" else "fallback")}
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == synth.BF16 else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d, "b": w.b,
+                   "topk": w.topk, "cap": w.cap, "seed": w.seed, "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (Q+K+V %d MiB > 126 MB)" % (
+                       (Qh.numel() + Kh.numel() + Vh.numel()) * Qh.element_size() >> 20)},
+        "e2e": {"value": round(world * wc["tokens"] / (float(e_ms.item()) * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
+        "roofline": roofline,
+        "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
+                    for k, v in kernels.items()},
+        "kernel_names": kernel_names,
+        "clocks": clk,
+        "peaks_source": peaks["source"],
+    }
+    return out
+
+
+# -------------------------------------------------------- oracle baseline --
+
+def oracle_sample(w, n_qb, seed=0, Q=None, K=None, V=None):
+    """Time the oracle on one (batch, kv head) unit: its pyramid, n_qb evenly spaced query blocks
+    (selection + attention of all their rows). Returns (seconds, est. seconds for the whole job, desc)."""
+    import oracle
+
+    if Q is None:
+        Q, K, V, _ = synth.generate(w)
+    nqb = oracle.num_qblocks(w)
+    U = w.B * w.Hkv
+    unit = seed % U
+    bi, hk = divmod(unit, w.Hkv)
+    qbs = np.unique(np.linspace(0, nqb - 1, num=min(n_qb, nqb)).round().astype(int))
+    t0 = time.perf_counter()
+    pyr = oracle.pyramid(w, K, [unit])
+    t1 = time.perf_counter()
+    idx_u, _, _ = oracle.select(w, Q, pyr, [unit], [(0, int(q)) for q in qbs])
+    t2 = time.perf_counter()
+    full_idx = -np.ones((w.B, w.Hkv, nqb, w.topk), dtype=np.int32)
+    full_idx[bi, hk, qbs] = idx_u
+    rows = []
+    first = w.q_offset // w.b
+    for q in qbs:
+        i = first + int(q)
+        p0, p1 = max(i * w.b, w.q_offset), min((i + 1) * w.b, w.q_offset + w.Nq)
+        for g in range(w.G):
+            hq = hk * w.G + g
+            rows += [((bi * w.Hq + hq) * w.Nq + (p - w.q_offset)) for p in range(p0, p1)]
+    oracle.attend(w, Q, K, V, full_idx, np.array(rows, dtype=np.int64))
+    t3 = time.perf_counter()
+    per_qb = ((t2 - t1) + (t3 - t2)) / len(qbs)
+    est = U * ((t1 - t0) + per_qb * nqb)
+    desc = (f"unit {unit} of {U}: pyramid + {len(qbs)} of {nqb} query blocks (evenly spaced; selection + "
+            f"attention of all their rows); whole-job time extrapolated x{U} units")
+    return t3 - t0, est, desc
+
+
+def cpu_baseline(w, budget_s=15.0):
+    Q, K, V, _ = synth.generate(w)
+    n = 4
+    took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V)
+    while took < budget_s * 0.4 and n < 4096:
+        n = min(4096, int(n * max(2.0, budget_s / max(took, 1e-3) * 0.5)))
+        took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(w.B * w.Nq / est, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": desc, "sample_seconds": round(took, 2)}
+
+
+def run_reference(args, w):
+    Q, K, V, _ = synth.generate(w)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    n_qb = 8
+    took, _, _ = oracle_sample(w, n_qb, Q=Q, K=K, V=V)
+    # size each step to ~4 s of host time so that the whole run ends within minutes
+    n_qb = max(1, min(4096, int(n_qb * 4.0 / max(took, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(w, max(1, n_qb // 4), Q=Q, K=K, V=V)
+    ests, tooks, desc = [], [], ""
+    for k in range(args.steps):
+        took, est, desc = oracle_sample(w, n_qb, seed=k, Q=Q, K=K, V=V)
+        ests.append(est)
+        tooks.append(took)
+    est = statistics.mean(ests)
+    value = w.B * w.Nq / est
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d,
+                       "b": w.b, "topk": w.topk, "cap": w.cap, "seed": w.seed},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": desc + f"; {args.steps} steps, mean sample {statistics.mean(tooks):.2f} s"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------- main --
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = synth.BY_NAME[args.workload]
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, w, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w)
+        elif rank == 0:
+            out["cpu_baseline"] = None
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

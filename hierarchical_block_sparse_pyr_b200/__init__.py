@@ -1,0 +1,185 @@
+"""Hierarchical (pyramid) top-K key-block selection + causal block-sparse attention on B200.
+
+Thin ctypes binding over ``lib/libpyr.so`` (the C ABI declared in
+``include/pyr.h``). Functions here only marshal arguments: torch tensors give
+device pointers and the current CUDA stream; every step of the computation
+runs in the library's sm_100a kernels. There is no CPU fallback: importing
+this package fails if the library is missing, and every call needs CUDA
+tensors.
+
+    pyr_build(shape, K, pyr)                  key pyramid (mean pooling)
+    pyr_select(shape, Q, pyr, idx, gap)       coarse-to-fine LogSumExp top-K
+    bsa_forward(shape, Q, K, V, idx, O, lse)  causal block-sparse attention
+    dense_forward(shape, Q, K, V, O, lse)     dense causal attention
+    forward(Q, K, V, b, topk, cap)            allocate outputs and run all three
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libpyr.so")
+
+PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = range(6)
+PYR_F32, PYR_BF16 = 0, 1
+
+ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_select", "bsa_forward",
+               "dense_forward", "pyr_strerror")
+
+
+class PyrShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "Hq", "Hkv", "N", "Nq", "q_offset", "d", "b", "topk", "cap",
+                                             "dtype")]
+
+    def __repr__(self):
+        return "PyrShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class PyrError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {strerror(code)} (status {code})")
+
+
+def _load_lib():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libpyr.so is missing at {LIB_PATH}; build it with `python -m hierarchical_block_sparse_pyr_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    sp = ctypes.POINTER(PyrShape)
+    vp = ctypes.c_void_p
+    lib.pyr_num_levels.argtypes = [sp]
+    lib.pyr_num_levels.restype = ctypes.c_int
+    lib.pyr_num_nodes.argtypes = [sp]
+    lib.pyr_num_nodes.restype = ctypes.c_int64
+    lib.pyr_num_qblocks.argtypes = [sp]
+    lib.pyr_num_qblocks.restype = ctypes.c_int64
+    lib.pyr_build.argtypes = [sp, vp, vp, vp, vp]
+    lib.pyr_build.restype = ctypes.c_int
+    lib.pyr_select.argtypes = [sp, vp, vp, vp, vp, vp, vp]
+    lib.pyr_select.restype = ctypes.c_int
+    lib.bsa_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.bsa_forward.restype = ctypes.c_int
+    lib.dense_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
+    lib.dense_forward.restype = ctypes.c_int
+    lib.pyr_strerror.argtypes = [ctypes.c_int]
+    lib.pyr_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load_lib()
+
+
+def strerror(code: int) -> str:
+    return _lib.pyr_strerror(code).decode()
+
+
+def make_shape(B, Hq, Hkv, N, Nq, q_offset, d, b, topk, cap, dtype) -> PyrShape:
+    if isinstance(dtype, torch.dtype):
+        dtype = {torch.float32: PYR_F32, torch.bfloat16: PYR_BF16}[dtype]
+    return PyrShape(B, Hq, Hkv, N, Nq, q_offset, d, b, topk, cap, dtype)
+
+
+def shape_of(w) -> PyrShape:
+    """PyrShape from any object with fields B, Hq, Hkv, N, Nq, q_offset, d, b, topk, cap, dtype."""
+    return make_shape(w.B, w.Hq, w.Hkv, w.N, w.Nq, w.q_offset, w.d, w.b, w.topk, w.cap, w.dtype)
+
+
+def num_levels(s: PyrShape) -> int:
+    return _lib.pyr_num_levels(ctypes.byref(s))
+
+
+def num_nodes(s: PyrShape) -> int:
+    return _lib.pyr_num_nodes(ctypes.byref(s))
+
+
+def num_qblocks(s: PyrShape) -> int:
+    return _lib.pyr_num_qblocks(ctypes.byref(s))
+
+
+def _dev(t, name, nullable=False):
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _check(rc, what):
+    if rc != PYR_OK:
+        raise PyrError(rc, what)
+
+
+def pyr_build(s: PyrShape, K, pyr, status=None, stream=None):
+    _check(_lib.pyr_build(ctypes.byref(s), _dev(K, "K"), _dev(pyr, "pyr"), _dev(status, "status", True),
+                          _stream(stream)), "pyr_build")
+
+
+def pyr_select(s: PyrShape, Q, pyr, idx, gap=None, status=None, stream=None):
+    _check(_lib.pyr_select(ctypes.byref(s), _dev(Q, "Q"), _dev(pyr, "pyr"), _dev(idx, "idx"),
+                           _dev(gap, "gap", True), _dev(status, "status", True), _stream(stream)), "pyr_select")
+
+
+def bsa_forward(s: PyrShape, Q, K, V, idx, O, lse=None, status=None, stream=None):
+    _check(_lib.bsa_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "idx"), _dev(O, "O"),
+                            _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)), "bsa_forward")
+
+
+def dense_forward(s: PyrShape, Q, K, V, O, lse=None, status=None, stream=None):
+    _check(_lib.dense_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(O, "O"),
+                              _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)),
+           "dense_forward")
+
+
+class Buffers:
+    """Device buffers of one forward pass (allocated by torch, owned by the caller)."""
+
+    def __init__(self, s: PyrShape, device="cuda"):
+        self.shape = s
+        nqb = num_qblocks(s)
+        dt = torch.float32 if s.dtype == PYR_F32 else torch.bfloat16
+        self.pyr = torch.empty((s.B, s.Hkv, num_nodes(s), s.d), dtype=torch.float32, device=device)
+        self.idx = torch.empty((s.B, s.Hkv, nqb, s.topk), dtype=torch.int32, device=device)
+        self.gap = torch.empty((s.B, s.Hkv, nqb), dtype=torch.float32, device=device)
+        self.O = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=dt, device=device)
+        self.lse = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def run(s: PyrShape, Q, K, V, buf: Buffers, stream=None, with_gap=True):
+    """Enqueue the whole path (pyramid, selection, attention) into buf."""
+    pyr_build(s, K, buf.pyr, buf.status, stream)
+    pyr_select(s, Q, buf.pyr, buf.idx, buf.gap if with_gap else None, buf.status, stream)
+    bsa_forward(s, Q, K, V, buf.idx, buf.O, buf.lse, buf.status, stream)
+    return buf
+
+
+def forward(Q, K, V, b: int, topk: int, cap: int, q_offset: int = 0):
+    """Allocate outputs and run pyramid + selection + block-sparse attention.
+
+    Q: [B, Hq, Nq, d]; K, V: [B, Hkv, N, d] CUDA tensors (fp32 or bf16).
+    Returns (O, lse, idx, gap); raises PyrError on a host-side error or on a
+    device-side status (read after synchronising the current stream).
+    """
+    B, Hq, Nq, d = Q.shape
+    N, Hkv = K.shape[2], K.shape[1]
+    s = make_shape(B, Hq, Hkv, N, Nq, q_offset, d, b, topk, cap, Q.dtype)
+    buf = run(s, Q, K, V, Buffers(s, Q.device))
+    torch.cuda.current_stream().synchronize()
+    code = int(buf.status.item())
+    if code:
+        raise PyrError(code, "device")
+    return buf.O, buf.lse, buf.idx, buf.gap

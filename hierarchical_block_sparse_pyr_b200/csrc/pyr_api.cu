@@ -1,0 +1,136 @@
+// C ABI of libpyr: argument validation, geometry, dispatch to the kernels.
+// Every entry point validates on the host, enqueues on the caller's stream
+// and returns; nothing here allocates device memory or synchronises.
+#include <stdint.h>
+
+#include "pyr_common.cuh"
+
+namespace pyr {
+size_t select_smem_bytes(const Geo& g);
+}
+
+using pyr::Geo;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Shape checks shared by every entry point. Returns PYR_OK and fills g.
+int make_geo(const pyr_shape* s, Geo* g) {
+  if (!s) return PYR_EINVAL;
+  if (s->B <= 0 || s->Hq <= 0 || s->Hkv <= 0 || s->Hq % s->Hkv || s->N <= 0 || s->Nq <= 0 || s->q_offset < 0 ||
+      (int64_t)s->q_offset + s->Nq > s->N || s->b <= 0 || s->d <= 0 || s->topk < 1 || s->cap < 2 || s->cap % 2 ||
+      s->topk > s->cap)
+    return PYR_EINVAL;
+  if (s->dtype != PYR_F32 && s->dtype != PYR_BF16) return PYR_EUNSUPPORTED;
+  if (s->d != 64 && s->d != 128) return PYR_EUNSUPPORTED;
+  if (s->b != 16 && s->b != 32 && s->b != 64 && s->b != 128) return PYR_EUNSUPPORTED;
+  if (s->cap > 128) return PYR_EUNSUPPORTED;
+  if (!(s->Nq == 1 || s->q_offset % s->b == 0)) return PYR_EUNSUPPORTED;
+  if ((int64_t)s->B * s->Hkv > 65535) return PYR_EUNSUPPORTED;
+  g->B = s->B;
+  g->Hq = s->Hq;
+  g->Hkv = s->Hkv;
+  g->G = s->Hq / s->Hkv;
+  g->N = s->N;
+  g->Nq = s->Nq;
+  g->q_offset = s->q_offset;
+  g->d = s->d;
+  g->b = s->b;
+  g->topk = s->topk;
+  g->cap = s->cap;
+  g->dtype = s->dtype;
+  g->nb = (int)(((int64_t)s->N + s->b - 1) / s->b);
+  int L = 0;
+  while (((int64_t)1 << L) < g->nb) L++;
+  if (L >= 31) return PYR_EUNSUPPORTED;
+  g->L = L;
+  int64_t off = 0;
+  for (int l = 0; l < 32; l++) {
+    g->lvl_n[l] = l <= L ? (int)((g->nb + ((int64_t)1 << l) - 1) >> l) : 0;
+    g->lvl_off[l] = (int)off;
+    off += g->lvl_n[l];
+  }
+  g->P = off;
+  g->i0 = s->q_offset / s->b;
+  g->nqb = (s->q_offset + s->Nq - 1) / s->b - g->i0 + 1;
+  int s0 = 0;
+  while (g->lvl_n[s0] > s->cap) s0++;
+  g->s0 = s0;
+  if (s0 >= 24) return PYR_EUNSUPPORTED;  // the selection kernel keeps partial means for 24 levels
+  if ((int64_t)g->G * (s->Nq < s->b ? s->Nq : s->b) > 1024) return PYR_EUNSUPPORTED;
+  return PYR_OK;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? PYR_OK : PYR_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int pyr_num_levels(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? g.L + 1 : 0;
+}
+
+int64_t pyr_num_nodes(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? g.P : 0;
+}
+
+int64_t pyr_num_qblocks(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? g.nqb : 0;
+}
+
+int pyr_build(const pyr_shape* s, const void* K, float* pyr, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!K || !pyr || !aligned16(K) || !aligned16(pyr)) return PYR_EINVAL;
+  return launch_status(pyr::launch_pyramid(g, K, pyr, dev_status, (cudaStream_t)stream));
+}
+
+int pyr_select(const pyr_shape* s, const void* Q, const float* pyr, int32_t* idx, float* gap, int* dev_status,
+               void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!Q || !pyr || !idx || !aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PYR_EINVAL;
+  if (pyr::select_smem_bytes(g) > 227 * 1024) return PYR_EUNSUPPORTED;
+  if (g.nqb > 2147483647) return PYR_EUNSUPPORTED;
+  return launch_status(pyr::launch_select(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
+}
+
+int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                float* lse, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return PYR_EINVAL;
+  return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
+}
+
+int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                  int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return PYR_EINVAL;
+  return launch_status(pyr::launch_attn_simt(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
+}
+
+const char* pyr_strerror(int code) {
+  switch (code) {
+    case PYR_OK: return "ok";
+    case PYR_EINVAL: return "invalid argument (null or misaligned pointer, or inconsistent shape)";
+    case PYR_EUNSUPPORTED: return "unsupported shape or dtype";
+    case PYR_ECUDA: return "CUDA launch failed";
+    case PYR_ETIMEOUT: return "a bounded device wait ran out";
+    case PYR_EBADIDX: return "idx lists a block that is not strictly before its query block, or not ascending";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Shared device helpers and the internal launch interface of libpyr.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pyr.h"
+
+namespace pyr {
+
+// Geometry derived from a validated pyr_shape.
+struct Geo {
+  int B, Hq, Hkv, G, N, Nq, q_offset, d, b, topk, cap, dtype;
+  int nb;       // key blocks
+  int L;        // top level (levels 0..L)
+  int nqb;      // query blocks per (batch, kv head)
+  int i0;       // first query block
+  int s0;       // first scored level: the finest with <= cap nodes
+  int64_t P;    // pyramid nodes per (batch, kv head)
+  int lvl_off[32];  // node offset of each level
+  int lvl_n[32];    // nodes of each level
+};
+
+inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
+
+// Device status word: the first error wins.
+__device__ __forceinline__ void report(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Launchers (one per kernel family). Each returns cudaSuccess or the launch error.
+cudaError_t launch_pyramid(const Geo& g, const void* K, float* pyr, int* status, cudaStream_t st);
+cudaError_t launch_select(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+                          cudaStream_t st);
+cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
+                             int dense, void* O, float* lse, int* status, cudaStream_t st);
+
+}  // namespace pyr

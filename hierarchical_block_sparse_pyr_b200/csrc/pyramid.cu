@@ -1,0 +1,227 @@
+// Key pyramid: level 0 = mean key of each block, level l = mean of the keys
+// under node (l, m) (PISA abstract: pooling builds the coarse-to-fine key
+// hierarchy; PHBA A.1.2: centroids average the block's key rows in fp32).
+//
+// HBM-bound: K is read exactly once with 16-byte loads and the pyramid
+// (about 2 nb d floats per head) is written once.
+//   pyr_chunk_kernel  one CTA per chunk of CB consecutive key blocks of one
+//                     (batch, kv head): one warp streams one block at a time
+//                     (lanes split the row into 16-byte vectors, the rest of
+//                     the warp splits rows), reduces with shuffles, and the
+//                     CTA then pools the chunk's subtree in shared memory.
+//   pyr_top_kernel    the levels above the chunk level, one CTA per
+//                     (unit, 16-element slice of d), entirely in shared memory.
+#include "pyr_common.cuh"
+
+namespace pyr {
+
+namespace {
+
+constexpr int kChunkThreads = 256;
+constexpr int kTopSlice = 16;
+constexpr int kTopThreads = 256;
+
+__device__ __forceinline__ int64_t tokens_in(int j0, int j1, int b, int N) {
+  int64_t t0 = (int64_t)j0 * b, t1 = (int64_t)j1 * b;
+  if (t1 > N) t1 = N;
+  return t1 > t0 ? t1 - t0 : 0;
+}
+
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ static void add(float* acc, uint4 v) {
+    acc[0] += __uint_as_float(v.x);
+    acc[1] += __uint_as_float(v.y);
+    acc[2] += __uint_as_float(v.z);
+    acc[3] += __uint_as_float(v.w);
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ static void add(float* acc, uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      acc[2 * k] += __uint_as_float(w[k] << 16);
+      acc[2 * k + 1] += __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// smem: two ping-pong level buffers of CB x D floats.
+template <typename T, int D>
+__global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __restrict__ K, float* __restrict__ pyr,
+                                                                  Geo g, int CB, int t_levels) {
+  constexpr int E = Vec<T>::E;
+  constexpr int VPR = D / E;        // 16-byte vectors per key row
+  constexpr int RLW = 32 / VPR;     // rows one warp instruction covers
+  static_assert(VPR <= 32 && 32 % VPR == 0, "row must fit a warp");
+  extern __shared__ float smem[];
+  float* cur = smem;
+  float* nxt = smem + (size_t)CB * D;
+
+  const int unit = blockIdx.y;
+  const int chunk = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = lane % VPR, rl = lane / VPR;
+  const int j_begin = chunk * CB;
+  const T* Ku = K + (size_t)unit * g.N * D;
+  float* pu = pyr + (size_t)unit * g.P * D;
+
+  // level 0: warp w handles blocks w, w + 8, ...
+  for (int jl = warp; jl < CB; jl += kChunkThreads / 32) {
+    const int j = j_begin + jl;
+    float acc[E];
+#pragma unroll
+    for (int k = 0; k < E; k++) acc[k] = 0.f;
+    int cnt = 0;
+    if (j < g.nb) {
+      const int t0 = j * g.b;
+      const int t1 = min(t0 + g.b, g.N);
+      cnt = t1 - t0;
+      const uint4* base = reinterpret_cast<const uint4*>(Ku + (size_t)t0 * D) + c;
+      int r = rl;
+      // 8 independent loads in flight per lane
+      for (; r + 7 * RLW < cnt; r += 8 * RLW) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; u++) v[u] = ldg_stream(base + (size_t)(r + u * RLW) * VPR);
+#pragma unroll
+        for (int u = 0; u < 8; u++) Vec<T>::add(acc, v[u]);
+      }
+      for (; r < cnt; r += RLW) Vec<T>::add(acc, ldg_stream(base + (size_t)r * VPR));
+    }
+#pragma unroll
+    for (int off = VPR; off < 32; off <<= 1)
+#pragma unroll
+      for (int k = 0; k < E; k++) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], off);
+    if (rl == 0) {
+      float* dst = cur + (size_t)jl * D + c * E;
+#pragma unroll
+      for (int k = 0; k < E; k++) dst[k] = acc[k];
+      if (j < g.nb) {
+        const float inv = 1.f / (float)cnt;
+        float4* o = reinterpret_cast<float4*>(pu + (size_t)j * D + c * E);
+#pragma unroll
+        for (int k = 0; k < E; k += 4) o[k / 4] = make_float4(acc[k] * inv, acc[k + 1] * inv, acc[k + 2] * inv,
+                                                              acc[k + 3] * inv);
+      }
+    }
+  }
+  __syncthreads();
+
+  // levels 1 .. t_levels inside the chunk
+  int n_loc = CB;
+  for (int l = 1; l <= t_levels; l++) {
+    n_loc >>= 1;
+    const int m0 = chunk * n_loc;
+    for (int x = threadIdx.x; x < n_loc * D; x += kChunkThreads) {
+      const int ml = x / D, e = x - ml * D;
+      const float s = cur[(size_t)(2 * ml) * D + e] + cur[(size_t)(2 * ml + 1) * D + e];
+      nxt[(size_t)ml * D + e] = s;
+      const int m = m0 + ml;
+      if (m < g.lvl_n[l]) {
+        const int j0 = m << l;
+        const int j1 = min((m + 1) << l, g.nb);
+        pu[(size_t)(g.lvl_off[l] + m) * D + e] = s / (float)tokens_in(j0, j1, g.b, g.N);
+      }
+    }
+    __syncthreads();
+    float* t = cur;
+    cur = nxt;
+    nxt = t;
+  }
+}
+
+// Levels t+1 .. L from level t, for one unit and a 16-wide slice of d.
+__global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(float* __restrict__ pyr, Geo g, int t) {
+  extern __shared__ float sm[];
+  const int unit = blockIdx.y;
+  const int e0 = blockIdx.x * kTopSlice;
+  float* pu = pyr + (size_t)unit * g.P * g.d;
+  const int nt = g.lvl_n[t];
+  float* cur = sm;
+  float* nxt = sm + (size_t)nt * kTopSlice;
+  // load level t as sums
+  for (int x = threadIdx.x; x < nt * kTopSlice; x += kTopThreads) {
+    const int m = x / kTopSlice, e = x - m * kTopSlice;
+    const int j0 = m << t, j1 = min((m + 1) << t, g.nb);
+    cur[x] = pu[(size_t)(g.lvl_off[t] + m) * g.d + e0 + e] * (float)tokens_in(j0, j1, g.b, g.N);
+  }
+  __syncthreads();
+  int n_prev = nt;
+  for (int l = t + 1; l <= g.L; l++) {
+    const int n = g.lvl_n[l];
+    for (int x = threadIdx.x; x < n * kTopSlice; x += kTopThreads) {
+      const int m = x / kTopSlice, e = x - m * kTopSlice;
+      float s = cur[(size_t)(2 * m) * kTopSlice + e];
+      if (2 * m + 1 < n_prev) s += cur[(size_t)(2 * m + 1) * kTopSlice + e];
+      nxt[x] = s;
+      const int j0 = m << l, j1 = min((m + 1) << l, g.nb);
+      pu[(size_t)(g.lvl_off[l] + m) * g.d + e0 + e] = s / (float)tokens_in(j0, j1, g.b, g.N);
+    }
+    __syncthreads();
+    float* tmp = cur;
+    cur = nxt;
+    nxt = tmp;
+    n_prev = n;
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_chunks(const Geo& g, const void* K, float* pyr, int CB, int t, cudaStream_t st) {
+  const size_t smem = (size_t)2 * CB * D * sizeof(float);
+  auto kern = pyr_chunk_kernel<T, D>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(ceil_div(g.nb, CB), g.B * g.Hkv);
+  kern<<<grid, kChunkThreads, smem, st>>>(reinterpret_cast<const T*>(K), pyr, g, CB, t);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_pyramid(const Geo& g, const void* K, float* pyr, int* status, cudaStream_t st) {
+  (void)status;
+  // Chunk: ~1024 key rows per CTA, and at most 1024 level-t nodes left for the top kernel.
+  int CB = 1;
+  while (CB * g.b < 1024) CB <<= 1;
+  while ((int64_t)CB * 1024 < g.nb) CB <<= 1;
+  int t = 0;
+  while ((1 << t) < CB) t++;
+  if (t > g.L) {  // the whole pyramid fits one chunk
+    t = g.L;
+    CB = 1 << t;
+  }
+  cudaError_t e;
+  if (g.dtype == PYR_BF16)
+    e = g.d == 128 ? launch_chunks<__nv_bfloat16, 128>(g, K, pyr, CB, t, st)
+                   : launch_chunks<__nv_bfloat16, 64>(g, K, pyr, CB, t, st);
+  else
+    e = g.d == 128 ? launch_chunks<float, 128>(g, K, pyr, CB, t, st) : launch_chunks<float, 64>(g, K, pyr, CB, t, st);
+  if (e != cudaSuccess || t >= g.L) return e;
+  const size_t smem = (size_t)2 * g.lvl_n[t] * kTopSlice * sizeof(float);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(pyr_top_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(g.d / kTopSlice, g.B * g.Hkv);
+  pyr_top_kernel<<<grid, kTopThreads, smem, st>>>(pyr, g, t);
+  return cudaGetLastError();
+}
+
+}  // namespace pyr

@@ -1,0 +1,173 @@
+/*
+ * pyr.h - C ABI of libpyr: hierarchical (pyramid) top-K key-block selection
+ * and causal block-sparse attention for NVIDIA B200 (sm_100a).
+ *
+ * The problem, as the pages state it: queries, keys and values go in; each
+ * query block gets a list of selected earlier key blocks; attention over
+ * those blocks plus the query's own block comes out, with its log-sum-exp.
+ *   - PISA abstract (peercurrent record): keys are pooled into a
+ *     coarse-to-fine hierarchy of O(log N) levels; selection starts at the
+ *     coarsest level and, level by level, applies LogSumExp scoring to a
+ *     bounded candidate set, passing the survivors' children to the next
+ *     finer level; the query-key score matrix is never materialised.
+ *   - PHBA summary (paperlayer.ai), A.1.2 "Routing metadata kernels": block
+ *     centroids average the block's key rows in fp32; routes go only to
+ *     strictly preceding blocks; unavailable route slots hold -1.
+ *   - PHBA summary, 3.1 "Top-K block routing" and A.1.3 "Query-tile fused
+ *     sparse forward kernel": the current block is always attended with local
+ *     causal attention; the forward pass keeps FlashAttention-style online
+ *     softmax accumulators and writes the output and the log-sum-exp.
+ *
+ * Conventions shared by every entry point
+ *   Layouts (row-major, contiguous, every base pointer 16-byte aligned):
+ *     Q, O  [B][Hq][Nq][d]     K, V  [B][Hkv][N][d]
+ *     pyr   [B][Hkv][P][d] fp32, level-major (level 0 first; node m of level
+ *           l covers key blocks [m 2^l, min((m+1) 2^l, nb)))
+ *     idx   [B][Hkv][nqb][topk] int32; gap [B][Hkv][nqb] fp32
+ *     lse   [B][Hq][Nq] fp32 (natural log)
+ *   Query row t sits at position q_offset + t. Key block j holds positions
+ *   [j b, min((j+1) b, N)); query block i holds the query rows whose
+ *   positions lie in [i b, (i+1) b). nb = ceil(N / b); nqb counts the query
+ *   blocks that hold at least one query row. Selection is shared by the
+ *   G = Hq / Hkv query heads of a kv head (grouped-query attention).
+ *   Supported: d in {64, 128}; b in {16, 32, 64, 128}; dtype PYR_F32 or
+ *   PYR_BF16 (Q, K, V and O share it); either decode (Nq == 1, any
+ *   q_offset < N) or block-aligned prefill (q_offset % b == 0 and
+ *   q_offset + Nq <= N); 1 <= topk <= cap <= 128, cap even; N % b may be
+ *   non-zero (a ragged last block).
+ *   Ownership: the caller allocates and owns every buffer; the library
+ *   allocates nothing, keeps no state between calls beyond cached kernel
+ *   attributes, and never frees caller memory.
+ *   Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *   default stream). Calls only enqueue work and return; results are ready
+ *   once the stream has been synchronised.
+ *   Errors: the return value is the host-side status (PYR_OK, PYR_EINVAL,
+ *   PYR_EUNSUPPORTED, PYR_ECUDA). Errors that only the device can see go to
+ *   *dev_status when dev_status is non-NULL: a kernel stores its code there
+ *   only if the word still holds PYR_OK, so the caller zeroes it before the
+ *   calls and reads it after synchronising. No entry point aborts, throws or
+ *   prints.
+ */
+#ifndef PYR_H
+#define PYR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols keep default visibility even when the library is built
+ * with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define PYR_API __attribute__((visibility("default")))
+#else
+#define PYR_API
+#endif
+
+#define PYR_OK 0
+#define PYR_EINVAL 1       /* a NULL or misaligned pointer, or an inconsistent shape */
+#define PYR_EUNSUPPORTED 2 /* a shape or dtype this build has no kernel for */
+#define PYR_ECUDA 3        /* the CUDA runtime refused a launch */
+#define PYR_ETIMEOUT 4     /* device: a bounded wait ran out (kernel returned early) */
+#define PYR_EBADIDX 5      /* device: idx held a block that is not strictly before its query block */
+
+#define PYR_F32 0
+#define PYR_BF16 1
+
+typedef struct pyr_shape {
+  int B;        /* batch */
+  int Hq;       /* query heads */
+  int Hkv;      /* key/value heads; Hq % Hkv == 0 */
+  int N;        /* key/value length */
+  int Nq;       /* query rows per head */
+  int q_offset; /* position of query row 0 */
+  int d;        /* head dimension */
+  int b;        /* block size: keys per key block, positions per query block */
+  int topk;     /* K: key blocks kept per query block (the diagonal block is extra) */
+  int cap;      /* candidate cap per pyramid level */
+  int dtype;    /* PYR_F32 or PYR_BF16 */
+} pyr_shape;
+
+/* Number of pyramid levels, L + 1 with L = ceil(log2 nb); 0 on a bad shape. */
+PYR_API int pyr_num_levels(const pyr_shape* s);
+
+/* Number of pyramid nodes per (batch, kv head), P = sum over levels of
+ * ceil(nb / 2^l); 0 on a bad shape. pyr holds B * Hkv * P * d floats. */
+PYR_API int64_t pyr_num_nodes(const pyr_shape* s);
+
+/* Query blocks per (batch, kv head), nqb; 0 on a bad shape. */
+PYR_API int64_t pyr_num_qblocks(const pyr_shape* s);
+
+/*
+ * pyr_build - the key pyramid (PISA abstract: pooling builds O(log N) levels;
+ * PHBA A.1.2: a centroid is the fp32 average of the block's key rows).
+ *   K   device, [B][Hkv][N][d] in s->dtype (read only).
+ *   pyr device, [B][Hkv][P][d] fp32 (written): node (l, m) is the mean of
+ *       all keys under it, level-major, level 0 first.
+ * Reads K once. Returns PYR_OK or a host-side error; nothing is written on
+ * error.
+ */
+PYR_API int pyr_build(const pyr_shape* s, const void* K, float* pyr, int* dev_status, void* stream);
+
+/*
+ * pyr_select - coarse-to-fine LogSumExp top-K key-block selection (PISA
+ * abstract; routes to strictly preceding blocks with -1 padding, PHBA A.1.2).
+ * For query block i of (batch, kv head), the node score is
+ *   S = ln sum_r exp(q_r . kbar / sqrt(d)) + ln n_valid,
+ * r running over every query row of block i in the G heads of the group;
+ * kbar and n_valid are the mean and token count of the node's part that lies
+ * before block i (nodes that start at or after block i are never scored).
+ * The walk starts at the finest level with at most `cap` nodes, with every
+ * valid node of that level as a candidate; each level above 0 keeps the best
+ * min(cap/2, #candidates) (ties to the lower node index) and passes their
+ * valid children on; level 0 keeps the best min(topk, #candidates).
+ *   Q   device, [B][Hq][Nq][d] in s->dtype.
+ *   pyr device, as written by pyr_build.
+ *   idx device, [B][Hkv][nqb][topk] int32 (written): the kept blocks in
+ *       ascending order, then -1. The query's own block is never listed.
+ *   gap device, [B][Hkv][nqb] fp32 or NULL (written): the smallest score
+ *       margin between the last kept and the first dropped candidate over
+ *       the scored levels (+inf if no level dropped one).
+ * Scoring accumulates in fp32.
+ */
+PYR_API int pyr_select(const pyr_shape* s, const void* Q, const float* pyr, int32_t* idx, float* gap, int* dev_status,
+               void* stream);
+
+/*
+ * bsa_forward - causal block-sparse attention (PHBA 3.1, 3.3 and A.1.3:
+ * routed blocks plus the current block, one online-softmax merge, output and
+ * log-sum-exp; the N x N score matrix is never formed).
+ * Row t (position p, query block i, kv head h = hq / G) attends to every key
+ * of the blocks idx[b][h][i - i0][*] (entries < 0 skipped) and to the keys of
+ * block i at positions <= p, with softmax scale 1/sqrt(d).
+ *   Q, K, V device, in s->dtype. idx device, as written by pyr_select: the
+ *           non-negative entries of a row must be strictly ascending and < i;
+ *           an entry that breaks this is skipped and PYR_EBADIDX is reported
+ *           in *dev_status (the -1 entries may appear anywhere).
+ *   O   device, [B][Hq][Nq][d] in s->dtype (written).
+ *   lse device, [B][Hq][Nq] fp32 or NULL (written).
+ * bf16 inputs run on the tcgen05 tensor cores (bf16 operands, fp32
+ * accumulation in tensor memory); fp32 inputs run in fp32 on the CUDA cores.
+ */
+PYR_API int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, void* O,
+                float* lse, int* dev_status, void* stream);
+
+/*
+ * dense_forward - plain causal attention over every key at position <= p
+ * (the FlashAttention-style consumer the PHAROS and PHBA pages compare
+ * against), for finding the context length at which selection pays off.
+ * Arguments as bsa_forward without idx; s->topk and s->cap are ignored.
+ */
+PYR_API int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                  int* dev_status, void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+PYR_API const char* pyr_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PYR_H */

@@ -1,0 +1,99 @@
+"""The C ABI: the library loads, exports every declared symbol, validates on the host.
+
+Nothing here launches a kernel: every call below returns from host-side
+validation before the CUDA runtime is touched, so it runs without a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"PYR_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    declared = _declared()
+    assert {"pyr_build", "pyr_select", "bsa_forward", "dense_forward", "pyr_strerror"} <= declared
+    lib = ctypes.CDLL(P.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(P.ABI_SYMBOLS) <= declared
+
+
+def test_geometry_matches_the_oracle():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    for w in synth.WORKLOADS + [synth.WORKLOADS[0].scaled(N=4000, Nq=4000), synth.WORKLOADS[1].scaled(N=100, Nq=1,
+                                                                                                       q_offset=99)]:
+        s = P.shape_of(w)
+        assert P.num_levels(s) == oracle.num_levels(w)
+        assert P.num_nodes(s) == oracle.num_nodes(w)
+        assert P.num_qblocks(s) == oracle.num_qblocks(w)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("Hq", 3, 1),          # Hq % Hkv != 0 with Hkv = 2
+    ("N", 0, 1),
+    ("topk", 0, 1),
+    ("cap", 7, 1),         # odd cap
+    ("topk", 40, 1),       # topk > cap
+    ("d", 96, 2),
+    ("b", 48, 2),
+    ("dtype", 5, 2),
+    ("q_offset", 10, 2),   # a prefill chunk that does not start on a block boundary
+])
+def test_host_validation_rejects_bad_shapes(field, value, code):
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    w = synth.WORKLOADS[0]
+    s = P.shape_of(w)
+    s.Hkv = 2
+    s.Nq = 1024
+    setattr(s, field, value)
+    lib = P._lib
+    rc = lib.pyr_build(ctypes.byref(s), 16, 16, None, None)
+    assert rc == code, P.strerror(rc)
+    rc = lib.pyr_select(ctypes.byref(s), 16, 16, 16, None, None, None)
+    assert rc == code
+
+
+def test_host_validation_rejects_null_and_misaligned_pointers():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    s = P.shape_of(synth.WORKLOADS[1])
+    lib = P._lib
+    assert lib.pyr_build(ctypes.byref(s), None, 16, None, None) == P.PYR_EINVAL
+    assert lib.pyr_build(ctypes.byref(s), 24, 16, None, None) == P.PYR_EINVAL
+    assert lib.pyr_select(ctypes.byref(s), 16, 16, None, None, None, None) == P.PYR_EINVAL
+    assert lib.bsa_forward(ctypes.byref(s), 16, 16, 16, None, 16, None, None, None) == P.PYR_EINVAL
+    assert lib.dense_forward(ctypes.byref(s), 16, 16, 16, 8, None, None, None) == P.PYR_EINVAL
+    assert lib.pyr_build(None, 16, 16, None, None) == P.PYR_EINVAL
+    for code in range(6):
+        assert isinstance(P.strerror(code), str) and P.strerror(code)
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    w = synth.WORKLOADS[0].scaled(N=256, Nq=256)
+    s = P.shape_of(w)
+    K = torch.zeros((1, 2, 256, 64))
+    with pytest.raises(TypeError):
+        P.pyr_build(s, K, torch.zeros((1, 2, P.num_nodes(s), 64)))
