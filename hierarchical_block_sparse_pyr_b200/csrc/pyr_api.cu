@@ -109,6 +109,8 @@ int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V,
   if (rc) return rc;
   if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
     return PYR_EINVAL;
+  if (pyr::attn_tc_supported(g))
+    return launch_status(pyr::launch_attn_tc(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
 }
 
@@ -118,6 +120,8 @@ int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* 
   int rc = make_geo(s, &g);
   if (rc) return rc;
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return PYR_EINVAL;
+  if (pyr::attn_tc_supported(g))
+    return launch_status(pyr::launch_attn_tc(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
 }
 

@@ -36,6 +36,10 @@ CASES = [
               dtype=BF16, seed=19, n_needle=0),
     W0.scaled(name="chunked_prefill", B=1, Hq=4, Hkv=2, N=2048, Nq=1024, q_offset=1024, d=128, b=64, topk=4, cap=8,
               dtype=BF16, seed=20),
+    W0.scaled(name="mha_bf16_odd_qblocks", B=1, Hq=2, Hkv=2, N=2100, Nq=2100, d=128, b=64, topk=5, cap=10,
+              dtype=BF16, seed=25),
+    W0.scaled(name="gqa2_bf16_b128", B=1, Hq=4, Hkv=2, N=3000, Nq=3000, d=128, b=128, topk=4, cap=8, dtype=BF16,
+              seed=26, needle_mode=synth.NEEDLE_LOGUNIFORM),
     W0.scaled(name="cap_covers_all", B=1, Hq=2, Hkv=2, N=1024, Nq=1024, d=64, b=64, topk=4, cap=16, dtype=F32,
               seed=21),
 ]
@@ -123,6 +127,22 @@ def test_bad_idx_is_reported_and_skipped():
     ok[0, 0, 5] = [1, -1]
     O_o, _ = oracle.attend(w, Q, K, V, ok, np.arange(512))
     assert np.abs(g["O"].double().numpy().reshape(-1, 64) - O_o).max() <= 1e-4
+
+
+def test_bad_idx_is_reported_and_skipped_on_the_tensor_core_path():
+    w = W0.scaled(name="bad_idx_tc", B=1, Hq=2, Hkv=1, N=640, Nq=640, d=128, b=64, topk=3, cap=6, dtype=BF16,
+                  seed=27)
+    Q, K, V, _ = synth.generate(w)
+    idx = -np.ones((1, 1, 10, 3), dtype=np.int32)
+    idx[0, 0, 6] = [4, 2, 5]  # 2 breaks the ascending order
+    idx[0, 0, 7] = [1, 7, -1]  # 7 is the diagonal block, not an earlier one
+    g = run_gpu(w, Q, K, V, idx=idx)
+    assert g["status"] == 5
+    ok = idx.copy()
+    ok[0, 0, 6] = [4, 5, -1]
+    ok[0, 0, 7] = [1, -1, -1]
+    O_o, lse_o = oracle.attend(w, Q, K, V, ok, np.arange(2 * 640))
+    check_out(w, g["O"].double().numpy().reshape(-1, 128), g["lse"].double().numpy().reshape(-1), O_o, lse_o)
 
 
 def test_future_keys_do_not_change_selection_or_output():
