@@ -97,8 +97,9 @@ int pyr_select(const pyr_shape* s, const void* Q, const float* pyr, int32_t* idx
   int rc = make_geo(s, &g);
   if (rc) return rc;
   if (!Q || !pyr || !idx || !aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PYR_EINVAL;
+  if (pyr::select_tc_supported(g))
+    return launch_status(pyr::launch_select_tc(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
   if (pyr::select_smem_bytes(g) > 227 * 1024) return PYR_EUNSUPPORTED;
-  if (g.nqb > 2147483647) return PYR_EUNSUPPORTED;
   return launch_status(pyr::launch_select(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
 }
 

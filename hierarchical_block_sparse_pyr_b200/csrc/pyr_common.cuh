@@ -48,6 +48,9 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 cudaError_t launch_pyramid(const Geo& g, const void* K, float* pyr, int* status, cudaStream_t st);
 cudaError_t launch_select(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
                           cudaStream_t st);
+bool select_tc_supported(const Geo& g);
+cudaError_t launch_select_tc(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+                             cudaStream_t st);
 bool attn_tc_supported(const Geo& g);
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
                            void* O, float* lse, int* status, cudaStream_t st);
