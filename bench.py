@@ -129,13 +129,19 @@ def src_hash(files):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"pyramid": ["pyramid.cu"], "select": ["select.cu"], "attention": ["attn_tc.cu", "tc_util.cuh"]}
+KERNEL_SOURCES = {"pyramid": ["pyramid.cu"], "select": ["select_tc.cu", "tc_util.cuh"], "attention": ["attn_tc.cu", "tc_util.cuh"]}
 
 
 def tc_attention(w):
     """True when bsa_forward takes the tcgen05 kernel for this workload (bf16, d=128, b in {64,128},
     G*b in {64,128,256}, not decode)."""
     return (w.dtype == synth.BF16 and w.d == 128 and w.b in (64, 128) and w.Nq > 1
+            and w.G * w.b in (64, 128, 256))
+
+
+def tc_select(w):
+    """True when pyr_select scores on the tensor cores (bf16, d=128, prefill, G*b in {64,128,256})."""
+    return (w.dtype == synth.BF16 and w.d == 128 and w.Nq > 1 and w.b % 64 == 0
             and w.G * w.b in (64, 128, 256))
 
 
@@ -332,10 +338,12 @@ def run_ours(args, w, rank, world, local_rank):
         "pyramid": dict(ms=avg["pyramid"], bound="hbm", achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9,
                         peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["pyr_bytes"],
                         traffic=measured_traffic("pyramid", w.name)),
-        "select": dict(ms=avg["select"], bound="alu",
+        "select": dict(ms=avg["select"], bound="tensor" if tc_select(w) else "alu",
                        achieved=wc["sel_flops"] / (avg["select"] * 1e-3) / 1e12,
-                       peak=148 * 128 * 2 * sm_clock * 1e6 / 1e12, unit="TFLOP/s", algorithmic=wc["sel_flops"],
+                       peak=(peaks["bf16_tflops_sustained"] if tc_select(w) else
+                             148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s", algorithmic=wc["sel_flops"],
                        hbm_gbs=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9,
+                       hbm_frac=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
                        traffic=measured_traffic("select", w.name)),
         "attention": dict(ms=avg["attention"], bound="tensor" if tc_attention(w) else "alu",
                           achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
@@ -459,9 +467,15 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n", type=int, default=None,
+                    help="shrink the context length (and query rows) of the workload: for profiling the same "
+                         "kernels on a smaller case; the default JSON line always uses the full workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = synth.BY_NAME[args.workload]
+    if args.n:
+        w = w.scaled(name=f"{w.name}@N={args.n}", N=args.n, Nq=1 if w.decode else args.n,
+                     q_offset=args.n - 1 if w.decode else 0)
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -14,9 +14,12 @@
 //                       lazily rescaled online softmax; P (bf16) is written
 //                       back into tensor memory over the S tile it came from;
 //                       epilogue;
-//   warp 4*MT           TMA producer: Q once, then K and V tiles of 64 keys;
+//   warp 4*MT           TMA producer of Q (once) and of the K tiles (64 keys);
 //   warp 4*MT+1         MMA issuer: S = Q K^T into TMEM (two S buffers),
-//                       O += P V with P read from TMEM, V from shared memory.
+//                       O += P V with P read from TMEM, V from shared memory;
+//   warp 4*MT+2         TMA producer of the V tiles.
+// K and V have separate rings: a K tile is released as soon as its QK MMA has
+// finished, so the next K loads run one tile ahead of the late PV use of V.
 // tcgen05 MMAs of one thread execute in issue order and a commit covers every
 // earlier MMA, so S buffer reuse needs no extra barrier: QK of tile t+2 is
 // issued after PV of tile t, and the softmax of tile t+2 starts only once the
@@ -44,14 +47,15 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 template <int MT, int NS>
 struct Plan {
   static constexpr int kQ = 0;                         // MT x [2 halves][128 rows][128 B]
-  static constexpr int kKV = kQ + MT * 32768;          // NS x (K [2][64][128 B], V [2][64][128 B])
-  static constexpr int kBar = kKV + NS * 32768;        // mbarriers
-  static constexpr int kNumBars = 1 + 2 * NS + 2 + 2 + 2;
+  static constexpr int kKV = kQ + MT * 32768;          // K ring: NS x [2][64][128 B], then V ring
+  static constexpr int kV = kKV + NS * 16384;
+  static constexpr int kBar = kV + NS * 16384;         // mbarriers
+  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;    // tmem slot, abort flag, tile count
   static constexpr int kTiles = kMisc + 16;            // tile entries: (block << 4) | modes
   static constexpr int kEnd = kTiles + kMaxTiles * 4;
   static constexpr int kBytes = kEnd + 1024;           // + alignment slack
-  static constexpr int kThreads = (4 * MT + 2) * 32;
+  static constexpr int kThreads = (4 * MT + 3) * 32;
   static constexpr int kTmemCols = MT == 1 ? 256 : 512;
   static constexpr int kMinBlocks = kBytes <= 113 * 1024 ? 2 : 1;
 };
@@ -80,9 +84,11 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
   uint64_t* bar_q = bars;
-  uint64_t* bar_kv_full = bars + 1;
-  uint64_t* bar_kv_free = bar_kv_full + NS;
-  uint64_t* bar_s_full = bar_kv_free + NS;  // [2]
+  uint64_t* bar_k_full = bars + 1;
+  uint64_t* bar_k_free = bar_k_full + NS;
+  uint64_t* bar_v_full = bar_k_free + NS;
+  uint64_t* bar_v_free = bar_v_full + NS;
+  uint64_t* bar_s_full = bar_v_free + NS;   // [2]
   uint64_t* bar_p_full = bar_s_full + 2;    // [2]
   uint64_t* bar_o = bar_p_full + 2;
   uint64_t* bar_drain = bar_o + 1;
@@ -101,7 +107,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   // ---- setup: barriers; the routed blocks of the tile's query blocks ----
   // The raw idx rows are staged in the K/V area, which no copy touches before
   // the tile list is built.
-  int* s_idx = reinterpret_cast<int*>(smem + PL::kKV);
+  int* s_idx = reinterpret_cast<int*>(smem + PL::kKV);  // the K ring, before any copy
   if (!dense) {
     for (int x = threadIdx.x; x < QB * g.topk; x += PL::kThreads) {
       const int q = x / g.topk, k = x - q * g.topk;
@@ -111,8 +117,10 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; s++) {
-      mbar_init(bar_kv_full + s, 1);
-      mbar_init(bar_kv_free + s, 1);
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_k_free + s, 1);
+      mbar_init(bar_v_full + s, 1);
+      mbar_init(bar_v_free + s, 1);
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(bar_s_full + b, 1);
@@ -206,41 +214,46 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   };
 
   unsigned char* sQ = smem + PL::kQ;
-  unsigned char* sKV = smem + PL::kKV;
+  unsigned char* sK = smem + PL::kKV;
+  unsigned char* sV = smem + PL::kV;
 
-  if (warp == softmax_warps) {
-    // ------------------------------------------------------------ producer
+  if (warp == softmax_warps || warp == softmax_warps + 2) {
+    // ------------------------------------------------------------ producers (K + Q, V)
+    const bool is_k = (warp == softmax_warps);
     if (lane == 0) {
       bool ok = true;
-      mbar_expect_tx(bar_q, MT * 32768);
-      for (int mt = 0; mt < MT; mt++)
-        for (int c = 0; c < 2; c++) {
-          const int r0 = mt * 128 + c * 64;
-          const int qsub = r0 / (g.G * g.b), within = r0 % (g.G * g.b);
-          const int gq = within / g.b, off = within % g.b;
-          const int row = (i_first + qsub) * g.b + off - g.q_offset;
-          const int head = bi * g.Hq + hk * g.G + gq;
-          for (int h = 0; h < 2; h++)
-            tma_load_3d(sQ + mt * 32768 + h * 16384 + c * 8192, &tmQ, h * 64, row, head, bar_q);
-        }
+      if (is_k) {
+        mbar_expect_tx(bar_q, MT * 32768);
+        for (int mt = 0; mt < MT; mt++)
+          for (int c = 0; c < 2; c++) {
+            const int r0 = mt * 128 + c * 64;
+            const int qsub = r0 / (g.G * g.b), within = r0 % (g.G * g.b);
+            const int gq = within / g.b, off = within % g.b;
+            const int row = (i_first + qsub) * g.b + off - g.q_offset;
+            const int head = bi * g.Hq + hk * g.G + gq;
+            for (int h = 0; h < 2; h++)
+              tma_load_3d(sQ + mt * 32768 + h * 16384 + c * 8192, &tmQ, h * 64, row, head, bar_q);
+          }
+      }
+      uint64_t* full = is_k ? bar_k_full : bar_v_full;
+      uint64_t* fre = is_k ? bar_k_free : bar_v_free;
+      unsigned char* ring = is_k ? sK : sV;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
       int t = 0;
       for (; t < T && ok; t++) {
         const int s = t % NS, k = t / NS;
-        if (k > 0) ok = mbar_wait(bar_kv_free + s, (k - 1) & 1, abort_flag);
+        if (k > 0) ok = mbar_wait(fre + s, (k - 1) & 1, abort_flag);
         if (!ok) break;
         int key0, mode;
         tile_info(t, &key0, &mode);
-        unsigned char* st = sKV + s * 32768;
-        mbar_expect_tx(bar_kv_full + s, 32768);
-        for (int h = 0; h < 2; h++) {
-          tma_load_3d(st + h * 8192, &tmK, h * 64, key0, unit, bar_kv_full + s);
-          tma_load_3d(st + 16384 + h * 8192, &tmV, h * 64, key0, unit, bar_kv_full + s);
-        }
+        unsigned char* st = ring + s * 16384;
+        mbar_expect_tx(full + s, 16384);
+        for (int h = 0; h < 2; h++) tma_load_3d(st + h * 8192, map, h * 64, key0, unit, full + s);
       }
       // drain: wait (bounded) for every copy issued so far before the CTA may exit
       volatile int no_abort = 0;
-      mbar_wait(bar_q, 0, &no_abort);
-      for (int u = max(0, t - NS); u < t; u++) mbar_wait(bar_kv_full + (u % NS), (u / NS) & 1, &no_abort);
+      if (is_k) mbar_wait(bar_q, 0, &no_abort);
+      for (int u = max(0, t - NS); u < t; u++) mbar_wait(full + (u % NS), (u / NS) & 1, &no_abort);
     }
     __syncwarp();
   } else if (warp == softmax_warps + 1) {
@@ -248,35 +261,37 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kKeys, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       int issued = 0;
       for (int t = 0; t <= T && ok; t++) {
         if (t < T) {
           const int s = t % NS, sb = t & 1;
-          ok = mbar_wait(bar_kv_full + s, (t / NS) & 1, abort_flag);
+          ok = mbar_wait(bar_k_full + s, (t / NS) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           for (int mt = 0; mt < MT; mt++)
             for (int kk = 0; kk < 8; kk++) {
               const uint64_t a = sdesc_sw128(aQ + mt * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-              const uint64_t b = sdesc_sw128(aKV + s * 32768 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+              const uint64_t b = sdesc_sw128(aK + s * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
               umma_bf16(tS + (mt * 2 + sb) * 64, a, b, idesc_qk, kk > 0);
             }
           umma_commit(bar_s_full + sb);
+          umma_commit(bar_k_free + s);
           issued++;
         }
         if (t >= 1) {
           const int u = t - 1, s = u % NS, pb = u & 1;
           ok = mbar_wait(bar_p_full + pb, (u >> 1) & 1, abort_flag);
+          if (ok) ok = mbar_wait(bar_v_full + s, (u / NS) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           for (int mt = 0; mt < MT; mt++)
             for (int kk = 0; kk < 4; kk++) {
-              const uint64_t b = sdesc_sw128(aKV + s * 32768 + 16384 + kk * 2048, 8192, 1024);
+              const uint64_t b = sdesc_sw128(aV + s * 16384 + kk * 2048, 8192, 1024);
               umma_bf16_ts(tO + mt * 128, tS + (mt * 2 + pb) * 64 + kk * 8, b, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
             }
-          umma_commit(bar_kv_free + s);
+          umma_commit(bar_v_free + s);
           umma_commit(bar_o);
           issued++;
         }
@@ -319,13 +334,24 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
       const int md = row_ok ? (mode >> (2 * qsub)) & 3 : 0;
       // valid keys: full -> every key < N; causal -> keys <= p
       const int lim = md == 0 ? 0 : (md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1));
-      float mx = -INFINITY;
+      if (lim < kKeys) {
 #pragma unroll
-      for (int c = 0; c < kKeys; c++) {
-        s[c] = c < lim ? s[c] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kKeys; c++) s[c] = c < lim ? s[c] : -INFINITY;
       }
-      const float m_new = fmaxf(m_ref, mx);
+      // row max of the raw scores (the positive scale commutes with max): 3-input tree
+      float mx;
+      {
+        float a[22];
+#pragma unroll
+        for (int k = 0; k < 21; k++) a[k] = fmax3(s[3 * k], s[3 * k + 1], s[3 * k + 2]);
+        a[21] = s[63];
+        float b2[8];
+#pragma unroll
+        for (int k = 0; k < 7; k++) b2[k] = fmax3(a[3 * k], a[3 * k + 1], a[3 * k + 2]);
+        b2[7] = a[21];
+        mx = fmax3(fmax3(b2[0], b2[1], b2[2]), fmax3(b2[3], b2[4], b2[5]), fmaxf(b2[6], b2[7]));
+      }
+      const float m_new = fmaxf(m_ref, mx * sl2);
       const bool need = (m_ref != -INFINITY) && (m_new > m_ref + kRescale);
       float factor = 1.f;
       if (need) {
@@ -351,15 +377,28 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
         }
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // p = 2^(s * sl2 - m): packed FMA, three quarters of the exponentials on
+      // the MUFU unit and one quarter on the FMA pipe; four packed partial sums
       uint32_t pk[32];
-      float part = 0.f;
+      const float2 scl = make_float2(sl2, sl2), off = make_float2(-m_use, -m_use);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
       for (int c = 0; c < 32; c++) {
-        const float e0 = ex2(s[2 * c] - m_use), e1 = ex2(s[2 * c + 1] - m_use);
-        part += e0 + e1;
-        pk[c] = pack_bf16(e0, e1);
+        const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), scl, off);
+        float2 e;
+        if ((c & 3) == 3) {
+          e.x = ex2_poly(x.x);
+          e.y = ex2_poly(x.y);
+        } else {
+          e.x = ex2(x.x);
+          e.y = ex2(x.y);
+        }
+        acc[c & 3] = __fadd2_rn(acc[c & 3], e);
+        pk[c] = pack_bf16(e.x, e.y);
       }
-      l_sum += part;
+      const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 sall = __fadd2_rn(s01, s23);
+      l_sum += sall.x + sall.y;
       tmem_st32u(tS_row + sb * 64, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -440,10 +479,10 @@ cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const voi
   if (g.b == 64) {
     if (rows == 64) return launch_cfg<1, 2, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
     if (rows == 128) return launch_cfg<1, 1, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
-    return launch_cfg<2, 1, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
+    return launch_cfg<2, 1, 64, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st);
   }
   if (rows == 128) return launch_cfg<1, 1, 128, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
-  return launch_cfg<2, 1, 128, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
+  return launch_cfg<2, 1, 128, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st);
 }
 
 namespace tc {

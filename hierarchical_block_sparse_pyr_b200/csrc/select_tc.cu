@@ -66,7 +66,7 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
 }
 
 template <int MC>
-__global__ void __launch_bounds__(kThreads) select_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                              const float* __restrict__ pyr, int32_t* __restrict__ idx,
                                                              float* __restrict__ gap_out, int* status, Geo g) {
   extern __shared__ unsigned char smem_raw[];
@@ -151,23 +151,38 @@ __global__ void __launch_bounds__(kThreads) select_tc_kernel(const __grid_consta
   for (int l = g.s0; l >= 0 && ok; l--) {
     const int nc = *s_nc;
     const bool start = (l == g.s0);
-    // ---- gather: warp w handles candidate rows w, w+4, ...; lane holds 4 of the 128 d-elements
-    for (int c = warp; c < nc; c += 4) {
-      const int m = start ? c : cand[c];
-      const bool straddle = l > 0 && ((m + 1) << l) > i;
-      const float4 v = straddle ? *reinterpret_cast<const float4*>(part + l * 128 + lane * 4)
-                                : __ldg(reinterpret_cast<const float4*>(pu + (size_t)(g.lvl_off[l] + m) * 128) + lane);
-      const float x[4] = {v.x, v.y, v.z, v.w};
-      float hi[4], lo[4];
+    // ---- gather: warp w handles candidate rows w, w+4, ...; lane holds 4 of the 128 d-elements.
+    // Rows are fetched 8 at a time so that their loads are in flight together.
+    const int nrow = nc > warp ? (nc - warp + 3) / 4 : 0;
+    for (int k0 = 0; k0 < nrow; k0 += 8) {
+      float4 v[8];
 #pragma unroll
-      for (int k = 0; k < 4; k++) {
-        hi[k] = __bfloat162float(__float2bfloat16_rn(x[k]));
-        lo[k] = x[k] - hi[k];
+      for (int k = 0; k < 8; k++) {
+        if (k0 + k < nrow) {
+          const int c = warp + 4 * (k0 + k);
+          const int m = start ? c : cand[c];
+          const bool straddle = l > 0 && ((m + 1) << l) > i;
+          v[k] = straddle ? *reinterpret_cast<const float4*>(part + l * 128 + lane * 4)
+                          : __ldg(reinterpret_cast<const float4*>(pu + (size_t)(g.lvl_off[l] + m) * 128) + lane);
+        }
       }
-      const int h = lane >> 4, c8 = (lane & 15) >> 1, half8 = (lane & 1) * 8;
-      const int off = h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4) + half8;
-      *reinterpret_cast<uint2*>(sAh + off) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
-      *reinterpret_cast<uint2*>(sAl + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+#pragma unroll
+      for (int k = 0; k < 8; k++) {
+        if (k0 + k < nrow) {
+          const int c = warp + 4 * (k0 + k);
+          const float x[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+          float hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            hi[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+            lo[e] = x[e] - hi[e];
+          }
+          const int h = lane >> 4, c8 = (lane & 15) >> 1, half8 = (lane & 1) * 8;
+          const int off = h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4) + half8;
+          *reinterpret_cast<uint2*>(sAh + off) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
+          *reinterpret_cast<uint2*>(sAl + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+        }
+      }
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -189,29 +204,47 @@ __global__ void __launch_bounds__(kThreads) select_tc_kernel(const __grid_consta
     nphase++;
     if (!ok) break;
     tc_fence_after();
-    // ---- LogSumExp over the valid query rows, one candidate per thread
+    // ---- LogSumExp over the valid query rows, one candidate per thread: pass 1 takes the
+    // max of the raw dot products (the positive scale commutes with max), pass 2 re-reads
+    // TMEM and sums 2^(x * scale - max) with packed FMAs and four independent partial sums.
     float m2 = -INFINITY, s2 = 0.f;
     const bool warp_has = MC == 128 ? (warp * 32 < nc) : (warp * 16 < nc);
     if (warp_has) {
+      const bool full = (rb == g.b);
       float v[32];
+      float mx = -INFINITY;
       for (int c0 = 0; c0 < R; c0 += 32) {
         tmem_ld32(my_lane_addr + c0, v);
         tmem_wait_ld();
-        float cm = -INFINITY;
+        if (!full) {
 #pragma unroll
-        for (int k = 0; k < 32; k++) {
-          const int r = c0 + k;
-          const bool valid = (r % g.b) < rb;  // column r = head * b + offset
-          v[k] = valid ? v[k] * sl2 : -INFINITY;
-          cm = fmaxf(cm, v[k]);
+          for (int k = 0; k < 32; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
         }
-        if (cm > m2) {
-          s2 = (m2 == -INFINITY) ? 0.f : s2 * ex2(m2 - cm);
-          m2 = cm;
-        }
+        float a[11];
 #pragma unroll
-        for (int k = 0; k < 32; k++) s2 += ex2(v[k] - m2);
+        for (int k = 0; k < 10; k++) a[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+        a[10] = fmaxf(v[30], v[31]);
+        mx = fmax3(mx, fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], a[8])),
+                   fmaxf(a[9], a[10]));
       }
+      m2 = mx * sl2;
+      const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      for (int c0 = 0; c0 < R; c0 += 32) {
+        tmem_ld32(my_lane_addr + c0, v);
+        tmem_wait_ld();
+        if (!full) {
+#pragma unroll
+          for (int k = 0; k < 32; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
+        }
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+          const float2 x = __ffma2_rn(make_float2(v[2 * k], v[2 * k + 1]), scl, off);
+          acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(ex2(x.x), ex2(x.y)));
+        }
+      }
+      const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+      s2 = t.x + t.y;
     }
     tc_fence_before();
     if (my_c >= 0 && my_c < nc) {
