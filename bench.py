@@ -76,6 +76,7 @@ def work_counts(w):
     # selection: candidates scored per level (upper bound per level: all valid nodes at s0, then <= cap)
     sel_flops = 0
     sel_exps = 0
+    sel_nodes = 0  # candidate node rows read, summed over query blocks
     att_pairs = 0
     for qb in range(nqb):
         i = first + qb
@@ -85,6 +86,7 @@ def work_counts(w):
         for l in range(s0, -1, -1):
             sel_flops += 2 * rows * nc * w.d
             sel_exps += rows * nc
+            sel_nodes += nc
             keep = min(w.cap // 2 if l > 0 else w.topk, nc)
             if l > 0:
                 # children of the kept nodes that start before i (at most 2 per kept node)
@@ -97,9 +99,13 @@ def work_counts(w):
     sel_exps *= U
     att_pairs *= U
     att_flops = 4 * w.d * att_pairs
-    pyr_bytes = U * (w.N * w.d * elt + P * w.d * 4)
+    if w.decode:
+        # one decode step: re-pool the last block and its ancestors (one node per level)
+        pyr_bytes = U * (min(w.b, w.N) * w.d * elt + len(lv) * w.d * 4)
+    else:
+        pyr_bytes = U * (w.N * w.d * elt + P * w.d * 4)
     q_bytes = w.B * w.Hq * w.Nq * w.d * elt
-    sel_bytes = q_bytes + U * P * w.d * 4 + U * nqb * w.topk * 4
+    sel_bytes = q_bytes + U * sel_nodes * w.d * 4 + U * nqb * w.topk * 4
     # attention: Q + O once; K, V of the selected + diagonal blocks once per query block and kv head
     kv_blocks = 0
     for qb in range(nqb):
@@ -129,7 +135,15 @@ def src_hash(files):
     return h.hexdigest()[:16]
 
 
-KERNEL_SOURCES = {"pyramid": ["pyramid.cu"], "select": ["select_tc.cu", "tc_util.cuh"], "attention": ["attn_tc.cu", "tc_util.cuh"]}
+def kernel_source(kernel, w):
+    """The .cu file whose code runs as `kernel` for workload w (its hash keys the ncu traffic record)."""
+    if kernel == "pyramid":
+        return "pyramid.cu"
+    if kernel == "select":
+        return "select_tc.cu" if tc_select(w) else "select.cu"
+    if w.decode:
+        return "attn_decode.cu"
+    return "attn_tc.cu" if tc_attention(w) else "attn_simt.cu"
 
 
 def tc_attention(w):
@@ -160,8 +174,8 @@ def measured_traffic(kernel, workload):
         return None
     with open(TRAFFIC_FILE) as f:
         t = json.load(f)
-    rec = t.get(workload, {}).get(kernel)
-    if not rec or rec.get("src_sha") != src_hash(KERNEL_SOURCES[kernel]):
+    rec = t.get(workload.name, {}).get(kernel)
+    if not rec or rec.get("src_sha") != src_hash([kernel_source(kernel, workload)]):
         return None
     return rec.get("bytes_per_launch")
 
@@ -223,6 +237,87 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(pw) if pw else None}
 
 
+# ------------------------------------------------------ multi-rank logic --
+
+def replica_workload(w, rank):
+    """The workload instance of one rank: same shape, its own seed (independent problems)."""
+    return w if rank == 0 else w.scaled(seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (the job's device time is the slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_max_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own instance in the max-over-ranks time."""
+    return world * tokens_per_rank / (ms_max_per_step * 1e-3)
+
+
+# ----------------------------------------------------------- dense path --
+
+def dense_flops(w):
+    """4 d FLOPs per attended (query, key) pair of plain causal attention."""
+    pairs = 0
+    for t in range(w.Nq) if w.Nq <= 4 else []:
+        pairs += w.q_offset + t + 1
+    if w.Nq > 4:
+        p0, p1 = w.q_offset, w.q_offset + w.Nq  # positions [p0, p1): sum of (p + 1)
+        pairs = (p1 * (p1 + 1) - p0 * (p0 + 1)) // 2
+    return 4 * w.d * pairs * w.B * w.Hq
+
+
+def time_dense(P, s, w, Q, K, V, buf, stream, steps, warmup):
+    """Event-timed dense_forward (plain causal attention) on the same inputs."""
+    steps = max(3, min(steps, 10)) if dense_flops(w) < 1e14 else 2  # a 1M-token dense pass takes seconds
+    for _ in range(1 if dense_flops(w) >= 1e14 else max(1, warmup // 2)):
+        P.dense_forward(s, Q, K, V, buf.O, buf.lse, buf.status, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        P.dense_forward(s, Q, K, V, buf.O, buf.lse, buf.status, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    return {"ms": round(ms, 4), "tflops": round(dense_flops(w) / (ms * 1e-3) / 1e12, 2)}
+
+
+def break_even(args, w):
+    """Sparse step (pyramid + selection + attention) vs dense causal attention over context lengths."""
+    import hierarchical_block_sparse_pyr_b200 as P
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    points = []
+    for n in (2048, 4096, 8192, 16384, 32768, 65536):
+        wn = w.scaled(name=f"{w.name}@N={n}", N=n, Nq=n, q_offset=0)
+        s = P.shape_of(wn)
+        Qh, Kh, Vh, _ = synth.generate(wn)
+        Q, K, V = Qh.cuda(), Kh.cuda(), Vh.cuda()
+        buf = P.Buffers(s)
+        for _ in range(3):
+            P.run(s, Q, K, V, buf, stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(10):
+            P.run(s, Q, K, V, buf, stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        sparse_ms = e0.elapsed_time(e1) / 10
+        dense = time_dense(P, s, wn, Q, K, V, buf, stream, 10, 3)
+        points.append({"N": n, "sparse_step_ms": round(sparse_ms, 4), "dense_ms": dense["ms"]})
+        del Q, K, V, buf
+        torch.cuda.empty_cache()
+    be = next((p["N"] for p in points if p["sparse_step_ms"] < p["dense_ms"]), None)
+    return {"metric": "break-even context length: pyramid + select + block-sparse attention vs dense causal",
+            "workload": w.name, "points": points, "break_even_N": be}
+
+
 # --------------------------------------------------------------- our arm --
 
 def count_launches(step):
@@ -244,16 +339,25 @@ def run_ours(args, w, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    w = replica_workload(w, rank)
     s = P.shape_of(w)
     Qh, Kh, Vh, _ = synth.generate(w, pin=True)
     Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
     buf = P.Buffers(s, dev)
     stream = torch.cuda.current_stream(dev)
 
+    # prefill builds the pyramid from K; a decode step refreshes only the nodes over the
+    # appended position (the pyramid of the prefilled context is built once, untimed)
+    if w.decode:
+        P.pyr_build(s, K, buf.pyr, buf.status, stream)
+
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        P.pyr_build(s, K, buf.pyr, buf.status, stream)
+        if w.decode:
+            P.pyr_update(s, K, buf.pyr, w.N - 1, buf.status, stream)
+        else:
+            P.pyr_build(s, K, buf.pyr, buf.status, stream)
         if ev:
             ev[1].record(stream)
         P.pyr_select(s, Q, buf.pyr, buf.idx, buf.gap, buf.status, stream)
@@ -293,10 +397,7 @@ def run_ours(args, w, rank, world, local_rank):
         per["pyramid"].append(ev[0].elapsed_time(ev[1]))
         per["select"].append(ev[1].elapsed_time(ev[2]))
         per["attention"].append(ev[2].elapsed_time(ev[3]))
-    ms_t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms_total, world, dev)
 
     # end to end through the binding: pinned host inputs -> device -> path -> O back to pinned host
     O_host = torch.empty(buf.O.shape, dtype=buf.O.dtype, pin_memory=True)
@@ -322,34 +423,37 @@ def run_ours(args, w, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = torch.tensor([e0.elapsed_time(e1) / e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev)
     if int(buf.status.item()) != 0:
         raise RuntimeError(f"device status {buf.status.item()}")
+
+    dense = time_dense(P, s, w, Q, K, V, buf, stream, args.steps, args.warmup)
 
     wc = work_counts(w)
     peaks = load_peaks()
     ms_step = ms_max / args.steps
-    value = world * wc["tokens"] / (ms_step * 1e-3)
+    value = job_throughput(wc["tokens"], world, ms_step)
     avg = {k: sum(v) / len(v) for k, v in per.items()}
     sm_clock = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
     kernels = {
-        "pyramid": dict(ms=avg["pyramid"], bound="hbm", achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9,
+        "pyramid": dict(ms=avg["pyramid"], bound="hbm", kernel="pyr_update" if w.decode else "pyr_build", achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9,
                         peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["pyr_bytes"],
-                        traffic=measured_traffic("pyramid", w.name)),
+                        traffic=measured_traffic("pyramid", w)),
         "select": dict(ms=avg["select"], bound="tensor" if tc_select(w) else "alu",
                        achieved=wc["sel_flops"] / (avg["select"] * 1e-3) / 1e12,
                        peak=(peaks["bf16_tflops_sustained"] if tc_select(w) else
                              148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s", algorithmic=wc["sel_flops"],
                        hbm_gbs=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9,
                        hbm_frac=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                       traffic=measured_traffic("select", w.name)),
-        "attention": dict(ms=avg["attention"], bound="tensor" if tc_attention(w) else "alu",
-                          achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
-                          peak=(peaks["bf16_tflops_sustained"] if tc_attention(w) else
-                                148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s",
-                          algorithmic=wc["att_flops"], traffic=measured_traffic("attention", w.name)),
+                       traffic=measured_traffic("select", w)),
+        "attention": (dict(ms=avg["attention"], bound="hbm", achieved=wc["att_bytes"] / (avg["attention"] * 1e-3) / 1e9,
+                           peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["att_bytes"],
+                           traffic=measured_traffic("attention", w)) if w.decode else
+                      dict(ms=avg["attention"], bound="tensor" if tc_attention(w) else "alu",
+                           achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
+                           peak=(peaks["bf16_tflops_sustained"] if tc_attention(w) else
+                                 148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s",
+                           algorithmic=wc["att_flops"], traffic=measured_traffic("attention", w))),
     }
     for k in kernels.values():
         k["frac"] = k["achieved"] / k["peak"]
@@ -368,12 +472,13 @@ def run_ours(args, w, rank, world, local_rank):
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (Q+K+V %d MiB > 126 MB)" % (
                        (Qh.numel() + Kh.numel() + Vh.numel()) * Qh.element_size() >> 20)},
-        "e2e": {"value": round(world * wc["tokens"] / (float(e_ms.item()) * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(wc["tokens"], world, e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
         "roofline": roofline,
         "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
                     for k, v in kernels.items()},
+        "dense": dict(dense, speedup_of_sparse_step=round(dense["ms"] / ms_step, 3)),
         "kernel_names": kernel_names,
         "clocks": clk,
         "peaks_source": peaks["source"],
@@ -467,6 +572,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--break-even", action="store_true",
+                    help="sweep the context length and report where the sparse step beats dense attention")
     ap.add_argument("--n", type=int, default=None,
                     help="shrink the context length (and query rows) of the workload: for profiling the same "
                          "kernels on a smaller case; the default JSON line always uses the full workload")
@@ -480,6 +587,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.break_even:
+        print(json.dumps(break_even(args, w)), flush=True)
+        return
 
     if args.impl == "reference":
         if rank == 0:

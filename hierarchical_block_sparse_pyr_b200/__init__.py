@@ -3,11 +3,12 @@
 Thin ctypes binding over ``lib/libpyr.so`` (the C ABI declared in
 ``include/pyr.h``). Functions here only marshal arguments: torch tensors give
 device pointers and the current CUDA stream; every step of the computation
-runs in the library's sm_100a kernels. There is no CPU fallback: importing
-this package fails if the library is missing, and every call needs CUDA
-tensors.
+runs in the library's sm_100a kernels. There is no CPU fallback: the library
+is loaded on first use and every call raises ImportError if it is missing;
+every call needs CUDA tensors.
 
     pyr_build(shape, K, pyr)                  key pyramid (mean pooling)
+    pyr_update(shape, K, pyr, from_pos)       refresh the nodes over rewritten key positions
     pyr_select(shape, Q, pyr, idx, gap)       coarse-to-fine LogSumExp top-K
     bsa_forward(shape, Q, K, V, idx, O, lse)  causal block-sparse attention
     dense_forward(shape, Q, K, V, O, lse)     dense causal attention
@@ -26,8 +27,8 @@ LIB_PATH = os.path.join(_PKG, "lib", "libpyr.so")
 PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = range(6)
 PYR_F32, PYR_BF16 = 0, 1
 
-ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_select", "bsa_forward",
-               "dense_forward", "pyr_strerror")
+ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_update", "pyr_select",
+               "bsa_forward", "dense_forward", "pyr_selftest_wait", "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -59,22 +60,34 @@ def _load_lib():
     lib.pyr_num_qblocks.restype = ctypes.c_int64
     lib.pyr_build.argtypes = [sp, vp, vp, vp, vp]
     lib.pyr_build.restype = ctypes.c_int
+    lib.pyr_update.argtypes = [sp, vp, vp, ctypes.c_int, vp, vp]
+    lib.pyr_update.restype = ctypes.c_int
     lib.pyr_select.argtypes = [sp, vp, vp, vp, vp, vp, vp]
     lib.pyr_select.restype = ctypes.c_int
     lib.bsa_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bsa_forward.restype = ctypes.c_int
     lib.dense_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.dense_forward.restype = ctypes.c_int
+    lib.pyr_selftest_wait.argtypes = [vp, vp]
+    lib.pyr_selftest_wait.restype = ctypes.c_int
     lib.pyr_strerror.argtypes = [ctypes.c_int]
     lib.pyr_strerror.restype = ctypes.c_char_p
     return lib
 
 
-_lib = _load_lib()
+_lib_handle = None
+
+
+def _L():
+    """The loaded libpyr (loaded once, on first use)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load_lib()
+    return _lib_handle
 
 
 def strerror(code: int) -> str:
-    return _lib.pyr_strerror(code).decode()
+    return _L().pyr_strerror(code).decode()
 
 
 def make_shape(B, Hq, Hkv, N, Nq, q_offset, d, b, topk, cap, dtype) -> PyrShape:
@@ -89,15 +102,15 @@ def shape_of(w) -> PyrShape:
 
 
 def num_levels(s: PyrShape) -> int:
-    return _lib.pyr_num_levels(ctypes.byref(s))
+    return _L().pyr_num_levels(ctypes.byref(s))
 
 
 def num_nodes(s: PyrShape) -> int:
-    return _lib.pyr_num_nodes(ctypes.byref(s))
+    return _L().pyr_num_nodes(ctypes.byref(s))
 
 
 def num_qblocks(s: PyrShape) -> int:
-    return _lib.pyr_num_qblocks(ctypes.byref(s))
+    return _L().pyr_num_qblocks(ctypes.byref(s))
 
 
 def _dev(t, name, nullable=False):
@@ -124,24 +137,34 @@ def _check(rc, what):
 
 
 def pyr_build(s: PyrShape, K, pyr, status=None, stream=None):
-    _check(_lib.pyr_build(ctypes.byref(s), _dev(K, "K"), _dev(pyr, "pyr"), _dev(status, "status", True),
+    _check(_L().pyr_build(ctypes.byref(s), _dev(K, "K"), _dev(pyr, "pyr"), _dev(status, "status", True),
                           _stream(stream)), "pyr_build")
 
 
+def pyr_update(s: PyrShape, K, pyr, from_pos: int, status=None, stream=None):
+    _check(_L().pyr_update(ctypes.byref(s), _dev(K, "K"), _dev(pyr, "pyr"), int(from_pos), _dev(status, "status", True),
+                           _stream(stream)), "pyr_update")
+
+
 def pyr_select(s: PyrShape, Q, pyr, idx, gap=None, status=None, stream=None):
-    _check(_lib.pyr_select(ctypes.byref(s), _dev(Q, "Q"), _dev(pyr, "pyr"), _dev(idx, "idx"),
+    _check(_L().pyr_select(ctypes.byref(s), _dev(Q, "Q"), _dev(pyr, "pyr"), _dev(idx, "idx"),
                            _dev(gap, "gap", True), _dev(status, "status", True), _stream(stream)), "pyr_select")
 
 
 def bsa_forward(s: PyrShape, Q, K, V, idx, O, lse=None, status=None, stream=None):
-    _check(_lib.bsa_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "idx"), _dev(O, "O"),
+    _check(_L().bsa_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "idx"), _dev(O, "O"),
                             _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)), "bsa_forward")
 
 
 def dense_forward(s: PyrShape, Q, K, V, O, lse=None, status=None, stream=None):
-    _check(_lib.dense_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(O, "O"),
+    _check(_L().dense_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(O, "O"),
                               _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)),
            "dense_forward")
+
+
+def selftest_wait(status, stream=None):
+    """Launch the bounded-wait self-test; status (int32 CUDA tensor) reads PYR_ETIMEOUT afterwards."""
+    _check(_L().pyr_selftest_wait(_dev(status, "status"), _stream(stream)), "pyr_selftest_wait")
 
 
 class Buffers:
@@ -151,12 +174,19 @@ class Buffers:
         self.shape = s
         nqb = num_qblocks(s)
         dt = torch.float32 if s.dtype == PYR_F32 else torch.bfloat16
-        self.pyr = torch.empty((s.B, s.Hkv, num_nodes(s), s.d), dtype=torch.float32, device=device)
+        # each node mean x is stored as the bf16 pair (hi, lo) = (RN(x), RN(x - hi))
+        self.pyr = torch.empty((s.B, s.Hkv, num_nodes(s), 2, s.d), dtype=torch.bfloat16, device=device)
         self.idx = torch.empty((s.B, s.Hkv, nqb, s.topk), dtype=torch.int32, device=device)
         self.gap = torch.empty((s.B, s.Hkv, nqb), dtype=torch.float32, device=device)
         self.O = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=dt, device=device)
         self.lse = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def pyramid_means(pyr: torch.Tensor) -> torch.Tensor:
+    """fp32 node means [..., P, d] from the (hi, lo) pair storage [..., P, 2, d]."""
+    p = pyr.float()
+    return p[..., 0, :] + p[..., 1, :]
 
 
 def run(s: PyrShape, Q, K, V, buf: Buffers, stream=None, with_gap=True):

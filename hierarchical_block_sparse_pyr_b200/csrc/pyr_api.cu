@@ -83,19 +83,30 @@ int64_t pyr_num_qblocks(const pyr_shape* s) {
   return make_geo(s, &g) == PYR_OK ? g.nqb : 0;
 }
 
-int pyr_build(const pyr_shape* s, const void* K, float* pyr, int* dev_status, void* stream) {
+int pyr_build(const pyr_shape* s, const void* K, void* pyr, int* dev_status, void* stream) {
   Geo g;
   int rc = make_geo(s, &g);
   if (rc) return rc;
   if (!K || !pyr || !aligned16(K) || !aligned16(pyr)) return PYR_EINVAL;
-  return launch_status(pyr::launch_pyramid(g, K, pyr, dev_status, (cudaStream_t)stream));
+  return launch_status(pyr::launch_pyramid(g, K, static_cast<__nv_bfloat16*>(pyr), dev_status, (cudaStream_t)stream));
 }
 
-int pyr_select(const pyr_shape* s, const void* Q, const float* pyr, int32_t* idx, float* gap, int* dev_status,
+int pyr_update(const pyr_shape* s, const void* K, void* pyr, int from_pos, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!K || !pyr || !aligned16(K) || !aligned16(pyr)) return PYR_EINVAL;
+  if (from_pos < 0 || from_pos >= s->N) return PYR_EINVAL;
+  return launch_status(
+      pyr::launch_pyramid_update(g, K, static_cast<__nv_bfloat16*>(pyr), from_pos, dev_status, (cudaStream_t)stream));
+}
+
+int pyr_select(const pyr_shape* s, const void* Q, const void* pyr_v, int32_t* idx, float* gap, int* dev_status,
                void* stream) {
   Geo g;
   int rc = make_geo(s, &g);
   if (rc) return rc;
+  const __nv_bfloat16* pyr = static_cast<const __nv_bfloat16*>(pyr_v);
   if (!Q || !pyr || !idx || !aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PYR_EINVAL;
   if (pyr::select_tc_supported(g))
     return launch_status(pyr::launch_select_tc(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
@@ -112,6 +123,8 @@ int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V,
     return PYR_EINVAL;
   if (pyr::attn_tc_supported(g))
     return launch_status(pyr::launch_attn_tc(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
+  if (pyr::attn_decode_supported(g))
+    return launch_status(pyr::launch_attn_decode(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
 }
 
@@ -123,6 +136,8 @@ int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* 
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return PYR_EINVAL;
   if (pyr::attn_tc_supported(g))
     return launch_status(pyr::launch_attn_tc(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
+  if (pyr::attn_decode_supported(g))
+    return launch_status(pyr::launch_attn_decode(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
 }
 

@@ -38,6 +38,20 @@ __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Pyramid node storage: a node mean x is kept as the unevaluated bf16 pair
+// hi = RN(x), lo = RN(x - hi) (|x - hi - lo| <= 2^-17 |x|), in a row of 2d
+// bf16: [hi_0 .. hi_{d-1} | lo_0 .. lo_{d-1}]. This is exactly the operand
+// format the tensor-core scoring consumes, so selection copies node rows
+// straight into its MMA operands.
+__device__ __forceinline__ void split_store(__nv_bfloat16* row, int d, int e, float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  row[e] = hi;
+  row[d + e] = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+__device__ __forceinline__ float split_load(const __nv_bfloat16* row, int d, int e) {
+  return __bfloat162float(row[e]) + __bfloat162float(row[d + e]);
+}
+
 // Order-preserving map of a float to uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -45,11 +59,16 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 }
 
 // Launchers (one per kernel family). Each returns cudaSuccess or the launch error.
-cudaError_t launch_pyramid(const Geo& g, const void* K, float* pyr, int* status, cudaStream_t st);
-cudaError_t launch_select(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int* status, cudaStream_t st);
+cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,
+                                  cudaStream_t st);
+bool attn_decode_supported(const Geo& g);
+cudaError_t launch_attn_decode(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
+                               int dense, void* O, float* lse, int* status, cudaStream_t st);
+cudaError_t launch_select(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                           cudaStream_t st);
 bool select_tc_supported(const Geo& g);
-cudaError_t launch_select_tc(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                              cudaStream_t st);
 bool attn_tc_supported(const Geo& g);
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,

@@ -3,7 +3,9 @@
 // hierarchy; PHBA A.1.2: centroids average the block's key rows in fp32).
 //
 // HBM-bound: K is read exactly once with 16-byte loads and the pyramid
-// (about 2 nb d floats per head) is written once.
+// (about 2 nb nodes of 4 d bytes per head) is written once. Means are
+// accumulated in fp32 and stored as bf16 (hi, lo) pairs; every level is
+// computed from fp32 sums, so the pair rounding never compounds.
 //   pyr_chunk_kernel  one CTA per chunk of CB consecutive key blocks of one
 //                     (batch, kv head): one warp streams one block at a time
 //                     (lanes split the row into 16-byte vectors, the rest of
@@ -62,7 +64,7 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
 
 // smem: two ping-pong level buffers of CB x D floats.
 template <typename T, int D>
-__global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __restrict__ K, float* __restrict__ pyr,
+__global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __restrict__ K, __nv_bfloat16* __restrict__ pyr,
                                                                   Geo g, int CB, int t_levels) {
   constexpr int E = Vec<T>::E;
   constexpr int VPR = D / E;        // 16-byte vectors per key row
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __res
   const int c = lane % VPR, rl = lane / VPR;
   const int j_begin = chunk * CB;
   const T* Ku = K + (size_t)unit * g.N * D;
-  float* pu = pyr + (size_t)unit * g.P * D;
+  __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 2 * D;
 
   // level 0: warp w handles blocks w, w + 8, ...
   for (int jl = warp; jl < CB; jl += kChunkThreads / 32) {
@@ -113,10 +115,24 @@ __global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __res
       for (int k = 0; k < E; k++) dst[k] = acc[k];
       if (j < g.nb) {
         const float inv = 1.f / (float)cnt;
-        float4* o = reinterpret_cast<float4*>(pu + (size_t)j * D + c * E);
+        uint32_t wh[E / 2], wl[E / 2];
 #pragma unroll
-        for (int k = 0; k < E; k += 4) o[k / 4] = make_float4(acc[k] * inv, acc[k + 1] * inv, acc[k + 2] * inv,
-                                                              acc[k + 3] * inv);
+        for (int k = 0; k < E / 2; k++) {
+          const float x0 = acc[2 * k] * inv, x1 = acc[2 * k + 1] * inv;
+          const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 lo = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+          wh[k] = *reinterpret_cast<const uint32_t*>(&h);
+          wl[k] = *reinterpret_cast<const uint32_t*>(&lo);
+        }
+        __nv_bfloat16* row = pu + (size_t)j * 2 * D + c * E;
+        if constexpr (E == 8) {
+          *reinterpret_cast<uint4*>(row) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          *reinterpret_cast<uint4*>(row + D) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        } else {
+          *reinterpret_cast<uint2*>(row) = make_uint2(wh[0], wh[1]);
+          *reinterpret_cast<uint2*>(row + D) = make_uint2(wl[0], wl[1]);
+        }
       }
     }
   }
@@ -135,7 +151,7 @@ __global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __res
       if (m < g.lvl_n[l]) {
         const int j0 = m << l;
         const int j1 = min((m + 1) << l, g.nb);
-        pu[(size_t)(g.lvl_off[l] + m) * D + e] = s / (float)tokens_in(j0, j1, g.b, g.N);
+        split_store(pu + (size_t)(g.lvl_off[l] + m) * 2 * D, D, e, s / (float)tokens_in(j0, j1, g.b, g.N));
       }
     }
     __syncthreads();
@@ -146,11 +162,11 @@ __global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __res
 }
 
 // Levels t+1 .. L from level t, for one unit and a 16-wide slice of d.
-__global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(float* __restrict__ pyr, Geo g, int t) {
+__global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(__nv_bfloat16* __restrict__ pyr, Geo g, int t) {
   extern __shared__ float sm[];
   const int unit = blockIdx.y;
   const int e0 = blockIdx.x * kTopSlice;
-  float* pu = pyr + (size_t)unit * g.P * g.d;
+  __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 2 * g.d;
   const int nt = g.lvl_n[t];
   float* cur = sm;
   float* nxt = sm + (size_t)nt * kTopSlice;
@@ -158,7 +174,7 @@ __global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(float* __restrict_
   for (int x = threadIdx.x; x < nt * kTopSlice; x += kTopThreads) {
     const int m = x / kTopSlice, e = x - m * kTopSlice;
     const int j0 = m << t, j1 = min((m + 1) << t, g.nb);
-    cur[x] = pu[(size_t)(g.lvl_off[t] + m) * g.d + e0 + e] * (float)tokens_in(j0, j1, g.b, g.N);
+    cur[x] = split_load(pu + (size_t)(g.lvl_off[t] + m) * 2 * g.d, g.d, e0 + e) * (float)tokens_in(j0, j1, g.b, g.N);
   }
   __syncthreads();
   int n_prev = nt;
@@ -170,7 +186,7 @@ __global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(float* __restrict_
       if (2 * m + 1 < n_prev) s += cur[(size_t)(2 * m + 1) * kTopSlice + e];
       nxt[x] = s;
       const int j0 = m << l, j1 = min((m + 1) << l, g.nb);
-      pu[(size_t)(g.lvl_off[l] + m) * g.d + e0 + e] = s / (float)tokens_in(j0, j1, g.b, g.N);
+      split_store(pu + (size_t)(g.lvl_off[l] + m) * 2 * g.d, g.d, e0 + e, s / (float)tokens_in(j0, j1, g.b, g.N));
     }
     __syncthreads();
     float* tmp = cur;
@@ -180,8 +196,55 @@ __global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(float* __restrict_
   }
 }
 
+// Incremental update after the keys at positions >= from_pos (same shape)
+// were rewritten, e.g. a decoded token written into the last slot: every
+// node whose key range reaches such a position is recomputed, one CTA per
+// (batch, kv head), thread e owning element e of d. Changed nodes are carried
+// level to level as fp32 sums in shared memory (at most 32 per level);
+// unchanged siblings are read back from their (hi, lo) pairs.
+constexpr int kUpdMax = 32;
+
+template <typename T>
+__global__ void __launch_bounds__(128) pyr_update_kernel(const T* __restrict__ K, __nv_bfloat16* __restrict__ pyr,
+                                                         Geo g, int j_first) {
+  __shared__ float sums[2][kUpdMax][128];
+  const int unit = blockIdx.x;
+  const int e = threadIdx.x;
+  if (e >= g.d) return;
+  const T* Ku = K + (size_t)unit * g.N * g.d;
+  __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 2 * g.d;
+  int cur = 0;
+  // level 0: the changed blocks, straight from K
+  for (int j = j_first; j < g.nb; j++) {
+    const int t0 = j * g.b, t1 = min(t0 + g.b, g.N);
+    float acc = 0.f;
+    for (int t = t0; t < t1; t++) acc += to_f32(Ku[(size_t)t * g.d + e]);
+    sums[cur][j - j_first][e] = acc;
+    split_store(pu + (size_t)j * 2 * g.d, g.d, e, acc / (float)(t1 - t0));
+  }
+  for (int l = 1; l <= g.L; l++) {
+    const int m0 = j_first >> l, c0 = j_first >> (l - 1);  // first changed node, first changed child
+    for (int m = m0; m < g.lvl_n[l]; m++) {
+      float s = 0.f;
+      for (int ch = 2 * m; ch <= 2 * m + 1 && ch < g.lvl_n[l - 1]; ch++) {
+        if (ch >= c0) {
+          s += sums[cur][ch - c0][e];
+        } else {
+          const int cj0 = ch << (l - 1), cj1 = min((ch + 1) << (l - 1), g.nb);
+          s += split_load(pu + (size_t)(g.lvl_off[l - 1] + ch) * 2 * g.d, g.d, e) *
+               (float)tokens_in(cj0, cj1, g.b, g.N);
+        }
+      }
+      sums[cur ^ 1][m - m0][e] = s;
+      const int j0 = m << l, j1 = min((m + 1) << l, g.nb);
+      split_store(pu + (size_t)(g.lvl_off[l] + m) * 2 * g.d, g.d, e, s / (float)tokens_in(j0, j1, g.b, g.N));
+    }
+    cur ^= 1;
+  }
+}
+
 template <typename T, int D>
-cudaError_t launch_chunks(const Geo& g, const void* K, float* pyr, int CB, int t, cudaStream_t st) {
+cudaError_t launch_chunks(const Geo& g, const void* K, __nv_bfloat16* pyr, int CB, int t, cudaStream_t st) {
   const size_t smem = (size_t)2 * CB * D * sizeof(float);
   auto kern = pyr_chunk_kernel<T, D>;
   if (smem > 48 * 1024) {
@@ -195,7 +258,19 @@ cudaError_t launch_chunks(const Geo& g, const void* K, float* pyr, int CB, int t
 
 }  // namespace
 
-cudaError_t launch_pyramid(const Geo& g, const void* K, float* pyr, int* status, cudaStream_t st) {
+cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,
+                                  cudaStream_t st) {
+  const int j_first = from_pos / g.b;
+  if (g.nb - j_first > kUpdMax) return launch_pyramid(g, K, pyr, status, st);
+  if (g.dtype == PYR_BF16)
+    pyr_update_kernel<__nv_bfloat16><<<g.B * g.Hkv, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(K), pyr, g,
+                                                                   j_first);
+  else
+    pyr_update_kernel<float><<<g.B * g.Hkv, 128, 0, st>>>(reinterpret_cast<const float*>(K), pyr, g, j_first);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int* status, cudaStream_t st) {
   (void)status;
   // Chunk: ~1024 key rows per CTA, and at most 1024 level-t nodes left for the top kernel.
   int CB = 1;

@@ -80,7 +80,7 @@ __device__ void bitonic_desc(unsigned long long* key, int n_pow2) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ Q, const float* __restrict__ pyr,
+__global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ Q, const __nv_bfloat16* __restrict__ pyr,
                                                           int32_t* __restrict__ idx, float* __restrict__ gap_out,
                                                           int* status, Geo g) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
     const int hq = hk * g.G + gg;
     Qs[(size_t)e * R + r] = Q[(((size_t)bi * g.Hq + hq) * g.Nq + t) * d + e];
   }
-  const float* pu = pyr + (size_t)unit * g.P * d;
+  const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 2 * d;
   // exact means of the straddling node's valid part, levels 1..s0
   for (int e = threadIdx.x; e < d; e += kThreads) {
     float acc = 0.f;
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
     for (int l = 1; l <= g.s0 && l < kMaxLevels; l++) {
       if ((i >> (l - 1)) & 1) {
         const int m = (i >> (l - 1)) - 1;  // whole left sibling at level l-1
-        acc += pu[(size_t)(g.lvl_off[l - 1] + m) * d + e] * (float)((int64_t)g.b << (l - 1));
+        acc += split_load(pu + (size_t)(g.lvl_off[l - 1] + m) * 2 * d, d, e) * (float)((int64_t)g.b << (l - 1));
       }
       const int cnt_blocks = i - ((i >> l) << l);
       part[l * d + e] = cnt_blocks > 0 ? acc / (float)((int64_t)cnt_blocks * g.b) : 0.f;
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
       const int m = cand[c];
       const int j0 = m << l;
       const bool straddle = ((m + 1) << l) > i && j0 < i && l > 0;
-      Mt[(size_t)e * CP + c] = straddle ? part[l * d + e] : pu[(size_t)(g.lvl_off[l] + m) * d + e];
+      Mt[(size_t)e * CP + c] = straddle ? part[l * d + e] : split_load(pu + (size_t)(g.lvl_off[l] + m) * 2 * d, d, e);
     }
     for (int c = threadIdx.x; c < nc; c += kThreads) {
       const int m = cand[c];
@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
 }
 
 template <typename T>
-cudaError_t launch_t(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+cudaError_t launch_t(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                      cudaStream_t st) {
   const SelSmem L = sel_layout(g.G * min(g.b, g.Nq), g.d, (int)sizeof(T), g.cap);
   auto kern = select_kernel<T>;
@@ -296,7 +296,7 @@ size_t select_smem_bytes(const Geo& g) {
   return sel_layout(g.G * min(g.b, g.Nq), g.d, elt, g.cap).total;
 }
 
-cudaError_t launch_select(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
+cudaError_t launch_select(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                           cudaStream_t st) {
   if (g.dtype == PYR_BF16) return launch_t<__nv_bfloat16>(g, Q, pyr, idx, gap, status, st);
   return launch_t<float>(g, Q, pyr, idx, gap, status, st);

@@ -5,11 +5,13 @@
 // PHBA A.1.2).
 //
 // One CTA (4 warps) per (batch, kv head, query block i). Per level:
-//   gather   the <= cap candidate node means (fp32; the node that straddles
-//            block i uses the exact mean of its part before i, from the
-//            binary decomposition of [m 2^l, i) into whole finer nodes) are
-//            split into bf16 hi + lo with x - hi - lo <= 2^-18 |x| and written
-//            in the 128B-swizzled K-major layout;
+//   gather   the <= cap candidate node rows are copied (cp.async, 16 bytes
+//            per thread) straight from the pyramid, which already stores every
+//            mean as a bf16 (hi, lo) pair, to their places in the 128B-swizzled
+//            K-major A operands; the one node that straddles block i
+//            uses the exact mean of its part before i, from the binary
+//            decomposition of [m 2^l, i) into whole finer nodes, split by a
+//            thread into hi + lo;
 //   score    D[candidate][row] = kbar . q_row on the tensor cores, as
 //            A_hi * Q^T + A_lo * Q^T (M = candidates: 64 or 128, N = the
 //            G*b query rows staged once by TMA, K = d), fp32 accumulation in
@@ -67,7 +69,7 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
 
 template <int MC>
 __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                             const float* __restrict__ pyr, int32_t* __restrict__ idx,
+                                                             const __nv_bfloat16* __restrict__ pyr, int32_t* __restrict__ idx,
                                                              float* __restrict__ gap_out, int* status, Geo g) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -125,12 +127,13 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     tmem_relinquish();
   }
   // exact means of the straddling node's part before i, levels 1..s0
-  const float* pu = pyr + (size_t)unit * g.P * 128;
+  const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 256;
   for (int e = threadIdx.x; e < 128; e += kThreads) {
     float acc = 0.f;
     part[e] = 0.f;
     for (int l = 1; l <= g.s0; l++) {
-      if ((i >> (l - 1)) & 1) acc += pu[(size_t)(g.lvl_off[l - 1] + (i >> (l - 1)) - 1) * 128 + e] * (float)(g.b << (l - 1));
+      if ((i >> (l - 1)) & 1)
+        acc += split_load(pu + (size_t)(g.lvl_off[l - 1] + (i >> (l - 1)) - 1) * 256, 128, e) * (float)(g.b << (l - 1));
       const int cnt = i - ((i >> l) << l);
       part[l * 128 + e] = cnt > 0 ? acc / (float)(cnt * g.b) : 0.f;
     }
@@ -151,37 +154,35 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   for (int l = g.s0; l >= 0 && ok; l--) {
     const int nc = *s_nc;
     const bool start = (l == g.s0);
-    // ---- gather: warp w handles candidate rows w, w+4, ...; lane holds 4 of the 128 d-elements.
-    // Rows are fetched 8 at a time so that their loads are in flight together.
-    const int nrow = nc > warp ? (nc - warp + 3) / 4 : 0;
-    for (int k0 = 0; k0 < nrow; k0 += 8) {
-      float4 v[8];
+    // ---- gather: every thread copies 16-byte chunks of the candidates' (hi, lo) rows with
+    // cp.async straight to their swizzled places in the A operands (consecutive threads take
+    // consecutive chunks of a row: coalesced, all copies in flight together); the straddling
+    // node's row (at most one per level) is written by warp 1 from the exact partial mean.
+    const int ms = (l > 0 && (i & ((1 << l) - 1)) != 0) ? (i >> l) : -1;  // the straddling node
+    for (int x = threadIdx.x; x < nc * 32; x += kThreads) {
+      const int c = x >> 5, q = x & 31;  // chunk q: 8 elements; 0..15 hi, 16..31 lo
+      const int m = start ? c : cand[c];
+      if (m == ms) continue;
+      const int h = (q >> 3) & 1, c8 = q & 7;
+      unsigned char* dst = ((q < 16) ? sAh : sAl) + h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4);
+      cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
+    }
+    cp_async_wait_all();
+    if (warp == 1 && ms >= 0) {
+      for (int c = 0; c < nc; c++) {
+        if ((start ? c : cand[c]) != ms) continue;
+        const float4 v = *reinterpret_cast<const float4*>(part + l * 128 + lane * 4);
+        const float x[4] = {v.x, v.y, v.z, v.w};
+        float hi[4], lo[4];
 #pragma unroll
-      for (int k = 0; k < 8; k++) {
-        if (k0 + k < nrow) {
-          const int c = warp + 4 * (k0 + k);
-          const int m = start ? c : cand[c];
-          const bool straddle = l > 0 && ((m + 1) << l) > i;
-          v[k] = straddle ? *reinterpret_cast<const float4*>(part + l * 128 + lane * 4)
-                          : __ldg(reinterpret_cast<const float4*>(pu + (size_t)(g.lvl_off[l] + m) * 128) + lane);
+        for (int e = 0; e < 4; e++) {
+          hi[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
+          lo[e] = x[e] - hi[e];
         }
-      }
-#pragma unroll
-      for (int k = 0; k < 8; k++) {
-        if (k0 + k < nrow) {
-          const int c = warp + 4 * (k0 + k);
-          const float x[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-          float hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; e++) {
-            hi[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
-            lo[e] = x[e] - hi[e];
-          }
-          const int h = lane >> 4, c8 = (lane & 15) >> 1, half8 = (lane & 1) * 8;
-          const int off = h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4) + half8;
-          *reinterpret_cast<uint2*>(sAh + off) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
-          *reinterpret_cast<uint2*>(sAl + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
-        }
+        const int h = lane >> 4, c8 = (lane & 15) >> 1, half8 = (lane & 1) * 8;
+        const int off = h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4) + half8;
+        *reinterpret_cast<uint2*>(sAh + off) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
+        *reinterpret_cast<uint2*>(sAl + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
       }
     }
     fence_proxy_async_smem();
@@ -329,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
 }
 
 template <int MC>
-cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const float* pyr, int32_t* idx, float* gap, int* status,
-                      cudaStream_t st) {
+cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
+                      int* status, cudaStream_t st) {
   const SelPlan L = sel_plan(g.G * g.b, MC, g.s0 + 1, 128);
   auto kern = select_tc_kernel<MC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
@@ -352,8 +353,8 @@ bool select_tc_supported(const Geo& g) {
   return sel_plan(R, MC, g.s0 + 1, 128).total <= 227 * 1024;
 }
 
-cudaError_t launch_select_tc(const Geo& g, const void* Q, const float* pyr, int32_t* idx, float* gap, int* status,
-                             cudaStream_t st) {
+cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
+                             int* status, cudaStream_t st) {
   CUtensorMap mq;
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq)) return cudaErrorInvalidValue;
   if (g.cap <= 64) return launch_mc<64>(g, mq, pyr, idx, gap, status, st);

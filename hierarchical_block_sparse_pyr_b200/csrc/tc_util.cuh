@@ -69,6 +69,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
 
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// 16-byte asynchronous global -> shared copy (bypassing L1), and the wait for
+// all of this thread's outstanding copies.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // ---- tensor memory ------------------------------------------------------
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
@@ -200,9 +209,10 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Host: 3-D TMA map over a [heads][rows][d] bf16 tensor with a box of 64 d-elements x
-// 64 rows x 1 head and 128-byte swizzle (rows past the end read as zeros).
-bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, int d, int rows, int heads);
+// Host: 3-D TMA map over a [heads][rows][inner] bf16 tensor with a box of 64
+// inner elements x box_rows rows x 1 head and 128-byte swizzle (rows past the
+// end read as zeros).
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, int inner, int rows, int heads, int box_rows = 64);
 
 }  // namespace tc
 }  // namespace pyr

@@ -21,8 +21,11 @@
  * Conventions shared by every entry point
  *   Layouts (row-major, contiguous, every base pointer 16-byte aligned):
  *     Q, O  [B][Hq][Nq][d]     K, V  [B][Hkv][N][d]
- *     pyr   [B][Hkv][P][d] fp32, level-major (level 0 first; node m of level
- *           l covers key blocks [m 2^l, min((m+1) 2^l, nb)))
+ *     pyr   [B][Hkv][P][2][d] bf16, level-major (level 0 first; node m of
+ *           level l covers key blocks [m 2^l, min((m+1) 2^l, nb))). Each node
+ *           mean x is stored as the unevaluated pair hi = RN_bf16(x),
+ *           lo = RN_bf16(x - hi) (row [hi | lo]); x = hi + lo to 2^-17
+ *           relative. This is the operand format of the tensor-core scoring.
  *     idx   [B][Hkv][nqb][topk] int32; gap [B][Hkv][nqb] fp32
  *     lse   [B][Hq][Nq] fp32 (natural log)
  *   Query row t sits at position q_offset + t. Key block j holds positions
@@ -94,7 +97,8 @@ typedef struct pyr_shape {
 PYR_API int pyr_num_levels(const pyr_shape* s);
 
 /* Number of pyramid nodes per (batch, kv head), P = sum over levels of
- * ceil(nb / 2^l); 0 on a bad shape. pyr holds B * Hkv * P * d floats. */
+ * ceil(nb / 2^l); 0 on a bad shape. pyr holds B * Hkv * P * 2 * d bf16
+ * values (4 * B * Hkv * P * d bytes). */
 PYR_API int64_t pyr_num_nodes(const pyr_shape* s);
 
 /* Query blocks per (batch, kv head), nqb; 0 on a bad shape. */
@@ -104,12 +108,27 @@ PYR_API int64_t pyr_num_qblocks(const pyr_shape* s);
  * pyr_build - the key pyramid (PISA abstract: pooling builds O(log N) levels;
  * PHBA A.1.2: a centroid is the fp32 average of the block's key rows).
  *   K   device, [B][Hkv][N][d] in s->dtype (read only).
- *   pyr device, [B][Hkv][P][d] fp32 (written): node (l, m) is the mean of
- *       all keys under it, level-major, level 0 first.
+ *   pyr device, [B][Hkv][P][2][d] bf16 pairs (written): node (l, m) holds
+ *       the mean of all keys under it, accumulated in fp32 and stored as
+ *       (hi, lo); level-major, level 0 first.
  * Reads K once. Returns PYR_OK or a host-side error; nothing is written on
  * error.
  */
-PYR_API int pyr_build(const pyr_shape* s, const void* K, float* pyr, int* dev_status, void* stream);
+PYR_API int pyr_build(const pyr_shape* s, const void* K, void* pyr, int* dev_status, void* stream);
+
+/*
+ * pyr_update - bring a pyramid up to date after the keys at positions
+ * >= from_pos (0 <= from_pos < N) were rewritten, with the shape unchanged;
+ * for example a decode step that writes its new key into the last slot. Only
+ * the nodes whose key range reaches such a position are recomputed (one node
+ * per level for a single position), from K for level 0 and from the children
+ * above; large rewrites (more than 32 blocks) fall back to a full rebuild.
+ *   K   device, [B][Hkv][N][d] in s->dtype (read only).
+ *   pyr device, as written by pyr_build for the same shape (updated in place).
+ * A context that grows past its current block count changes the level sizes
+ * and needs pyr_build.
+ */
+PYR_API int pyr_update(const pyr_shape* s, const void* K, void* pyr, int from_pos, int* dev_status, void* stream);
 
 /*
  * pyr_select - coarse-to-fine LogSumExp top-K key-block selection (PISA
@@ -132,8 +151,8 @@ PYR_API int pyr_build(const pyr_shape* s, const void* K, float* pyr, int* dev_st
  *       the scored levels (+inf if no level dropped one).
  * Scoring accumulates in fp32.
  */
-PYR_API int pyr_select(const pyr_shape* s, const void* Q, const float* pyr, int32_t* idx, float* gap, int* dev_status,
-               void* stream);
+PYR_API int pyr_select(const pyr_shape* s, const void* Q, const void* pyr, int32_t* idx, float* gap,
+                       int* dev_status, void* stream);
 
 /*
  * bsa_forward - causal block-sparse attention (PHBA 3.1, 3.3 and A.1.3:
@@ -162,6 +181,15 @@ PYR_API int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const 
  */
 PYR_API int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
                   int* dev_status, void* stream);
+
+/*
+ * pyr_selftest_wait - exercise the bounded waits the kernels rely on: one
+ * kernel waits on an mbarrier that nothing arrives on and must give up after
+ * its limit (about a second), store PYR_ETIMEOUT in *dev_status (device, must
+ * not be NULL; zeroed by the caller) and return, leaving the context usable.
+ * Not part of the method: a failure-detection check for callers and tests.
+ */
+PYR_API int pyr_selftest_wait(int* dev_status, void* stream);
 
 /* Static, NUL-terminated description of a status code. */
 PYR_API const char* pyr_strerror(int code);

@@ -65,7 +65,7 @@ def test_host_validation_rejects_bad_shapes(field, value, code):
     s.Hkv = 2
     s.Nq = 1024
     setattr(s, field, value)
-    lib = P._lib
+    lib = P._L()
     rc = lib.pyr_build(ctypes.byref(s), 16, 16, None, None)
     assert rc == code, P.strerror(rc)
     rc = lib.pyr_select(ctypes.byref(s), 16, 16, 16, None, None, None)
@@ -76,7 +76,7 @@ def test_host_validation_rejects_null_and_misaligned_pointers():
     import hierarchical_block_sparse_pyr_b200 as P
 
     s = P.shape_of(synth.WORKLOADS[1])
-    lib = P._lib
+    lib = P._L()
     assert lib.pyr_build(ctypes.byref(s), None, 16, None, None) == P.PYR_EINVAL
     assert lib.pyr_build(ctypes.byref(s), 24, 16, None, None) == P.PYR_EINVAL
     assert lib.pyr_select(ctypes.byref(s), 16, 16, None, None, None, None) == P.PYR_EINVAL

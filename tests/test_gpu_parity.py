@@ -40,6 +40,10 @@ CASES = [
               dtype=BF16, seed=25),
     W0.scaled(name="gqa2_bf16_b128", B=1, Hq=4, Hkv=2, N=3000, Nq=3000, d=128, b=128, topk=4, cap=8, dtype=BF16,
               seed=26, needle_mode=synth.NEEDLE_LOGUNIFORM),
+    W0.scaled(name="decode_mha_b128", B=2, Hq=2, Hkv=2, N=9000, Nq=1, q_offset=8999, d=128, b=128, topk=6, cap=12,
+              dtype=BF16, seed=28, n_needle=3, needle_mode=synth.NEEDLE_DECODE),
+    W0.scaled(name="decode_gqa8", B=2, Hq=16, Hkv=2, N=4096, Nq=1, q_offset=4095, d=128, b=64, topk=20, cap=40,
+              dtype=BF16, seed=29, n_needle=4, needle_mode=synth.NEEDLE_DECODE),
     W0.scaled(name="cap_covers_all", B=1, Hq=2, Hkv=2, N=1024, Nq=1024, d=64, b=64, topk=4, cap=16, dtype=F32,
               seed=21),
 ]
@@ -91,7 +95,8 @@ def test_parity_small(w):
               O_o2, lse_o2)
 
 
-@pytest.mark.parametrize("w", [CASES[0], CASES[1], CASES[2], CASES[4], CASES[8]], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [CASES[0], CASES[1], CASES[2], CASES[4], CASES[8], CASES[13], CASES[14]],
+                         ids=lambda w: w.name)
 def test_dense_parity(w):
     Q, K, V, _ = synth.generate(w)
     g = run_gpu(w, Q, K, V, dense=True)
@@ -100,6 +105,38 @@ def test_dense_parity(w):
     O_o, lse_o = oracle.attend(w, Q, K, V, None, rows, dense=True)
     check_out(w, g["O"].double().numpy().reshape(-1, w.d)[rows], g["lse"].double().numpy().reshape(-1)[rows],
               O_o, lse_o)
+
+
+@pytest.mark.parametrize("case", [
+    dict(w=W0.scaled(name="upd_decode", B=2, Hq=4, Hkv=2, N=8192, Nq=8192, d=128, b=64, topk=4, cap=8, dtype=BF16,
+                     seed=30), from_pos=8191),
+    dict(w=W0.scaled(name="upd_ragged_f32", B=1, Hq=2, Hkv=2, N=3000, Nq=3000, d=64, b=32, topk=4, cap=8, dtype=F32,
+                     seed=31), from_pos=2500),
+    dict(w=W0.scaled(name="upd_rebuild", B=1, Hq=2, Hkv=2, N=8192, Nq=8192, d=128, b=64, topk=4, cap=8,
+                     dtype=BF16, seed=32), from_pos=100),
+], ids=lambda c: c["w"].name)
+def test_pyr_update_matches_a_rebuild_and_the_oracle(case):
+    """Rewrite the keys at positions >= from_pos, update the pyramid in place, compare."""
+    import hierarchical_block_sparse_pyr_b200 as P
+    w, from_pos = case["w"], case["from_pos"]
+    Q, K, V, _ = synth.generate(w)
+    s = P.shape_of(w)
+    Kd = K.cuda()
+    buf = P.Buffers(s)
+    P.pyr_build(s, Kd, buf.pyr, buf.status)
+    K2 = K.clone()
+    K2[:, :, from_pos:] = synth.normal(77, 14, K2[:, :, from_pos:].shape, K.dtype) * 2
+    Kd.copy_(K2)
+    P.pyr_update(s, Kd, buf.pyr, from_pos, buf.status)
+    fresh = P.Buffers(s)
+    P.pyr_build(s, Kd, fresh.pyr, fresh.status)
+    torch.cuda.synchronize()
+    assert int(buf.status.item()) == 0
+    upd = P.pyramid_means(buf.pyr).cpu().double().numpy()
+    reb = P.pyramid_means(fresh.pyr).cpu().double().numpy()
+    pyr_o = oracle.pyramid(w, K2, list(range(w.B * w.Hkv)))
+    check_pyramid(upd.reshape(pyr_o.shape), pyr_o)
+    assert np.abs(upd - reb).max() <= 2e-5 * (1 + np.abs(reb).max())
 
 
 def test_all_blocks_selected_equals_dense_on_gpu():
