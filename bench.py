@@ -328,7 +328,7 @@ def count_launches(step):
             step()
             torch.cuda.synchronize()
         names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
-        ours = [n for n in names if any(k in n for k in ("pyr_", "select_kernel", "attn_", "bsa_", "dense_"))]
+        ours = [n for n in names if any(k in n for k in ("pyr_", "select_", "attn_"))]
         return len(ours), sorted(set(ours))
     except Exception as ex:  # profiler unavailable: report unknown
         return None, [f"profiler unavailable: {ex}"]

@@ -24,7 +24,7 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 128;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 4;
 constexpr int kMaxG = 32;
 constexpr int kMaxList = 130;
 
@@ -297,16 +297,20 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const __nv_bfloat
     cg::cluster_group cluster = cg::this_cluster();
     // per row: the global max, the weights 2^(m_r - M) of the CTAs' partial states, 1 / sum
     for (int gg = tid; gg < G; gg += kThreads) {
-      float mr[kMaxCluster], M = -INFINITY;
-      for (int r = 0; r < CS; r++) {
-        mr[r] = *cluster.map_shared_rank(m_run + gg, r);
-        M = fmaxf(M, mr[r]);
+      float mr[kMaxCluster], lr[kMaxCluster], M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; r++) {
+        mr[r] = r < CS ? *cluster.map_shared_rank(m_run + gg, r) : -INFINITY;
+        lr[r] = r < CS ? *cluster.map_shared_rank(l_run + gg, r) : 0.f;
       }
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; r++) M = fmaxf(M, mr[r]);
       float L = 0.f;
-      for (int r = 0; r < CS; r++) {
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; r++) {
         const float w = mr[r] == -INFINITY ? 0.f : ex2(mr[r] - M);
         wts[gg * kMaxCluster + r] = w;
-        L += w * *cluster.map_shared_rank(l_run + gg, r);
+        L += w * lr[r];
       }
       wts[GM * kMaxCluster + gg] = L > 0.f ? 1.f / L : 0.f;
       const size_t orow = ((size_t)bi * g.Hq + hk * G + gg) * g.Nq;
@@ -315,8 +319,12 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const __nv_bfloat
     __syncthreads();
     for (int x = tid; x < G * D; x += kThreads) {
       const int gg = x / D;
+      float part[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; r++) part[r] = r < CS ? *cluster.map_shared_rank(po + x, r) : 0.f;
       float a = 0.f;
-      for (int r = 0; r < CS; r++) a += wts[gg * kMaxCluster + r] * *cluster.map_shared_rank(po + x, r);
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; r++) a += r < CS ? wts[gg * kMaxCluster + r] * part[r] : 0.f;
       const size_t orow = ((size_t)bi * g.Hq + hk * G + gg) * g.Nq;
       O[orow * D + (x - gg * D)] = __float2bfloat16_rn(a * wts[GM * kMaxCluster + gg]);
     }
