@@ -70,6 +70,12 @@ def _load():
         lib.ora_select.restype = ctypes.c_int
         lib.ora_attend.argtypes = [sp, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P]
         lib.ora_attend.restype = ctypes.c_int
+        lib.ora_route_invert.argtypes = [sp, _P, ctypes.c_int32, _P, _P]
+        lib.ora_route_invert.restype = ctypes.c_int
+        lib.ora_attend_bwd_q.argtypes = [sp, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P]
+        lib.ora_attend_bwd_q.restype = ctypes.c_int
+        lib.ora_attend_bwd_kv.argtypes = [sp, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P]
+        lib.ora_attend_bwd_kv.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -184,3 +190,63 @@ def attend(w, Q, K, V, idx, rows, dense: bool = False):
     if rc:
         raise ValueError(f"ora_attend rc={rc}")
     return O, lse
+
+
+# ---- backward (PHBA summary, A.1.2 block-major route metadata; A.1.4 sparse backward) ----
+
+F64 = 2  # oracle-only element type (float64 tensors), for finite-difference pins
+
+
+def _idx_arr(idx):
+    if idx is None:
+        return np.zeros(1, dtype=np.int32)
+    return np.ascontiguousarray(np.asarray(idx, dtype=np.int32))
+
+
+def route_invert(w, idx):
+    """Block-major form of the routes: (offset [U, nb+1], rho [U, nqb*topk]) int32.
+
+    For unit u and key block j, rho[u, offset[u, j]:offset[u, j+1]] lists, ascending,
+    the query blocks qb (row index of idx) whose routes contain j; the diagonal block
+    is not listed. Entries of rho past offset[u, nb] are -1.
+    """
+    idx = _idx_arr(idx)
+    U, nqb = w.B * w.Hkv, num_qblocks(w)
+    nb = (w.N + w.b - 1) // w.b
+    offset = np.zeros((U, nb + 1), dtype=np.int32)
+    rho = np.full((U, max(nqb * w.topk, 1)), -1, dtype=np.int32)
+    for u in range(U):
+        off_u = np.zeros(nb + 1, dtype=np.int32)
+        rho_u = np.full(max(nqb * w.topk, 1), -1, dtype=np.int32)
+        rc = _load().ora_route_invert(ctypes.byref(shape_of(w)), _ptr(idx), u, _ptr(off_u), _ptr(rho_u))
+        if rc == 2:
+            raise ValueError("ora_route_invert: idx lists a block that is not strictly before the query block, or repeats")
+        if rc:
+            raise ValueError(f"ora_route_invert rc={rc}")
+        offset[u], rho[u] = off_u, rho_u
+    return offset, rho
+
+
+def attend_bwd_q(w, Q, K, V, dO, idx, rows, dense: bool = False):
+    """dQ [n, d] float64 of sum(dO * O) for flat query rows ((b*Hq + hq)*Nq + t)."""
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    dQ = np.empty((len(rows), w.d), dtype=np.float64)
+    rc = _load().ora_attend_bwd_q(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(_idx_arr(idx)),
+                                  len(rows), _ptr(rows), 1 if dense else 0, _ptr(dQ))
+    if rc:
+        raise ValueError(f"ora_attend_bwd_q rc={rc}")
+    return dQ
+
+
+def attend_bwd_kv(w, Q, K, V, dO, idx, blocks, dense: bool = False):
+    """(dK, dV) [n, b, d] float64 of sum(dO * O) for key blocks given as (unit, j) pairs."""
+    nb = (w.N + w.b - 1) // w.b
+    blocks = np.asarray(blocks, dtype=np.int64).reshape(-1, 2)
+    flat = np.ascontiguousarray(blocks[:, 0] * nb + blocks[:, 1])
+    dK = np.empty((len(flat), w.b, w.d), dtype=np.float64)
+    dV = np.empty((len(flat), w.b, w.d), dtype=np.float64)
+    rc = _load().ora_attend_bwd_kv(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(_idx_arr(idx)),
+                                   len(flat), _ptr(flat), 1 if dense else 0, _ptr(dK), _ptr(dV))
+    if rc:
+        raise ValueError(f"ora_attend_bwd_kv rc={rc}")
+    return dK, dV

@@ -57,7 +57,7 @@ typedef struct {
   int d;          /* head dim */
   int b;          /* block size (keys per block, query rows per block) */
   int topk, cap;  /* final K and per-level candidate cap */
-  int dtype;      /* 0 = fp32, 1 = bf16 */
+  int dtype;      /* 0 = fp32, 1 = bf16, 2 = fp64 (oracle only: finite-difference pins) */
 } ora_shape;
 
 enum { ORA_OK = 0, ORA_EINVAL = 1, ORA_EBADIDX = 2 };
@@ -66,6 +66,7 @@ enum { ORA_OK = 0, ORA_EINVAL = 1, ORA_EBADIDX = 2 };
 
 static double elem(const void* base, int dtype, int64_t i) {
   if (dtype == 0) return (double)((const float*)base)[i];
+  if (dtype == 2) return ((const double*)base)[i];
   uint32_t u = (uint32_t)((const uint16_t*)base)[i] << 16;
   float f;
   memcpy(&f, &u, 4);
@@ -434,6 +435,194 @@ int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, 
     }
     lse[r] = l;
     free(sc);
+    free(keys);
+  }
+  return bad ? ORA_EBADIDX : ORA_OK;
+}
+
+/* ---- backward: block-major route metadata and gradients ----------------- */
+/*
+ * PHBA summary, A.1.2 "Routing metadata kernels": for the backward pass the
+ * query-centric routes are re-expressed block-major: per key block, the
+ * contiguous range of the query rows that route to it, formed by counting the
+ * assignments per block, prefix-summing the counts and scattering the ids.
+ * Route indices are non-differentiable.
+ * PHBA summary, A.1.4 "Sparse backward kernel": the block-major schedule
+ * enumerates, for each key block, the query rows that attend it; scores and
+ * probabilities are recomputed from the log-sum-exp instead of being stored.
+ *
+ * Readings: rho lists query-block indices qb (the row index into idx, all G
+ * heads of the kv group implied), ascending within each key block's range;
+ * the diagonal block (always attended) is not listed, as in idx. Gradients
+ * are those of the scalar sum_t dO_t . O_t with respect to Q, K and V, with
+ * the routes held fixed; O and the log-sum-exp are recomputed here in double.
+ */
+
+/* offset[0..nb], rho[0..offset[nb]) for one (batch, kv head) unit. */
+int ora_route_invert(const ora_shape* s, const int32_t* idx, int32_t unit, int32_t* offset, int32_t* rho) {
+  if (!s || !idx || !offset || !rho) return ORA_EINVAL;
+  const int64_t nb = num_blocks(s), nqb = ora_num_qblocks(s), first = ora_first_qblock(s);
+  const int32_t* u = idx + (int64_t)unit * nqb * s->topk;
+  /* count the assignments per key block */
+  for (int64_t j = 0; j <= nb; j++) offset[j] = 0;
+  for (int64_t q = 0; q < nqb; q++)
+    for (int k = 0; k < s->topk; k++) {
+      const int64_t j = u[q * s->topk + k];
+      if (j < 0) continue;
+      int rep = 0;
+      for (int k2 = 0; k2 < k; k2++) rep |= (u[q * s->topk + k2] == j);
+      if (j >= first + q || rep) return ORA_EBADIDX;
+      offset[j + 1]++;
+    }
+  /* prefix sums give each block a contiguous range */
+  for (int64_t j = 0; j < nb; j++) offset[j + 1] += offset[j];
+  /* scatter the query blocks in ascending order */
+  int32_t* fill = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nb > 0 ? nb : 1));
+  for (int64_t j = 0; j < nb; j++) fill[j] = offset[j];
+  for (int64_t q = 0; q < nqb; q++)
+    for (int k = 0; k < s->topk; k++) {
+      const int64_t j = u[q * s->topk + k];
+      if (j >= 0) rho[fill[j]++] = (int32_t)q;
+    }
+  free(fill);
+  return ORA_OK;
+}
+
+/* The attended key positions of one query row (routed blocks, then the
+ * diagonal block up to the row's position), as in ora_attend. */
+static int64_t row_keys(const ora_shape* s, const int32_t* idx, int dense, int64_t row, int64_t* keys, int* bad) {
+  const int G = s->Hq / s->Hkv;
+  const int64_t nqb = ora_num_qblocks(s), first = ora_first_qblock(s);
+  const int64_t t = row % s->Nq, bh = row / s->Nq;
+  const int64_t bi = bh / s->Hq, hq = bh % s->Hq, hk = hq / G;
+  const int64_t p = s->q_offset + t, i = p / s->b;
+  int64_t nk = 0;
+  if (dense) {
+    for (int64_t k = 0; k <= p; k++) keys[nk++] = k;
+    return nk;
+  }
+  const int32_t* row_idx = idx + ((bi * s->Hkv + hk) * nqb + (i - first)) * s->topk;
+  for (int k = 0; k < s->topk; k++) {
+    const int64_t j = row_idx[k];
+    if (j < 0) continue;
+    int rep = 0;
+    for (int k2 = 0; k2 < k; k2++) rep |= (row_idx[k2] == j);
+    if (j >= i || rep) {
+      *bad = 1;
+      continue;
+    }
+    for (int64_t x = j * s->b; x < (j + 1) * s->b && x < s->N; x++) keys[nk++] = x;
+  }
+  for (int64_t x = i * s->b; x <= p; x++) keys[nk++] = x;
+  return nk;
+}
+
+/* For one query row: P_k, and dS_k = P_k (dO . v_k - dO . O) over its keys. */
+static void row_grad(const ora_shape* s, const void* Q, const void* K, const void* V, const void* dO, int64_t row,
+                     const int64_t* keys, int64_t nk, double* P, double* dS) {
+  const int d = s->d, G = s->Hq / s->Hkv;
+  const int64_t bh = row / s->Nq, bi = bh / s->Hq, hk = (bh % s->Hq) / G;
+  const int64_t qbase = row * d, kvbase = (bi * s->Hkv + hk) * (int64_t)s->N * d;
+  const double scale = 1.0 / sqrt((double)d);
+  double mx = -INFINITY;
+  for (int64_t k = 0; k < nk; k++) {
+    double dot = 0.0;
+    for (int e = 0; e < d; e++) dot += elem(Q, s->dtype, qbase + e) * elem(K, s->dtype, kvbase + keys[k] * d + e);
+    P[k] = dot * scale;
+    if (P[k] > mx) mx = P[k];
+  }
+  double sum = 0.0;
+  for (int64_t k = 0; k < nk; k++) sum += exp(P[k] - mx);
+  const double lse = mx + log(sum);
+  double D = 0.0; /* dO . O with O = sum_k P_k v_k */
+  for (int64_t k = 0; k < nk; k++) {
+    P[k] = exp(P[k] - lse);
+    double dp = 0.0;
+    for (int e = 0; e < d; e++) dp += elem(dO, s->dtype, qbase + e) * elem(V, s->dtype, kvbase + keys[k] * d + e);
+    dS[k] = dp;
+    D += P[k] * dp;
+  }
+  for (int64_t k = 0; k < nk; k++) dS[k] = P[k] * (dS[k] - D);
+}
+
+/* dQ for the listed flat query rows ((b*Hq + hq)*Nq + t): dQ_t = sum_k dS_k k_k / sqrt(d). */
+int ora_attend_bwd_q(const ora_shape* s, const void* Q, const void* K, const void* V, const void* dO,
+                     const int32_t* idx, int nrows, const int64_t* rows, int dense, double* dQ) {
+  if (!s || !Q || !K || !V || !dO || !rows || !dQ || (!dense && !idx)) return ORA_EINVAL;
+  const int d = s->d, G = s->Hq / s->Hkv;
+  const double scale = 1.0 / sqrt((double)d);
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+  for (int r = 0; r < nrows; r++) {
+    const int64_t p = s->q_offset + rows[r] % s->Nq;
+    const int64_t cap_keys = dense ? p + 1 : (int64_t)(s->topk + 1) * s->b;
+    int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap_keys);
+    double* P = (double*)malloc(sizeof(double) * (size_t)cap_keys);
+    double* dS = (double*)malloc(sizeof(double) * (size_t)cap_keys);
+    const int64_t nk = row_keys(s, idx, dense, rows[r], keys, &bad);
+    row_grad(s, Q, K, V, dO, rows[r], keys, nk, P, dS);
+    const int64_t bh = rows[r] / s->Nq, bi = bh / s->Hq, hk = (bh % s->Hq) / G;
+    const int64_t kvbase = (bi * s->Hkv + hk) * (int64_t)s->N * d;
+    for (int e = 0; e < d; e++) {
+      double acc = 0.0;
+      for (int64_t k = 0; k < nk; k++) acc += dS[k] * elem(K, s->dtype, kvbase + keys[k] * d + e);
+      dQ[(int64_t)r * d + e] = acc * scale;
+    }
+    free(dS);
+    free(P);
+    free(keys);
+  }
+  return bad ? ORA_EBADIDX : ORA_OK;
+}
+
+/* dK and dV of the listed key blocks (entries unit * nb + j): every query row of
+ * every head of the kv group whose keys include a position of block j contributes
+ * dK_x += dS_x q_t / sqrt(d) and dV_x += P_x dO_t. Output [nblk][b][d]; positions
+ * at or beyond N stay zero. */
+int ora_attend_bwd_kv(const ora_shape* s, const void* Q, const void* K, const void* V, const void* dO,
+                      const int32_t* idx, int nblk, const int64_t* blocks, int dense, double* dK, double* dV) {
+  if (!s || !Q || !K || !V || !dO || !blocks || !dK || !dV || (!dense && !idx)) return ORA_EINVAL;
+  const int d = s->d, G = s->Hq / s->Hkv, b = s->b;
+  const int64_t nb = num_blocks(s), nqb = ora_num_qblocks(s), first = ora_first_qblock(s);
+  const double scale = 1.0 / sqrt((double)d);
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+  for (int n = 0; n < nblk; n++) {
+    const int64_t unit = blocks[n] / nb, j = blocks[n] % nb;
+    const int64_t bi = unit / s->Hkv, hk = unit % s->Hkv;
+    double* gk = dK + (int64_t)n * b * d;
+    double* gv = dV + (int64_t)n * b * d;
+    for (int64_t x = 0; x < (int64_t)b * d; x++) gk[x] = gv[x] = 0.0;
+    const int64_t cap_keys = dense ? s->N : (int64_t)(s->topk + 1) * b;
+    int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap_keys);
+    double* P = (double*)malloc(sizeof(double) * (size_t)cap_keys);
+    double* dS = (double*)malloc(sizeof(double) * (size_t)cap_keys);
+    for (int64_t q = 0; q < nqb; q++) {
+      const int64_t i = first + q;
+      /* does query block i attend block j? (the diagonal always; otherwise through its routes) */
+      int uses = dense ? (i >= j) : (i == j);
+      if (!dense && i > j)
+        for (int k = 0; k < s->topk; k++) uses |= (idx[((unit * nqb) + q) * s->topk + k] == j);
+      if (!uses) continue;
+      for (int gg = 0; gg < G; gg++) {
+        const int64_t hq = hk * G + gg;
+        for (int64_t p = (i * b > s->q_offset ? i * b : s->q_offset); p < (i + 1) * b && p < s->q_offset + s->Nq; p++) {
+          const int64_t row = (bi * s->Hq + hq) * s->Nq + (p - s->q_offset);
+          const int64_t nk = row_keys(s, idx, dense, row, keys, &bad);
+          row_grad(s, Q, K, V, dO, row, keys, nk, P, dS);
+          for (int64_t k = 0; k < nk; k++) {
+            if (keys[k] / b != j) continue;
+            const int64_t x = keys[k] - j * b;
+            for (int e = 0; e < d; e++) {
+              gk[x * d + e] += dS[k] * elem(Q, s->dtype, row * d + e) * scale;
+              gv[x * d + e] += P[k] * elem(dO, s->dtype, row * d + e);
+            }
+          }
+        }
+      }
+    }
+    free(dS);
+    free(P);
     free(keys);
   }
   return bad ? ORA_EBADIDX : ORA_OK;
