@@ -4,24 +4,30 @@
 // next finer level; routes only to strictly preceding blocks, -1 padding,
 // PHBA A.1.2).
 //
-// One CTA (4 warps) per (batch, kv head, query block i). Per level:
-//   gather   the <= cap candidate node rows are copied (cp.async, 16 bytes
-//            per thread) straight from the pyramid, which already stores every
-//            mean as a bf16 (hi, lo) pair, to their places in the 128B-swizzled
-//            K-major A operands; the one node that straddles block i
-//            uses the exact mean of its part before i, from the binary
-//            decomposition of [m 2^l, i) into whole finer nodes, split by a
-//            thread into hi + lo;
+// One CTA (4 warps) per (batch, kv head, query block i). The walk is a chain
+// of dependent levels, so the kernel is built for latency: per level it takes
+// four block-wide barriers and one batch of MMAs.
+//   prologue the G*b query rows are staged once by TMA (the N operand); the
+//            start level's candidates are requested at once; the nodes that
+//            straddle block i (one per level) get the exact means of their
+//            parts before i, from the binary decomposition of [m 2^l, i) into
+//            whole finer nodes, stored as (hi, lo) rows in shared memory;
+//   gather   the <= cap candidate rows are copied (cp.async, 16 bytes per
+//            thread) straight from the pyramid, which already stores every
+//            mean as a bf16 (hi, lo) pair, to their places in the
+//            128B-swizzled K-major A operands (the straddling node's row from
+//            shared memory);
 //   score    D[candidate][row] = kbar . q_row on the tensor cores, as
-//            A_hi * Q^T + A_lo * Q^T (M = candidates: 64 or 128, N = the
-//            G*b query rows staged once by TMA, K = d), fp32 accumulation in
-//            tensor memory. Each TMEM lane then holds one candidate's dot
-//            products with every query row, so the LogSumExp over rows is a
-//            per-thread reduction; S = LSE(q.kbar / sqrt(d)) + ln n_valid;
+//            A_hi * Q^T + A_lo * Q^T (M = candidate slots: 64 or 128, N = G*b,
+//            K = d), fp32 accumulation in tensor memory. Each TMEM lane holds
+//            one candidate's dot products with every query row, so the
+//            LogSumExp over rows is a per-thread reduction (one pass, online
+//            max); S = LSE(q.kbar / sqrt(d)) + ln n_valid;
 //   select   a parallel rank count over packed 64-bit keys (order-preserving
 //            score bits over the inverted node index: ties go to the lower
-//            index), keep cap/2 (levels > 0) or topk (level 0), and a warp
-//            scan compacts the surviving nodes' valid children.
+//            index) keeps cap/2 (levels > 0) or topk (level 0); the kept node
+//            of rank r writes its children to candidate slots 2r and 2r + 1
+//            (-1 for a child that does not exist or starts at or after block i).
 // q is exactly representable in bf16, so the only rounding beyond fp32
 // accumulation is the hi/lo split of the means.
 #include "pyr_common.cuh"
@@ -35,9 +41,10 @@ using namespace tc;
 
 constexpr int kThreads = 128;
 constexpr int kMaxCap = 128;
+constexpr int kMaxLevels = 16;  // scored levels: s0 + 1 <= 16 (nb <= 2^15 * cap)
 
 struct SelPlan {
-  int q, a_hi, a_lo, part, keys, cand, kept, misc, bars, total;
+  int q, a_hi, a_lo, ppair, keys, cand, kept, misc, bars, total;
 };
 
 // R: query rows (N of the MMA); MC: candidate rows (M of the MMA); levels: s0 + 1.
@@ -47,24 +54,27 @@ __host__ __device__ inline SelPlan sel_plan(int R, int MC, int levels, int d) {
   p.q = o;     o += R * d * 2;           // [2 halves][R][128 B]
   p.a_hi = o;  o += MC * d * 2;          // [2 halves][MC][128 B]
   p.a_lo = o;  o += MC * d * 2;
-  p.part = o;  o += levels * d * 4;      // straddling-node means, fp32
-  p.keys = o;  o += kMaxCap * 8;
+  p.ppair = o; o += levels * d * 4;      // straddling-node means as (hi, lo) rows, [level][2][d] bf16
+  p.keys = o;  o += (kMaxCap + 2) * 8;
   p.cand = o;  o += kMaxCap * 4;
   p.kept = o;  o += kMaxCap * 4;
-  p.misc = o;  o += 64;                  // nc, gap, tmem slot, abort flag, boundary scores
+  p.misc = o;  o += 64;                  // gap, tmem slot, abort flag, boundary scores
   p.bars = o;  o += 16;                  // q_full, mma_done
   p.total = o + 1024;                    // + alignment slack
   return p;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
 __device__ __forceinline__ float key_score(unsigned long long k) {
   const uint32_t u = (uint32_t)(k >> 32);
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+// Offset of 16-byte chunk q (0..15 hi, 16..31 lo) of candidate slot c inside its
+// 128B-swizzled K-major A operand (two d-halves of MC rows x 128 bytes).
+template <int MC>
+__device__ __forceinline__ int a_chunk_off(int c, int q) {
+  const int h = (q >> 3) & 1, c8 = q & 7;
+  return h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4);
 }
 
 template <int MC>
@@ -79,39 +89,49 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   unsigned char* sQ = smem + L.q;
   unsigned char* sAh = smem + L.a_hi;
   unsigned char* sAl = smem + L.a_lo;
-  float* part = reinterpret_cast<float*>(smem + L.part);
+  unsigned char* ppair = smem + L.ppair;
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem + L.keys);
   int* cand = reinterpret_cast<int*>(smem + L.cand);
   int* kept = reinterpret_cast<int*>(smem + L.kept);
-  int* s_nc = reinterpret_cast<int*>(smem + L.misc);
-  float* s_gap = reinterpret_cast<float*>(smem + L.misc + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc + 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 12);
+  float* s_gap = reinterpret_cast<float*>(smem + L.misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 8);
   float* s_edge = reinterpret_cast<float*>(smem + L.misc + 16);  // [0]: last kept, [1]: first dropped
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bar_mma = bar_q + 1;
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qb = blockIdx.x, unit = blockIdx.y;
   const int bi = unit / g.Hkv, hk = unit % g.Hkv;
   const int i = g.i0 + qb;
   const int p0 = max(i * g.b, g.q_offset);
   const int rb = min((i + 1) * g.b, g.q_offset + g.Nq) - p0;  // valid rows per head
   const int tcols = R <= 64 ? 64 : (R <= 128 ? 128 : 256);
-  // this thread's candidate (TMEM lane): M=128 -> lane t; M=64 -> rows 16w..16w+15 in lanes 32w..32w+15
-  const int my_c = MC == 128 ? threadIdx.x : (lane < 16 ? warp * 16 + lane : -1);
+  // this thread's candidate slot (TMEM lane): M=128 -> lane t; M=64 -> rows 16w..16w+15 in lanes 32w..32w+15
+  const int my_c = MC == 128 ? tid : (lane < 16 ? warp * 16 + lane : -1);
+  const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 256;
+  // the node of level l that straddles block i (its part before i is scored), or -1
+  auto straddler = [&](int l) { return (l > 0 && (i & ((1 << l) - 1)) != 0) ? (i >> l) : -1; };
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     mbar_init(bar_q, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
     *abort_flag = 0;
     *s_gap = __int_as_float(0x7f800000);
-    // start level: every node of level s0 that begins before block i
-    *s_nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  // start level s0: every node that begins before block i, node m in slot m
+  int nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
+  {
+    const int ms = straddler(g.s0);
+    for (int x = tid; x < nc * 32; x += kThreads) {
+      const int c = x >> 5, q = x & 31;
+      if (c == ms) continue;
+      cp_async16(((q < 16) ? sAh : sAl) + a_chunk_off<MC>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+    }
+  }
+  __syncthreads();  // barrier init visible before the TMA uses it
+  if (tid == 0) {
     // the G*b query rows: per head, b/64 boxes of 64 rows x 64 d per d-half
     mbar_expect_tx(bar_q, R * 256);
     for (int gg = 0; gg < g.G; gg++)
@@ -126,179 +146,171 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     tmem_alloc(tmem_slot, tcols);
     tmem_relinquish();
   }
-  // exact means of the straddling node's part before i, levels 1..s0
-  const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 256;
-  for (int e = threadIdx.x; e < 128; e += kThreads) {
+  // exact means of the straddling nodes' parts before i, levels 1..s0, stored as (hi, lo)
+  // rows: [m 2^l, i) is the union of the whole level-(l'-1) nodes (i >> (l'-1)) - 1 for the
+  // set bits l'-1 < l of i; all their loads are issued before any is used
+  {
+    const int e = tid;  // d = 128 = kThreads: one element per thread
+    float v[kMaxLevels];
+#pragma unroll
+    for (int l = 1; l < kMaxLevels; l++)
+      v[l] = (l <= g.s0 && ((i >> (l - 1)) & 1))
+                 ? split_load(pu + (size_t)(g.lvl_off[l - 1] + (i >> (l - 1)) - 1) * 256, 128, e) * (float)(g.b << (l - 1))
+                 : 0.f;
     float acc = 0.f;
-    part[e] = 0.f;
-    for (int l = 1; l <= g.s0; l++) {
-      if ((i >> (l - 1)) & 1)
-        acc += split_load(pu + (size_t)(g.lvl_off[l - 1] + (i >> (l - 1)) - 1) * 256, 128, e) * (float)(g.b << (l - 1));
+    __nv_bfloat16* pp = reinterpret_cast<__nv_bfloat16*>(ppair);
+#pragma unroll
+    for (int l = 1; l < kMaxLevels; l++) {
+      if (l > g.s0) break;
+      acc += v[l];
       const int cnt = i - ((i >> l) << l);
-      part[l * 128 + e] = cnt > 0 ? acc / (float)(cnt * g.b) : 0.f;
+      const float x = cnt > 0 ? acc / (float)(cnt * g.b) : 0.f;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      pp[l * 256 + e] = hi;
+      pp[l * 256 + 128 + e] = __float2bfloat16_rn(x - __bfloat162float(hi));
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  {
+    // the start level's straddling node (slot = its index) from its (hi, lo) row
+    const int ms = straddler(g.s0);
+    if (ms >= 0 && ms < nc && tid < 32)
+      *reinterpret_cast<uint4*>(((tid < 16) ? sAh : sAl) + a_chunk_off<MC>(ms, tid)) =
+          *reinterpret_cast<const uint4*>(ppair + g.s0 * 512 + tid * 16);
+  }
   const uint32_t tD = *tmem_slot;
   const uint32_t my_lane_addr = tD + ((uint32_t)(warp * 32) << 16);
   const float sl2 = rsqrtf((float)g.d) * 1.4426950408889634f;
   const uint32_t idesc = idesc_bf16_f32(MC, R, 0, 0);
+  // shared-memory descriptors of the operands' first K step; the K steps add fixed offsets
+  const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024), dH0 = sdesc_sw128(smem_u32(sAh), 16, 1024),
+                 dL0 = sdesc_sw128(smem_u32(sAl), 16, 1024);
+  const uint32_t q_half = (uint32_t)R * 8, a_half = (uint32_t)MC * 8;  // a d-half, in 16-byte units
   bool ok = true;
-  if (threadIdx.x == 0) ok = mbar_wait(bar_q, 0, abort_flag);
+  if (tid == 0) ok = mbar_wait(bar_q, 0, abort_flag);
   ok = __syncthreads_and(ok);
   int nphase = 0;
   int32_t* out = idx + ((size_t)unit * g.nqb + qb) * g.topk;
 
   for (int l = g.s0; l >= 0 && ok; l--) {
-    const int nc = *s_nc;
     const bool start = (l == g.s0);
-    // ---- gather: every thread copies 16-byte chunks of the candidates' (hi, lo) rows with
-    // cp.async straight to their swizzled places in the A operands (consecutive threads take
-    // consecutive chunks of a row: coalesced, all copies in flight together); the straddling
-    // node's row (at most one per level) is written by warp 1 from the exact partial mean.
-    const int ms = (l > 0 && (i & ((1 << l) - 1)) != 0) ? (i >> l) : -1;  // the straddling node
-    for (int x = threadIdx.x; x < nc * 32; x += kThreads) {
-      const int c = x >> 5, q = x & 31;  // chunk q: 8 elements; 0..15 hi, 16..31 lo
-      const int m = start ? c : cand[c];
-      if (m == ms) continue;
-      const int h = (q >> 3) & 1, c8 = q & 7;
-      unsigned char* dst = ((q < 16) ? sAh : sAl) + h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4);
-      cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
-    }
-    cp_async_wait_all();
-    if (warp == 1 && ms >= 0) {
-      for (int c = 0; c < nc; c++) {
-        if ((start ? c : cand[c]) != ms) continue;
-        const float4 v = *reinterpret_cast<const float4*>(part + l * 128 + lane * 4);
-        const float x[4] = {v.x, v.y, v.z, v.w};
-        float hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-          hi[e] = __bfloat162float(__float2bfloat16_rn(x[e]));
-          lo[e] = x[e] - hi[e];
-        }
-        const int h = lane >> 4, c8 = (lane & 15) >> 1, half8 = (lane & 1) * 8;
-        const int off = h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4) + half8;
-        *reinterpret_cast<uint2*>(sAh + off) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
-        *reinterpret_cast<uint2*>(sAl + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+    // ---- gather (levels below the start): every thread copies 16-byte chunks of the
+    // candidates' (hi, lo) rows with cp.async straight to their swizzled places in the A
+    // operands; the straddling node's row comes from shared memory instead; empty slots
+    // (-1) are left as they are: their D rows are never read
+    if (!start) {
+      const int ms = straddler(l);
+      for (int x = tid; x < nc * 32; x += kThreads) {
+        const int c = x >> 5, q = x & 31;
+        const int m = cand[c];
+        if (m < 0) continue;
+        unsigned char* dst = ((q < 16) ? sAh : sAl) + a_chunk_off<MC>(c, q);
+        if (m == ms)
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
+        else
+          cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
       }
     }
+    cp_async_wait_all();
     fence_proxy_async_smem();
     __syncthreads();
-    // ---- score on the tensor cores
-    if (threadIdx.x == 0) {
+    // ---- score on the tensor cores: D = A_hi Q^T + A_lo Q^T over 8 K steps of 16
+    if (tid == 0) {
       tc_fence_after();
-      const uint32_t aQ = smem_u32(sQ), aH = smem_u32(sAh), aL = smem_u32(sAl);
+#pragma unroll
       for (int kk = 0; kk < 8; kk++) {
-        const uint64_t b = sdesc_sw128(aQ + (kk >> 2) * (R * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t ah = sdesc_sw128(aH + (kk >> 2) * (MC * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t al = sdesc_sw128(aL + (kk >> 2) * (MC * 128) + (kk & 3) * 32, 16, 1024);
-        umma_bf16(tD, ah, b, idesc, kk > 0);
-        umma_bf16(tD, al, b, idesc, 1);
+        const uint32_t oq = (kk >> 2) * q_half + (kk & 3) * 2, oa = (kk >> 2) * a_half + (kk & 3) * 2;
+        umma_bf16(tD, dH0 + oa, dQ0 + oq, idesc, kk > 0);
+        umma_bf16(tD, dL0 + oa, dQ0 + oq, idesc, 1);
       }
       umma_commit(bar_mma);
     }
+    // this slot's node, read before any slot is rewritten below
+    const int my_m = (my_c >= 0 && my_c < nc) ? (start ? my_c : cand[my_c]) : -1;
     ok = mbar_wait(bar_mma, nphase & 1, abort_flag);
     ok = __syncthreads_and(ok);  // block-uniform: the loop below has block-wide barriers
     nphase++;
     if (!ok) break;
     tc_fence_after();
-    // ---- LogSumExp over the valid query rows, one candidate per thread: pass 1 takes the
-    // max of the raw dot products (the positive scale commutes with max), pass 2 re-reads
-    // TMEM and sums 2^(x * scale - max) with packed FMAs and four independent partial sums.
+    // ---- LogSumExp over the valid query rows, one candidate per thread, one pass over
+    // TMEM in batches of 64 columns with an online max (the positive scale commutes with max)
     float m2 = -INFINITY, s2 = 0.f;
     const bool warp_has = MC == 128 ? (warp * 32 < nc) : (warp * 16 < nc);
     if (warp_has) {
       const bool full = (rb == g.b);
-      float v[32];
-      float mx = -INFINITY;
-      for (int c0 = 0; c0 < R; c0 += 32) {
+      float v[64];
+      for (int c0 = 0; c0 < R; c0 += 64) {
         tmem_ld32(my_lane_addr + c0, v);
+        tmem_ld32(my_lane_addr + c0 + 32, v + 32);
         tmem_wait_ld();
         if (!full) {
 #pragma unroll
-          for (int k = 0; k < 32; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
+          for (int k = 0; k < 64; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
         }
-        float a[11];
+        float a[22];
 #pragma unroll
-        for (int k = 0; k < 10; k++) a[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
-        a[10] = fmaxf(v[30], v[31]);
-        mx = fmax3(mx, fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], a[8])),
-                   fmaxf(a[9], a[10]));
-      }
-      m2 = mx * sl2;
-      const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      for (int c0 = 0; c0 < R; c0 += 32) {
-        tmem_ld32(my_lane_addr + c0, v);
-        tmem_wait_ld();
-        if (!full) {
+        for (int k = 0; k < 21; k++) a[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+        a[21] = v[63];
 #pragma unroll
-          for (int k = 0; k < 32; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
-        }
+        for (int k = 0; k < 7; k++) a[k] = fmax3(a[3 * k], a[3 * k + 1], a[3 * k + 2]);
+        const float bm = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[21])) * sl2;
+        const float mn = fmaxf(m2, bm);
+        if (mn == -INFINITY) continue;  // nothing valid yet
+        s2 *= ex2(m2 - mn);  // 0 on the first valid batch (m2 = -inf)
+        m2 = mn;
+        const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int k = 0; k < 16; k++) {
+        for (int k = 0; k < 32; k++) {
           const float2 x = __ffma2_rn(make_float2(v[2 * k], v[2 * k + 1]), scl, off);
           acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(ex2(x.x), ex2(x.y)));
         }
+        const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        s2 += t.x + t.y;
       }
-      const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-      s2 = t.x + t.y;
     }
     tc_fence_before();
-    if (my_c >= 0 && my_c < nc) {
-      const int m = start ? my_c : cand[my_c];
-      const int j0 = m << l;
-      const int j1 = min(min((m + 1) << l, g.nb), i);
+    unsigned long long my_key = 0ull;  // empty slots rank below every node
+    if (my_m >= 0) {
+      const int j0 = my_m << l;
+      const int j1 = min(min((my_m + 1) << l, g.nb), i);
       const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
       const float sc = (m2 + __log2f(s2)) * 0.6931471805599453f + __logf(nval);
-      keys[my_c] = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
+      my_key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)my_m);
     }
-    __syncthreads();
-    // ---- keep the best: rank = number of strictly larger keys
+    if (my_c >= 0 && my_c < nc + 1) keys[my_c] = my_key;  // slot nc: a zero pad for the paired reads
+    const int n_valid = __syncthreads_count(my_m >= 0);
+    // ---- keep the best: rank = number of strictly larger keys; a kept node of rank r puts its
+    // children (those that exist and start before block i; -1 otherwise) in slots 2r, 2r + 1
     const int want = l > 0 ? g.cap / 2 : g.topk;
-    const int keep = min(want, nc);
-    if (my_c >= 0 && my_c < nc) {
-      const unsigned long long k = keys[my_c];
+    const int keep = min(want, n_valid);
+    if (my_m >= 0) {
       int rank = 0;
-      for (int c = 0; c < nc; c++) rank += keys[c] > k;
-      if (rank < keep) kept[rank] = (int)(0xFFFFFFFFu - (uint32_t)(k & 0xFFFFFFFFull));
-      if (rank == keep - 1) s_edge[0] = key_score(k);
-      if (rank == keep) s_edge[1] = key_score(k);
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
+      for (int c = 0; c < (nc + 1) / 2; c++) {
+        const ulonglong2 kv = k2[c];
+        rank += (kv.x > my_key) + (kv.y > my_key);
+      }
+      if (rank < keep) {
+        if (l > 0) {
+          const int c1 = 2 * my_m + 1;
+          cand[2 * rank] = 2 * my_m;
+          cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+        } else {
+          kept[rank] = my_m;
+        }
+      }
+      if (rank == keep - 1) s_edge[0] = key_score(my_key);
+      if (rank == keep) s_edge[1] = key_score(my_key);
     }
     __syncthreads();
-    if (l > 0) {
-      // children of the kept nodes that exist and start before block i, compacted by warp 0
-      if (warp == 0) {
-        if (lane == 0 && keep < nc && keep > 0) *s_gap = fminf(*s_gap, s_edge[0] - s_edge[1]);
-        int base = 0;
-        for (int k0 = 0; k0 < keep; k0 += 32) {
-          const int k = k0 + lane;
-          int m = -1, cnt = 0;
-          if (k < keep) {
-            m = kept[k];
-            cnt = 1 + ((2 * m + 1 < g.lvl_n[l - 1] && ((2 * m + 1) << (l - 1)) < i) ? 1 : 0);
-          }
-          int incl = cnt;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          const int pos = base + incl - cnt;
-          if (cnt > 0) cand[pos] = 2 * m;
-          if (cnt > 1) cand[pos + 1] = 2 * m + 1;
-          base += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) *s_nc = base;
-      }
-      __syncthreads();
-    } else {
+    if (tid == 0 && keep < n_valid && keep > 0) *s_gap = fminf(*s_gap, s_edge[0] - s_edge[1]);
+    nc = 2 * keep;
+    if (l == 0) {
       // the kept blocks in ascending order, then -1
-      if (threadIdx.x == 0 && keep < nc && keep > 0) *s_gap = fminf(*s_gap, s_edge[0] - s_edge[1]);
-      for (int k = threadIdx.x; k < g.topk; k += kThreads) {
+      for (int k = tid; k < g.topk; k += kThreads) {
         if (k < keep) {
           const int m = kept[k];
           int pos = 0;
@@ -309,12 +321,12 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
         }
       }
       __syncthreads();
-      if (gap_out && threadIdx.x == 0) gap_out[(size_t)unit * g.nqb + qb] = *s_gap;
+      if (gap_out && tid == 0) gap_out[(size_t)unit * g.nqb + qb] = *s_gap;
     }
   }
 
   // ---- teardown
-  if (threadIdx.x == 0 && nphase > 0 && !ok) {
+  if (tid == 0 && nphase > 0 && !ok) {
     // the last MMA batch may still be in flight after an abort: let it finish
     umma_commit(bar_mma);
     volatile int no_abort = 0;
@@ -322,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   }
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) report(status, PYR_ETIMEOUT);
+  if (*abort_flag && tid == 0) report(status, PYR_ETIMEOUT);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tD, tcols);
@@ -349,6 +361,7 @@ bool select_tc_supported(const Geo& g) {
   const int R = g.G * g.b;
   if (R != 64 && R != 128 && R != 256) return false;
   if (g.q_offset % g.b != 0) return false;
+  if (g.s0 >= kMaxLevels) return false;
   const int MC = g.cap <= 64 ? 64 : 128;
   return sel_plan(R, MC, g.s0 + 1, 128).total <= 227 * 1024;
 }
