@@ -12,6 +12,9 @@ every call needs CUDA tensors.
     pyr_select(shape, Q, pyr, idx, gap)       coarse-to-fine LogSumExp top-K
     bsa_forward(shape, Q, K, V, idx, O, lse)  causal block-sparse attention
     dense_forward(shape, Q, K, V, O, lse)     dense causal attention
+    bsa_route_invert(shape, idx, offset, rho) routes in block-major form (for the backward)
+    bsa_backward(shape, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV)
+                                              gradients of the block-sparse attention
     forward(Q, K, V, b, topk, cap)            allocate outputs and run all three
 """
 from __future__ import annotations
@@ -28,7 +31,8 @@ PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = ran
 PYR_F32, PYR_BF16 = 0, 1
 
 ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_update", "pyr_select",
-               "bsa_forward", "dense_forward", "pyr_selftest_wait", "pyr_strerror")
+               "bsa_forward", "dense_forward", "bsa_route_invert", "bsa_backward", "pyr_selftest_wait",
+               "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -68,6 +72,10 @@ def _load_lib():
     lib.bsa_forward.restype = ctypes.c_int
     lib.dense_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.dense_forward.restype = ctypes.c_int
+    lib.bsa_route_invert.argtypes = [sp, vp, vp, vp, vp, vp]
+    lib.bsa_route_invert.restype = ctypes.c_int
+    lib.bsa_backward.argtypes = [sp] + [vp] * 15
+    lib.bsa_backward.restype = ctypes.c_int
     lib.pyr_selftest_wait.argtypes = [vp, vp]
     lib.pyr_selftest_wait.restype = ctypes.c_int
     lib.pyr_strerror.argtypes = [ctypes.c_int]
@@ -162,6 +170,18 @@ def dense_forward(s: PyrShape, Q, K, V, O, lse=None, status=None, stream=None):
            "dense_forward")
 
 
+def bsa_route_invert(s: PyrShape, idx, offset, rho, status=None, stream=None):
+    _check(_L().bsa_route_invert(ctypes.byref(s), _dev(idx, "idx"), _dev(offset, "offset"), _dev(rho, "rho"),
+                                 _dev(status, "status", True), _stream(stream)), "bsa_route_invert")
+
+
+def bsa_backward(s: PyrShape, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, status=None, stream=None):
+    args = [_dev(t, n) for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (lse, "lse"), (dO, "dO"), (idx, "idx"),
+                                    (offset, "offset"), (rho, "rho"), (delta, "delta"), (dQ, "dQ"), (dK, "dK"),
+                                    (dV, "dV"))]
+    _check(_L().bsa_backward(ctypes.byref(s), *args, _dev(status, "status", True), _stream(stream)), "bsa_backward")
+
+
 def selftest_wait(status, stream=None):
     """Launch the bounded-wait self-test; status (int32 CUDA tensor) reads PYR_ETIMEOUT afterwards."""
     _check(_L().pyr_selftest_wait(_dev(status, "status"), _stream(stream)), "pyr_selftest_wait")
@@ -181,6 +201,30 @@ class Buffers:
         self.O = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=dt, device=device)
         self.lse = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
+
+
+class BackwardBuffers:
+    """Device buffers of one backward pass (allocated by torch, owned by the caller)."""
+
+    def __init__(self, s: PyrShape, device="cuda"):
+        self.shape = s
+        nqb = num_qblocks(s)
+        nb = (s.N + s.b - 1) // s.b
+        dt = torch.float32 if s.dtype == PYR_F32 else torch.bfloat16
+        self.offset = torch.empty((s.B * s.Hkv, nb + 1), dtype=torch.int32, device=device)
+        self.rho = torch.empty((s.B * s.Hkv, nqb * s.topk), dtype=torch.int32, device=device)
+        self.delta = torch.empty((s.B, s.Hq, s.Nq), dtype=torch.float32, device=device)
+        self.dQ = torch.empty((s.B, s.Hq, s.Nq, s.d), dtype=dt, device=device)
+        self.dK = torch.empty((s.B, s.Hkv, s.N, s.d), dtype=dt, device=device)
+        self.dV = torch.empty((s.B, s.Hkv, s.N, s.d), dtype=dt, device=device)
+
+
+def run_backward(s: PyrShape, Q, K, V, dO, fwd: "Buffers", bwd: BackwardBuffers, stream=None):
+    """Enqueue route inversion and the gradients of the forward pass held in fwd."""
+    bsa_route_invert(s, fwd.idx, bwd.offset, bwd.rho, fwd.status, stream)
+    bsa_backward(s, Q, K, V, fwd.O, fwd.lse, dO, fwd.idx, bwd.offset, bwd.rho, bwd.delta, bwd.dQ, bwd.dK, bwd.dV,
+                 fwd.status, stream)
+    return bwd
 
 
 def pyramid_means(pyr: torch.Tensor) -> torch.Tensor:

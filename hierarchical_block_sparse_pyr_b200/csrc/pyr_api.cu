@@ -141,6 +141,36 @@ int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* 
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
 }
 
+int bsa_route_invert(const pyr_shape* s, const int32_t* idx, int32_t* offset, int32_t* rho, int* dev_status,
+                     void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!idx || !offset || !rho || !aligned16(idx) || ((uintptr_t)offset & 3u) || ((uintptr_t)rho & 3u))
+    return PYR_EINVAL;
+  return launch_status(pyr::launch_route_invert(g, idx, offset, rho, dev_status, (cudaStream_t)stream));
+}
+
+int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const void* V, const void* O, const float* lse,
+                 const void* dO, const int32_t* idx, const int32_t* offset, const int32_t* rho, float* delta,
+                 void* dQ, void* dK, void* dV, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  const void* need[] = {Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV};
+  for (const void* p : need)
+    if (!p) return PYR_EINVAL;
+  const void* vec[] = {Q, K, V, O, dO, dQ, dK, dV, idx};
+  for (const void* p : vec)
+    if (!aligned16(p)) return PYR_EINVAL;
+  if (((uintptr_t)lse & 3u) || ((uintptr_t)delta & 3u) || ((uintptr_t)offset & 3u) || ((uintptr_t)rho & 3u))
+    return PYR_EINVAL;
+  if (s->q_offset != 0 || s->Nq != s->N) return PYR_EUNSUPPORTED;
+  (void)dev_status;
+  return launch_status(pyr::launch_backward_simt(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV,
+                                                 (cudaStream_t)stream));
+}
+
 const char* pyr_strerror(int code) {
   switch (code) {
     case PYR_OK: return "ok";

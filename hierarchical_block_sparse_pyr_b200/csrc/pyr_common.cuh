@@ -73,6 +73,11 @@ cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* p
 bool attn_tc_supported(const Geo& g);
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
                            void* O, float* lse, int* status, cudaStream_t st);
+cudaError_t launch_route_invert(const Geo& g, const int32_t* idx, int32_t* offset, int32_t* rho, int* status,
+                                cudaStream_t st);
+cudaError_t launch_backward_simt(const Geo& g, const void* Q, const void* K, const void* V, const void* O,
+                                 const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
+                                 const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, cudaStream_t st);
 cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
                              int dense, void* O, float* lse, int* status, cudaStream_t st);
 

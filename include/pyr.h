@@ -183,6 +183,52 @@ PYR_API int dense_forward(const pyr_shape* s, const void* Q, const void* K, cons
                   int* dev_status, void* stream);
 
 /*
+ * bsa_route_invert - the routes in block-major form, for the backward pass
+ * (PHBA summary, A.1.2 "Routing metadata kernels": count the assignments per
+ * key block, prefix-sum the counts into contiguous ranges, scatter the query
+ * ids into them; route indices carry no gradient).
+ *   idx    device, [B][Hkv][nqb][topk] int32, as written by pyr_select.
+ *   offset device, [B*Hkv][nb + 1] int32 (written): unit u's key block j owns
+ *          rho[u][offset[u][j] .. offset[u][j+1]).
+ *   rho    device, [B*Hkv][nqb * topk] int32 (written): in each range, the
+ *          query blocks qb (row index of idx) whose routes list j, ascending;
+ *          entries past offset[u][nb] are -1. The query's own (diagonal)
+ *          block is never listed.
+ * A route that is not strictly before its query block, or that repeats in
+ * its row, is left out and PYR_EBADIDX is reported in *dev_status. The result
+ * does not depend on thread timing (each range is sorted).
+ */
+PYR_API int bsa_route_invert(const pyr_shape* s, const int32_t* idx, int32_t* offset, int32_t* rho, int* dev_status,
+                             void* stream);
+
+/*
+ * bsa_backward - gradients of causal block-sparse attention (PHBA summary,
+ * A.1.4 "Sparse backward kernel": a block-major schedule walks, for every key
+ * block, the query rows that attend it; scores and probabilities are
+ * recomputed on chip from the saved log-sum-exp). With the routes held fixed
+ * and L = sum over rows of dO_t . O_t:
+ *   P_tk = exp(q_t . k_k / sqrt(d) - lse_t),  D_t = dO_t . O_t,
+ *   dS_tk = P_tk (dO_t . v_k - D_t),
+ *   dQ_t = sum_k dS_tk k_k / sqrt(d),  dK_k = sum_t dS_tk q_t / sqrt(d),
+ *   dV_k = sum_t P_tk dO_t,
+ * t running over the rows of all G heads of the key's kv head.
+ *   Q, K, V, O, dO device, in s->dtype (O and lse as written by bsa_forward).
+ *   lse    device, [B][Hq][Nq] fp32.
+ *   idx    device, as given to bsa_forward.
+ *   offset, rho device, as written by bsa_route_invert from the same idx.
+ *   delta  device, [B][Hq][Nq] fp32 workspace (overwritten with D_t).
+ *   dQ     device, [B][Hq][Nq][d] in s->dtype (written).
+ *   dK, dV device, [B][Hkv][N][d] in s->dtype (written, zero where no row
+ *          attends).
+ * Supported: whole-sequence prefill (q_offset == 0 and Nq == N); other
+ * shapes return PYR_EUNSUPPORTED. Accumulation is fp32.
+ */
+PYR_API int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const void* V, const void* O,
+                         const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
+                         const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, int* dev_status,
+                         void* stream);
+
+/*
  * pyr_selftest_wait - exercise the bounded waits the kernels rely on: one
  * kernel waits on an mbarrier that nothing arrives on and must give up after
  * its limit (about a second), store PYR_ETIMEOUT in *dev_status (device, must

@@ -143,5 +143,14 @@ def normal(seed: int, stream: int, shape, dtype=torch.float32, scale: float = 1.
     return t
 
 
+STREAM_DO = 6  # the upstream gradient dO of the backward pass (streams 0-5 are the forward inputs)
+
+
+def grad_output(w: Workload, pin: bool = False) -> torch.Tensor:
+    """Seeded upstream gradient dO [B, Hq, Nq, d] ~ N(0, 1) in the workload dtype (CPU tensor)."""
+    t = normal(w.seed, STREAM_DO, (w.B, w.Hq, w.Nq, w.d), w.torch_dtype)
+    return t.pin_memory() if pin else t
+
+
 def normal_np(seed: int, stream: int, shape, scale: float = 1.0) -> np.ndarray:
     return normal(seed, stream, shape, torch.float32, scale).double().numpy()
