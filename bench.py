@@ -287,6 +287,33 @@ def time_dense(P, s, w, Q, K, V, buf, stream, steps, warmup):
     return {"ms": round(ms, 4), "tflops": round(dense_flops(w) / (ms * 1e-3) / 1e12, 2)}
 
 
+def time_backward(P, s, w, Q, K, V, buf, stream, steps, warmup):
+    """Event-timed backward (route inversion + gradients) of the forward pass held in buf.
+
+    Algorithmic FLOPs: 8 d per attended (query, key) pair (S and dP recomputed, dQ, dK, dV products).
+    """
+    dO = synth.grad_output(w).cuda()
+    bwd = P.BackwardBuffers(s)
+    P.run(s, Q, K, V, buf, stream)
+    for _ in range(max(1, warmup)):
+        P.run_backward(s, Q, K, V, dO, buf, bwd, stream)
+    torch.cuda.synchronize()
+    steps = max(2, min(steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        P.run_backward(s, Q, K, V, dO, buf, bwd, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {buf.status.item()}")
+    ms = e0.elapsed_time(e1) / steps
+    flops = 2 * work_counts(w)["att_flops"]
+    del bwd, dO
+    return {"ms": round(ms, 4), "algorithmic_tflop": round(flops / 1e12, 4),
+            "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "path": "tcgen05 (bf16, d=128, b in {64, 128}) else fp32 CUDA cores"}
+
+
 def break_even(args, w):
     """Sparse step (pyramid + selection + attention) vs dense causal attention over context lengths."""
     import hierarchical_block_sparse_pyr_b200 as P
@@ -428,6 +455,8 @@ def run_ours(args, w, rank, world, local_rank):
         raise RuntimeError(f"device status {buf.status.item()}")
 
     dense = time_dense(P, s, w, Q, K, V, buf, stream, args.steps, args.warmup)
+    backward = (time_backward(P, s, w, Q, K, V, buf, stream, args.steps, args.warmup)
+                if args.backward and not w.decode else None)
 
     wc = work_counts(w)
     peaks = load_peaks()
@@ -479,6 +508,7 @@ def run_ours(args, w, rank, world, local_rank):
         "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
                     for k, v in kernels.items()},
         "dense": dict(dense, speedup_of_sparse_step=round(dense["ms"] / ms_step, 3)),
+        **({"backward": backward} if backward else {}),
         "kernel_names": kernel_names,
         "clocks": clk,
         "peaks_source": peaks["source"],
@@ -572,6 +602,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward pass (route inversion + gradients) of the forward step")
     ap.add_argument("--break-even", action="store_true",
                     help="sweep the context length and report where the sparse step beats dense attention")
     ap.add_argument("--n", type=int, default=None,

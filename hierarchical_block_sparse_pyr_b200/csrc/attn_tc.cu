@@ -50,7 +50,7 @@ struct Plan {
   static constexpr int kKV = kQ + MT * 32768;          // K ring: NS x [2][64][128 B], then V ring
   static constexpr int kV = kKV + NS * 16384;
   static constexpr int kBar = kV + NS * 16384;         // mbarriers
-  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 2;
+  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;    // tmem slot, abort flag, tile count
   static constexpr int kTiles = kMisc + 16;            // tile entries: (block << 4) | modes
   static constexpr int kEnd = kTiles + kMaxTiles * 4;
@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   uint64_t* bar_p_full = bar_s_full + 2;    // [2]
   uint64_t* bar_o = bar_p_full + 2;
   uint64_t* bar_drain = bar_o + 1;
+  uint64_t* bar_done = bar_drain + 1;  // every MMA of the CTA finished (one phase)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
   int* s_ntiles = reinterpret_cast<int*>(smem + PL::kMisc + 8);
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     }
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
+    mbar_init(bar_done, 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -296,6 +298,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
           issued++;
         }
       }
+      if (ok) umma_commit(bar_done);  // after the last P.V: the epilogue may read O
       if (issued > 0) {
         // every MMA issued so far must finish before the CTA frees its tensor memory
         umma_commit(bar_drain);
@@ -406,7 +409,9 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
       if (lane == 0) mbar_arrive(bar_p_full + sb);
     }
     // ---- epilogue ----
-    if (ok) ok = warp_wait(bar_o, (T - 1) & 1, abort_flag);
+    // the last P.V: wait on the one-phase barrier, not on bar_o, whose parity can alias when the
+    // P.V of tile T-2 is still in flight (s_full of tile T-1 only guarantees P.V of tile T-3)
+    if (ok) ok = warp_wait(bar_done, 0, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;

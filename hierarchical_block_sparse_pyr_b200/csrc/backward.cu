@@ -283,7 +283,7 @@ inline int grid_for(int64_t n, int threads) {
 template <typename T, int DPL>
 cudaError_t launch_grads(const Geo& g, const void* Q, const void* K, const void* V, const void* O, const float* lse,
                          const void* dO, const int32_t* idx, const int32_t* offset, const int32_t* rho, float* delta,
-                         void* dQ, void* dK, void* dV, cudaStream_t st) {
+                         void* dQ, void* dK, void* dV, int parts, cudaStream_t st) {
   const int64_t rows = (int64_t)g.B * g.Hq * g.Nq, keys = (int64_t)g.B * g.Hkv * g.N;
   const unsigned rgrid = (unsigned)((rows + kWarpsPerCta - 1) / kWarpsPerCta);
   const unsigned kgrid = (unsigned)((keys + kWarpsPerCta - 1) / kWarpsPerCta);
@@ -291,10 +291,13 @@ cudaError_t launch_grads(const Geo& g, const void* Q, const void* K, const void*
   const T* k = static_cast<const T*>(K);
   const T* v = static_cast<const T*>(V);
   const T* d = static_cast<const T*>(dO);
-  bwd_delta_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(static_cast<const T*>(O), d, delta, g);
-  bwd_dq_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(q, k, v, d, lse, delta, idx, static_cast<T*>(dQ), g);
-  bwd_dkdv_kernel<T, DPL><<<kgrid, kWarpsPerCta * 32, 0, st>>>(q, k, v, d, lse, delta, offset, rho,
-                                                               static_cast<T*>(dK), static_cast<T*>(dV), g);
+  if (parts & kBwdDelta)
+    bwd_delta_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(static_cast<const T*>(O), d, delta, g);
+  if (parts & kBwdDq)
+    bwd_dq_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(q, k, v, d, lse, delta, idx, static_cast<T*>(dQ), g);
+  if (parts & kBwdDkdv)
+    bwd_dkdv_kernel<T, DPL><<<kgrid, kWarpsPerCta * 32, 0, st>>>(q, k, v, d, lse, delta, offset, rho,
+                                                                 static_cast<T*>(dK), static_cast<T*>(dV), g);
   return cudaGetLastError();
 }
 
@@ -314,14 +317,16 @@ cudaError_t launch_route_invert(const Geo& g, const int32_t* idx, int32_t* offse
 
 cudaError_t launch_backward_simt(const Geo& g, const void* Q, const void* K, const void* V, const void* O,
                                  const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
-                                 const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, cudaStream_t st) {
+                                 const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, int parts,
+                                 cudaStream_t st) {
   if (g.dtype == PYR_F32) {
-    if (g.d == 64) return launch_grads<float, 2>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, st);
-    return launch_grads<float, 4>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, st);
+    if (g.d == 64)
+      return launch_grads<float, 2>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, parts, st);
+    return launch_grads<float, 4>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, parts, st);
   }
   if (g.d == 64)
-    return launch_grads<__nv_bfloat16, 2>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, st);
-  return launch_grads<__nv_bfloat16, 4>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, st);
+    return launch_grads<__nv_bfloat16, 2>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, parts, st);
+  return launch_grads<__nv_bfloat16, 4>(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, parts, st);
 }
 
 }  // namespace pyr

@@ -166,9 +166,17 @@ int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const void* V
   if (((uintptr_t)lse & 3u) || ((uintptr_t)delta & 3u) || ((uintptr_t)offset & 3u) || ((uintptr_t)rho & 3u))
     return PYR_EINVAL;
   if (s->q_offset != 0 || s->Nq != s->N) return PYR_EUNSUPPORTED;
-  (void)dev_status;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (pyr::backward_tc_supported(g)) {
+    cudaError_t e = pyr::launch_backward_simt(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV,
+                                              pyr::kBwdDelta, st);
+    if (e == cudaSuccess) e = pyr::launch_backward_dq_tc(g, Q, K, V, dO, lse, delta, idx, dQ, dev_status, st);
+    if (e == cudaSuccess)
+      e = pyr::launch_backward_dkdv_tc(g, Q, K, V, dO, lse, delta, offset, rho, dK, dV, dev_status, st);
+    return launch_status(e);
+  }
   return launch_status(pyr::launch_backward_simt(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV,
-                                                 (cudaStream_t)stream));
+                                                 pyr::kBwdDelta | pyr::kBwdDq | pyr::kBwdDkdv, st));
 }
 
 const char* pyr_strerror(int code) {

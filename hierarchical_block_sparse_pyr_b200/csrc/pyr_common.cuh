@@ -75,9 +75,19 @@ cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const voi
                            void* O, float* lse, int* status, cudaStream_t st);
 cudaError_t launch_route_invert(const Geo& g, const int32_t* idx, int32_t* offset, int32_t* rho, int* status,
                                 cudaStream_t st);
+// parts of the SIMT backward to launch (bit mask)
+constexpr int kBwdDelta = 1, kBwdDq = 2, kBwdDkdv = 4;
 cudaError_t launch_backward_simt(const Geo& g, const void* Q, const void* K, const void* V, const void* O,
                                  const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
-                                 const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, cudaStream_t st);
+                                 const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, int parts,
+                                 cudaStream_t st);
+bool backward_tc_supported(const Geo& g);
+cudaError_t launch_backward_dkdv_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
+                                    const float* lse, const float* delta, const int32_t* offset, const int32_t* rho,
+                                    void* dK, void* dV, int* status, cudaStream_t st);
+cudaError_t launch_backward_dq_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
+                                  const float* lse, const float* delta, const int32_t* idx, void* dQ, int* status,
+                                  cudaStream_t st);
 cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
                              int dense, void* O, float* lse, int* status, cudaStream_t st);
 

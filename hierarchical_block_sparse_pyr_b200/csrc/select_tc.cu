@@ -43,19 +43,30 @@ constexpr int kThreads = 128;
 constexpr int kMaxCap = 128;
 constexpr int kMaxLevels = 16;  // scored levels: s0 + 1 <= 16 (nb <= 2^15 * cap)
 
-struct SelPlan {
-  int q, a_hi, a_lo, ppair, keys, cand, kept, misc, bars, total;
+// Candidate rows of the scoring MMA. A candidate's mean is the pair (hi, lo); both rows go
+// into the same A operand, in the same quarter of the M rows (so in the same warp's TMEM
+// lanes): quarter q holds H = MC/8 candidates, their hi rows first, then their lo rows.
+// One tile of MC rows scores CPT = MC/2 candidates; NT tiles cover the cap.
+template <int MC, int NT>
+struct SelCfg {
+  static constexpr int CPT = MC / 2;        // candidates per tile
+  static constexpr int H = MC / 8;          // candidates per quarter (TMEM lanes 0..H-1: hi, H..2H-1: lo)
+  static constexpr int kATile = MC * 256;   // one tile: [2 d-halves][MC rows][128 B]
+  static constexpr int kMinBlocks = MC == 64 ? 5 : 2;
 };
 
-// R: query rows (N of the MMA); MC: candidate rows (M of the MMA); levels: s0 + 1.
-__host__ __device__ inline SelPlan sel_plan(int R, int MC, int levels, int d) {
+struct SelPlan {
+  int q, a, ppair, keys, cand, kept, misc, bars, total;
+};
+
+// R: query rows (N of the MMA); a_bytes: the A tiles; levels: s0 + 1.
+__host__ __device__ inline SelPlan sel_plan(int R, int a_bytes, int levels, int d) {
   SelPlan p;
   int o = 0;
   p.q = o;     o += R * d * 2;           // [2 halves][R][128 B]
-  p.a_hi = o;  o += MC * d * 2;          // [2 halves][MC][128 B]
-  p.a_lo = o;  o += MC * d * 2;
+  p.a = o;     o += a_bytes;             // NT x [2 halves][MC][128 B]
   p.ppair = o; o += levels * d * 4;      // straddling-node means as (hi, lo) rows, [level][2][d] bf16
-  p.keys = o;  o += (kMaxCap + 2) * 8;
+  p.keys = o;  o += (kMaxCap + 8) * 8;
   p.cand = o;  o += kMaxCap * 4;
   p.kept = o;  o += kMaxCap * 4;
   p.misc = o;  o += 64;                  // gap, tmem slot, abort flag, boundary scores
@@ -69,26 +80,30 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
   return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
 
-// Offset of 16-byte chunk q (0..15 hi, 16..31 lo) of candidate slot c inside its
-// 128B-swizzled K-major A operand (two d-halves of MC rows x 128 bytes).
-template <int MC>
+// Byte offset, inside the A tiles, of 16-byte chunk q (0..15: hi elements 8q..8q+7;
+// 16..31: the same elements of lo) of candidate slot c (128B-swizzled, K-major).
+template <int MC, int NT>
 __device__ __forceinline__ int a_chunk_off(int c, int q) {
-  const int h = (q >> 3) & 1, c8 = q & 7;
-  return h * (MC * 128) + (c >> 3) * 1024 + (c & 7) * 128 + ((c8 ^ (c & 7)) << 4);
+  using C = SelCfg<MC, NT>;
+  const int t = c / C::CPT, cc = c - t * C::CPT;
+  const int quarter = cc / C::H, w = cc - quarter * C::H;
+  const int row = quarter * (MC / 4) + (q >= 16 ? C::H : 0) + w;
+  const int q16 = q & 15, h = q16 >> 3, c8 = q16 & 7;
+  return t * C::kATile + h * (MC * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((c8 ^ (row & 7)) << 4);
 }
 
-template <int MC>
-__global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                             const __nv_bfloat16* __restrict__ pyr, int32_t* __restrict__ idx,
-                                                             float* __restrict__ gap_out, int* status, Geo g) {
+template <int MC, int NT>
+__global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
+    select_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __nv_bfloat16* __restrict__ pyr,
+                     int32_t* __restrict__ idx, float* __restrict__ gap_out, int* status, Geo g) {
+  using C = SelCfg<MC, NT>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int R = g.G * g.b;  // query rows of a full block (N of the MMA)
-  const SelPlan L = sel_plan(R, MC, g.s0 + 1, 128);
+  const SelPlan L = sel_plan(R, NT * C::kATile, g.s0 + 1, 128);
   unsigned char* sQ = smem + L.q;
-  unsigned char* sAh = smem + L.a_hi;
-  unsigned char* sAl = smem + L.a_lo;
+  unsigned char* sA = smem + L.a;
   unsigned char* ppair = smem + L.ppair;
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem + L.keys);
   int* cand = reinterpret_cast<int*>(smem + L.cand);
@@ -106,11 +121,13 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   const int i = g.i0 + qb;
   const int p0 = max(i * g.b, g.q_offset);
   const int rb = min((i + 1) * g.b, g.q_offset + g.Nq) - p0;  // valid rows per head
-  const int tcols = R <= 64 ? 64 : (R <= 128 ? 128 : 256);
-  // this thread's candidate slot (TMEM lane): M=128 -> lane t; M=64 -> rows 16w..16w+15 in lanes 32w..32w+15
-  const int my_c = MC == 128 ? tid : (lane < 16 ? warp * 16 + lane : -1);
+  const int tcols = NT * R <= 64 ? 64 : (NT * R <= 128 ? 128 : (NT * R <= 256 ? 256 : 512));
+  // scoring role of this thread: TMEM lane `lane` of warp `warp` holds, in each tile t, the hi
+  // (role 0) or lo (role 1) dot products of candidate t*CPT + warp*H + (lane % H)
+  const bool scorer = lane < 2 * C::H;
+  const int role = (lane / C::H) & 1;
+  const int my_cq = warp * C::H + (lane % C::H);  // candidate within a tile
   const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 256;
-  // the node of level l that straddles block i (its part before i is scored), or -1
   auto straddler = [&](int l) { return (l > 0 && (i & ((1 << l) - 1)) != 0) ? (i >> l) : -1; };
 
   if (tid == 0) {
@@ -127,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     for (int x = tid; x < nc * 32; x += kThreads) {
       const int c = x >> 5, q = x & 31;
       if (c == ms) continue;
-      cp_async16(((q < 16) ? sAh : sAl) + a_chunk_off<MC>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+      cp_async16(sA + a_chunk_off<MC, NT>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
     }
   }
   __syncthreads();  // barrier init visible before the TMA uses it
@@ -177,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     // the start level's straddling node (slot = its index) from its (hi, lo) row
     const int ms = straddler(g.s0);
     if (ms >= 0 && ms < nc && tid < 32)
-      *reinterpret_cast<uint4*>(((tid < 16) ? sAh : sAl) + a_chunk_off<MC>(ms, tid)) =
+      *reinterpret_cast<uint4*>(sA + a_chunk_off<MC, NT>(ms, tid)) =
           *reinterpret_cast<const uint4*>(ppair + g.s0 * 512 + tid * 16);
   }
   const uint32_t tD = *tmem_slot;
@@ -185,9 +202,8 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   const float sl2 = rsqrtf((float)g.d) * 1.4426950408889634f;
   const uint32_t idesc = idesc_bf16_f32(MC, R, 0, 0);
   // shared-memory descriptors of the operands' first K step; the K steps add fixed offsets
-  const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024), dH0 = sdesc_sw128(smem_u32(sAh), 16, 1024),
-                 dL0 = sdesc_sw128(smem_u32(sAl), 16, 1024);
-  const uint32_t q_half = (uint32_t)R * 8, a_half = (uint32_t)MC * 8;  // a d-half, in 16-byte units
+  const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024), dA0 = sdesc_sw128(smem_u32(sA), 16, 1024);
+  const uint32_t q_half = (uint32_t)R * 8;  // a d-half of Q, in 16-byte units
   bool ok = true;
   if (tid == 0) ok = mbar_wait(bar_q, 0, abort_flag);
   ok = __syncthreads_and(ok);
@@ -198,15 +214,15 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     const bool start = (l == g.s0);
     // ---- gather (levels below the start): every thread copies 16-byte chunks of the
     // candidates' (hi, lo) rows with cp.async straight to their swizzled places in the A
-    // operands; the straddling node's row comes from shared memory instead; empty slots
-    // (-1) are left as they are: their D rows are never read
+    // operand; the straddling node's row comes from shared memory instead; empty slots (-1)
+    // are left as they are: their D rows are never read
     if (!start) {
       const int ms = straddler(l);
       for (int x = tid; x < nc * 32; x += kThreads) {
         const int c = x >> 5, q = x & 31;
         const int m = cand[c];
         if (m < 0) continue;
-        unsigned char* dst = ((q < 16) ? sAh : sAl) + a_chunk_off<MC>(c, q);
+        unsigned char* dst = sA + a_chunk_off<MC, NT>(c, q);
         if (m == ms)
           *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
         else
@@ -216,90 +232,117 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
     cp_async_wait_all();
     fence_proxy_async_smem();
     __syncthreads();
-    // ---- score on the tensor cores: D = A_hi Q^T + A_lo Q^T over 8 K steps of 16
+    const int ntiles = (nc + C::CPT - 1) / C::CPT;  // tiles holding at least one candidate
+    // ---- score on the tensor cores: D_t = A_t Q^T (hi and lo rows of the candidates of
+    // tile t), 8 K steps of 16 per tile
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; kk++) {
-        const uint32_t oq = (kk >> 2) * q_half + (kk & 3) * 2, oa = (kk >> 2) * a_half + (kk & 3) * 2;
-        umma_bf16(tD, dH0 + oa, dQ0 + oq, idesc, kk > 0);
-        umma_bf16(tD, dL0 + oa, dQ0 + oq, idesc, 1);
+      for (int t = 0; t < NT; t++) {
+        if (t >= ntiles) break;
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++) {
+          const uint32_t oq = (kk >> 2) * q_half + (kk & 3) * 2;
+          const uint32_t oa = (t * C::kATile + (kk >> 2) * (MC * 128)) / 16 + (kk & 3) * 2;
+          umma_bf16(tD + t * R, dA0 + oa, dQ0 + oq, idesc, kk > 0);
+        }
       }
       umma_commit(bar_mma);
     }
-    // this slot's node, read before any slot is rewritten below
-    const int my_m = (my_c >= 0 && my_c < nc) ? (start ? my_c : cand[my_c]) : -1;
+    // this thread's slot (rank phase: slot = tid) and its node, read before any slot is rewritten
+    const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
     ok = mbar_wait(bar_mma, nphase & 1, abort_flag);
     ok = __syncthreads_and(ok);  // block-uniform: the loop below has block-wide barriers
     nphase++;
     if (!ok) break;
     tc_fence_after();
-    // ---- LogSumExp over the valid query rows, one candidate per thread, one pass over
-    // TMEM in batches of 64 columns with an online max (the positive scale commutes with max)
-    float m2 = -INFINITY, s2 = 0.f;
-    const bool warp_has = MC == 128 ? (warp * 32 < nc) : (warp * 16 < nc);
-    if (warp_has) {
-      const bool full = (rb == g.b);
+    // ---- LogSumExp over the valid query rows. The two lanes of a candidate (hi, lo) swap
+    // halves of every 64-column batch with one shuffle each, so that each holds hi + lo for 32
+    // columns; each keeps an online max and sum over its columns, and the pair merges at the end
+    const bool full = (rb == g.b);
+#pragma unroll 1
+    for (int t = 0; t < ntiles; t++) {
+      const int c = t * C::CPT + my_cq;
+      if (!__any_sync(0xffffffffu, scorer && c < nc)) continue;  // warp-uniform
+      float m2 = -INFINITY, s2 = 0.f;
       float v[64];
       for (int c0 = 0; c0 < R; c0 += 64) {
-        tmem_ld32(my_lane_addr + c0, v);
-        tmem_ld32(my_lane_addr + c0 + 32, v + 32);
+        tmem_ld32(my_lane_addr + t * R + c0, v);
+        tmem_ld32(my_lane_addr + t * R + c0 + 32, v + 32);
         tmem_wait_ld();
+        float x[32];
+#pragma unroll
+        for (int k = 0; k < 32; k++) {
+          const float send = role ? v[k] : v[32 + k];
+          const float recv = __shfl_xor_sync(0xffffffffu, send, C::H);
+          x[k] = (role ? v[32 + k] : v[k]) + recv;
+        }
+        const int colb = c0 + role * 32;  // first column of this lane's half
         if (!full) {
 #pragma unroll
-          for (int k = 0; k < 64; k++) v[k] = ((c0 + k) % g.b) < rb ? v[k] : -INFINITY;
+          for (int k = 0; k < 32; k++) x[k] = ((colb + k) % g.b) < rb ? x[k] : -INFINITY;
         }
-        float a[22];
+        float a[11];
 #pragma unroll
-        for (int k = 0; k < 21; k++) a[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
-        a[21] = v[63];
-#pragma unroll
-        for (int k = 0; k < 7; k++) a[k] = fmax3(a[3 * k], a[3 * k + 1], a[3 * k + 2]);
-        const float bm = fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[21])) * sl2;
+        for (int k = 0; k < 10; k++) a[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+        a[10] = fmaxf(x[30], x[31]);
+        const float bm =
+            fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], fmax3(a[8], a[9], a[10]))) * sl2;
         const float mn = fmaxf(m2, bm);
-        if (mn == -INFINITY) continue;  // nothing valid yet
-        s2 *= ex2(m2 - mn);  // 0 on the first valid batch (m2 = -inf)
+        if (mn == -INFINITY) continue;  // nothing valid yet in this lane's columns
+        s2 *= ex2(m2 - mn);             // 0 on the first valid batch (m2 = -inf)
         m2 = mn;
         const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int k = 0; k < 32; k++) {
-          const float2 x = __ffma2_rn(make_float2(v[2 * k], v[2 * k + 1]), scl, off);
-          acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(ex2(x.x), ex2(x.y)));
+        for (int k = 0; k < 16; k++) {
+          const float2 y = __ffma2_rn(make_float2(x[2 * k], x[2 * k + 1]), scl, off);
+          acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(ex2(y.x), ex2(y.y)));
         }
-        const float2 t = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        s2 += t.x + t.y;
+        const float2 sum = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        s2 += sum.x + sum.y;
+      }
+      // merge the pair's (max, sum)
+      const float mo = __shfl_xor_sync(0xffffffffu, m2, C::H), so = __shfl_xor_sync(0xffffffffu, s2, C::H);
+      const float M = fmaxf(m2, mo);
+      const float S = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
+      if (scorer && role == 0 && c < nc) {
+        const int m = start ? c : cand[c];
+        unsigned long long key = 0ull;  // empty slots rank below every node
+        if (m >= 0) {
+          const int j0 = m << l;
+          const int j1 = min(min((m + 1) << l, g.nb), i);
+          const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
+          const float sc = (M + __log2f(S)) * 0.6931471805599453f + __logf(nval);
+          key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
+        }
+        keys[c] = key;
       }
     }
     tc_fence_before();
-    unsigned long long my_key = 0ull;  // empty slots rank below every node
-    if (my_m >= 0) {
-      const int j0 = my_m << l;
-      const int j1 = min(min((my_m + 1) << l, g.nb), i);
-      const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
-      const float sc = (m2 + __log2f(s2)) * 0.6931471805599453f + __logf(nval);
-      my_key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)my_m);
-    }
-    if (my_c >= 0 && my_c < nc + 1) keys[my_c] = my_key;  // slot nc: a zero pad for the paired reads
-    const int n_valid = __syncthreads_count(my_m >= 0);
+    const int nc8 = (nc + 7) & ~7;
+    if (tid >= nc && tid < nc8) keys[tid] = 0ull;  // zero pad for the 8-wide reads
+    const int n_valid = __syncthreads_count(slot_m >= 0);
     // ---- keep the best: rank = number of strictly larger keys; a kept node of rank r puts its
     // children (those that exist and start before block i; -1 otherwise) in slots 2r, 2r + 1
     const int want = l > 0 ? g.cap / 2 : g.topk;
     const int keep = min(want, n_valid);
-    if (my_m >= 0) {
+    if (slot_m >= 0) {
+      const unsigned long long my_key = keys[tid];
       int rank = 0;
       const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
-      for (int c = 0; c < (nc + 1) / 2; c++) {
-        const ulonglong2 kv = k2[c];
-        rank += (kv.x > my_key) + (kv.y > my_key);
+      for (int c = 0; c < nc8 / 2; c += 4) {
+        const ulonglong2 a0 = k2[c], a1 = k2[c + 1], a2 = k2[c + 2], a3 = k2[c + 3];
+        rank += (a0.x > my_key) + (a0.y > my_key) + (a1.x > my_key) + (a1.y > my_key) + (a2.x > my_key) +
+                (a2.y > my_key) + (a3.x > my_key) + (a3.y > my_key);
       }
       if (rank < keep) {
         if (l > 0) {
-          const int c1 = 2 * my_m + 1;
-          cand[2 * rank] = 2 * my_m;
+          const int c1 = 2 * slot_m + 1;
+          cand[2 * rank] = 2 * slot_m;
           cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
         } else {
-          kept[rank] = my_m;
+          kept[rank] = slot_m;
         }
       }
       if (rank == keep - 1) s_edge[0] = key_score(my_key);
@@ -341,17 +384,21 @@ __global__ void __launch_bounds__(kThreads, MC == 64 ? 4 : 2) select_tc_kernel(c
   }
 }
 
-template <int MC>
+template <int MC, int NT>
 cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
                       int* status, cudaStream_t st) {
-  const SelPlan L = sel_plan(g.G * g.b, MC, g.s0 + 1, 128);
-  auto kern = select_tc_kernel<MC>;
+  const SelPlan L = sel_plan(g.G * g.b, NT * SelCfg<MC, NT>::kATile, g.s0 + 1, 128);
+  auto kern = select_tc_kernel<MC, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nqb, g.B * g.Hkv);
   kern<<<grid, kThreads, L.total, st>>>(mq, pyr, idx, gap, status, g);
   return cudaGetLastError();
 }
+
+// (MC, NT) for a cap: 32 candidates per M=64 tile, 64 per M=128 tile
+inline int sel_tiles(int cap) { return cap <= 64 ? 1 : 2; }
+inline int sel_mc(int cap) { return cap <= 32 ? 64 : 128; }
 
 }  // namespace
 
@@ -362,16 +409,18 @@ bool select_tc_supported(const Geo& g) {
   if (R != 64 && R != 128 && R != 256) return false;
   if (g.q_offset % g.b != 0) return false;
   if (g.s0 >= kMaxLevels) return false;
-  const int MC = g.cap <= 64 ? 64 : 128;
-  return sel_plan(R, MC, g.s0 + 1, 128).total <= 227 * 1024;
+  const int NT = sel_tiles(g.cap), MC = sel_mc(g.cap);
+  if (NT * R > 512) return false;  // tensor-memory columns
+  return sel_plan(R, NT * MC * 256, g.s0 + 1, 128).total <= 227 * 1024;
 }
 
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
                              int* status, cudaStream_t st) {
   CUtensorMap mq;
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq)) return cudaErrorInvalidValue;
-  if (g.cap <= 64) return launch_mc<64>(g, mq, pyr, idx, gap, status, st);
-  return launch_mc<128>(g, mq, pyr, idx, gap, status, st);
+  if (g.cap <= 32) return launch_mc<64, 1>(g, mq, pyr, idx, gap, status, st);
+  if (g.cap <= 64) return launch_mc<128, 1>(g, mq, pyr, idx, gap, status, st);
+  return launch_mc<128, 2>(g, mq, pyr, idx, gap, status, st);
 }
 
 }  // namespace pyr

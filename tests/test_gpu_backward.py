@@ -112,17 +112,20 @@ def test_backward_full_32k_sampled():
     rows = np.unique(np.concatenate([rng.choice(total, 160, replace=False), [0, total - 1]]))
     _close(w, g["dQ"].reshape(-1, w.d)[rows], oracle.attend_bwd_q(w, Q, K, V, dO, g["idx"], rows), "dQ")
     nb = (w.N + w.b - 1) // w.b
-    blocks = [(0, 0), (0, nb - 1), (7, 3), (15, nb // 2)]
+    blocks = [(0, 0), (0, nb - 1), (3, 1), (7, 3), (9, 100), (12, nb - 2), (15, nb // 2), (15, 257)]
     dK, dV = oracle.attend_bwd_kv(w, Q, K, V, dO, g["idx"], blocks)
     gk = g["dK"].reshape(w.B * w.Hkv, nb, w.b, w.d)
     gv = g["dV"].reshape(w.B * w.Hkv, nb, w.b, w.d)
     _close(w, np.stack([gk[u, j] for u, j in blocks]), dK, "dK")
     _close(w, np.stack([gv[u, j] for u, j in blocks]), dV, "dV")
-    # identities on every unit: sum_k dK_k = 0 and sum_k dV_k = sum_t dO_t, up to the bf16 rounding of
-    # the outputs and of O, whose errors add like a random walk over the keys: compared with the L2
-    # norm over the keys (the random-walk scale), they stay well under 5 %
+    # identities on every unit, up to rounding that adds like a random walk over keys and rows and
+    # is compared with the L2 norm over the keys:
+    #   sum_k dV_k = sum_t dO_t (each row's probabilities sum to one): only the bf16 rounding of
+    #     P and of the outputs enters, well under 5 %;
+    #   sum_k dK_k = 0 (each row's dS sums to zero): D_t is formed from the bf16 output O, and its
+    #     error (up to |dO_t| |O_t| 2^-9) enters every row's sum, so this is only a coarse check
     sk = g["dK"].reshape(w.B * w.Hkv, w.N, w.d).astype(np.float64)
     sv = g["dV"].reshape(w.B * w.Hkv, w.N, w.d).astype(np.float64)
     do = dO.float().numpy().reshape(w.B * w.Hkv, -1, w.d).astype(np.float64)
-    assert (np.abs(sk.sum(1)) <= 0.05 * np.linalg.norm(sk, axis=1)).all()
     assert (np.abs(sv.sum(1) - do.sum(1)) <= 0.05 * np.linalg.norm(sv, axis=1)).all()
+    assert (np.abs(sk.sum(1)) <= 0.25 * np.linalg.norm(sk, axis=1)).all()
