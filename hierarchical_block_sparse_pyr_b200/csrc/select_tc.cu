@@ -43,15 +43,19 @@ constexpr int kThreads = 128;
 constexpr int kMaxCap = 128;
 constexpr int kMaxLevels = 16;  // scored levels: s0 + 1 <= 16 (nb <= 2^15 * cap)
 
-// Candidate rows of the scoring MMA. A candidate's mean is the pair (hi, lo); both rows go
-// into the same A operand, in the same quarter of the M rows (so in the same warp's TMEM
-// lanes): quarter q holds H = MC/8 candidates, their hi rows first, then their lo rows.
-// One tile of MC rows scores CPT = MC/2 candidates; NT tiles cover the cap.
-template <int MC, int NT>
+// Candidate rows of the scoring MMA. A candidate's mean is the pair (hi, lo).
+// STACK: both rows go into one A operand, in the same quarter of the M rows (so in the
+//   same warp's TMEM lanes): quarter q holds H = MC/8 candidates, their hi rows first, then
+//   their lo rows; one tile of MC rows scores CPT = MC/2 candidates, and the lane pair adds
+//   hi + lo with a shuffle. For caps that leave M rows empty otherwise (cap <= MC/2).
+// !STACK: hi rows and lo rows are two A operands with the candidate at the same row, both
+//   MMAs accumulate into one D; one tile scores CPT = MC candidates (cap = MC).
+template <int MC, int NT, bool STACK>
 struct SelCfg {
-  static constexpr int CPT = MC / 2;        // candidates per tile
-  static constexpr int H = MC / 8;          // candidates per quarter (TMEM lanes 0..H-1: hi, H..2H-1: lo)
-  static constexpr int kATile = MC * 256;   // one tile: [2 d-halves][MC rows][128 B]
+  static constexpr int CPT = STACK ? MC / 2 : MC;       // candidates per tile
+  static constexpr int H = STACK ? MC / 8 : MC / 4;     // candidates per TMEM warp quarter
+  static constexpr int kAOp = MC * 256;                 // one operand: [2 d-halves][MC rows][128 B]
+  static constexpr int kATile = STACK ? kAOp : 2 * kAOp;
   static constexpr int kMinBlocks = MC == 64 ? 5 : 2;
 };
 
@@ -82,21 +86,28 @@ __device__ __forceinline__ float key_score(unsigned long long k) {
 
 // Byte offset, inside the A tiles, of 16-byte chunk q (0..15: hi elements 8q..8q+7;
 // 16..31: the same elements of lo) of candidate slot c (128B-swizzled, K-major).
-template <int MC, int NT>
+template <int MC, int NT, bool STACK>
 __device__ __forceinline__ int a_chunk_off(int c, int q) {
-  using C = SelCfg<MC, NT>;
+  using C = SelCfg<MC, NT, STACK>;
   const int t = c / C::CPT, cc = c - t * C::CPT;
-  const int quarter = cc / C::H, w = cc - quarter * C::H;
-  const int row = quarter * (MC / 4) + (q >= 16 ? C::H : 0) + w;
+  int row, op;
+  if (STACK) {
+    const int quarter = cc / C::H, w = cc - quarter * C::H;
+    row = quarter * (MC / 4) + (q >= 16 ? C::H : 0) + w;
+    op = 0;
+  } else {
+    row = cc;
+    op = q >= 16 ? C::kAOp : 0;
+  }
   const int q16 = q & 15, h = q16 >> 3, c8 = q16 & 7;
-  return t * C::kATile + h * (MC * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((c8 ^ (row & 7)) << 4);
+  return t * C::kATile + op + h * (MC * 128) + (row >> 3) * 1024 + (row & 7) * 128 + ((c8 ^ (row & 7)) << 4);
 }
 
-template <int MC, int NT>
-__global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
+template <int MC, int NT, bool STACK>
+__global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __nv_bfloat16* __restrict__ pyr,
                      int32_t* __restrict__ idx, float* __restrict__ gap_out, int* status, Geo g) {
-  using C = SelCfg<MC, NT>;
+  using C = SelCfg<MC, NT, STACK>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -123,9 +134,10 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
   const int rb = min((i + 1) * g.b, g.q_offset + g.Nq) - p0;  // valid rows per head
   const int tcols = NT * R <= 64 ? 64 : (NT * R <= 128 ? 128 : (NT * R <= 256 ? 256 : 512));
   // scoring role of this thread: TMEM lane `lane` of warp `warp` holds, in each tile t, the hi
-  // (role 0) or lo (role 1) dot products of candidate t*CPT + warp*H + (lane % H)
-  const bool scorer = lane < 2 * C::H;
-  const int role = (lane / C::H) & 1;
+  // (role 0) or lo (role 1) dot products of candidate t*CPT + warp*H + (lane % H) (STACK), or
+  // their sum for candidate t*CPT + warp*32 + lane (!STACK, role 0)
+  const bool scorer = STACK ? lane < 2 * C::H : true;
+  const int role = STACK ? (lane / C::H) & 1 : 0;
   const int my_cq = warp * C::H + (lane % C::H);  // candidate within a tile
   const __nv_bfloat16* pu = pyr + (size_t)unit * g.P * 256;
   auto straddler = [&](int l) { return (l > 0 && (i & ((1 << l) - 1)) != 0) ? (i >> l) : -1; };
@@ -144,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
     for (int x = tid; x < nc * 32; x += kThreads) {
       const int c = x >> 5, q = x & 31;
       if (c == ms) continue;
-      cp_async16(sA + a_chunk_off<MC, NT>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+      cp_async16(sA + a_chunk_off<MC, NT, STACK>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
     }
   }
   __syncthreads();  // barrier init visible before the TMA uses it
@@ -194,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
     // the start level's straddling node (slot = its index) from its (hi, lo) row
     const int ms = straddler(g.s0);
     if (ms >= 0 && ms < nc && tid < 32)
-      *reinterpret_cast<uint4*>(sA + a_chunk_off<MC, NT>(ms, tid)) =
+      *reinterpret_cast<uint4*>(sA + a_chunk_off<MC, NT, STACK>(ms, tid)) =
           *reinterpret_cast<const uint4*>(ppair + g.s0 * 512 + tid * 16);
   }
   const uint32_t tD = *tmem_slot;
@@ -222,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
         const int c = x >> 5, q = x & 31;
         const int m = cand[c];
         if (m < 0) continue;
-        unsigned char* dst = sA + a_chunk_off<MC, NT>(c, q);
+        unsigned char* dst = sA + a_chunk_off<MC, NT, STACK>(c, q);
         if (m == ms)
           *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
         else
@@ -245,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
           const uint32_t oq = (kk >> 2) * q_half + (kk & 3) * 2;
           const uint32_t oa = (t * C::kATile + (kk >> 2) * (MC * 128)) / 16 + (kk & 3) * 2;
           umma_bf16(tD + t * R, dA0 + oa, dQ0 + oq, idesc, kk > 0);
+          if (!STACK) umma_bf16(tD + t * R, dA0 + oa + C::kAOp / 16, dQ0 + oq, idesc, 1);
         }
       }
       umma_commit(bar_mma);
@@ -266,28 +279,32 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
       if (!__any_sync(0xffffffffu, scorer && c < nc)) continue;  // warp-uniform
       float m2 = -INFINITY, s2 = 0.f;
       float v[64];
+      constexpr int NX = STACK ? 32 : 64;  // columns of a 64-column batch that this lane reduces
       for (int c0 = 0; c0 < R; c0 += 64) {
         tmem_ld32(my_lane_addr + t * R + c0, v);
         tmem_ld32(my_lane_addr + t * R + c0 + 32, v + 32);
         tmem_wait_ld();
-        float x[32];
+        if (STACK) {
 #pragma unroll
-        for (int k = 0; k < 32; k++) {
-          const float send = role ? v[k] : v[32 + k];
-          const float recv = __shfl_xor_sync(0xffffffffu, send, C::H);
-          x[k] = (role ? v[32 + k] : v[k]) + recv;
+          for (int k = 0; k < 32; k++) {
+            const float send = role ? v[k] : v[32 + k];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, C::H);
+            v[k] = (role ? v[32 + k] : v[k]) + recv;
+          }
         }
-        const int colb = c0 + role * 32;  // first column of this lane's half
+        const int colb = c0 + role * 32;  // first column of this lane's columns
         if (!full) {
 #pragma unroll
-          for (int k = 0; k < 32; k++) x[k] = ((colb + k) % g.b) < rb ? x[k] : -INFINITY;
+          for (int k = 0; k < NX; k++) v[k] = ((colb + k) % g.b) < rb ? v[k] : -INFINITY;
         }
-        float a[11];
+        float a[NX / 3 + 1];
 #pragma unroll
-        for (int k = 0; k < 10; k++) a[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
-        a[10] = fmaxf(x[30], x[31]);
-        const float bm =
-            fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmax3(a[6], a[7], fmax3(a[8], a[9], a[10]))) * sl2;
+        for (int k = 0; k < NX / 3; k++) a[k] = fmax3(v[3 * k], v[3 * k + 1], v[3 * k + 2]);
+        a[NX / 3] = NX % 3 == 2 ? fmaxf(v[NX - 2], v[NX - 1]) : v[NX - 1];
+        float bm = a[0];
+#pragma unroll
+        for (int k = 1; k < NX / 3 + 1; k++) bm = fmaxf(bm, a[k]);
+        bm *= sl2;
         const float mn = fmaxf(m2, bm);
         if (mn == -INFINITY) continue;  // nothing valid yet in this lane's columns
         s2 *= ex2(m2 - mn);             // 0 on the first valid batch (m2 = -inf)
@@ -295,17 +312,20 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
         const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
         float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-        for (int k = 0; k < 16; k++) {
-          const float2 y = __ffma2_rn(make_float2(x[2 * k], x[2 * k + 1]), scl, off);
+        for (int k = 0; k < NX / 2; k++) {
+          const float2 y = __ffma2_rn(make_float2(v[2 * k], v[2 * k + 1]), scl, off);
           acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(ex2(y.x), ex2(y.y)));
         }
         const float2 sum = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
         s2 += sum.x + sum.y;
       }
       // merge the pair's (max, sum)
-      const float mo = __shfl_xor_sync(0xffffffffu, m2, C::H), so = __shfl_xor_sync(0xffffffffu, s2, C::H);
-      const float M = fmaxf(m2, mo);
-      const float S = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
+      float M = m2, S = s2;
+      if (STACK) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m2, C::H), so = __shfl_xor_sync(0xffffffffu, s2, C::H);
+        M = fmaxf(m2, mo);
+        S = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
+      }
       if (scorer && role == 0 && c < nc) {
         const int m = start ? c : cand[c];
         unsigned long long key = 0ull;  // empty slots rank below every node
@@ -384,11 +404,11 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT>::kMinBlocks)
   }
 }
 
-template <int MC, int NT>
+template <int MC, int NT, bool STACK>
 cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
                       int* status, cudaStream_t st) {
-  const SelPlan L = sel_plan(g.G * g.b, NT * SelCfg<MC, NT>::kATile, g.s0 + 1, 128);
-  auto kern = select_tc_kernel<MC, NT>;
+  const SelPlan L = sel_plan(g.G * g.b, NT * SelCfg<MC, NT, STACK>::kATile, g.s0 + 1, 128);
+  auto kern = select_tc_kernel<MC, NT, STACK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nqb, g.B * g.Hkv);
@@ -396,9 +416,9 @@ cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const __nv_bfloat16* 
   return cudaGetLastError();
 }
 
-// (MC, NT) for a cap: 32 candidates per M=64 tile, 64 per M=128 tile
-inline int sel_tiles(int cap) { return cap <= 64 ? 1 : 2; }
-inline int sel_mc(int cap) { return cap <= 32 ? 64 : 128; }
+// the A operand bytes for a cap: stacked M=64 (cap <= 32), stacked M=128 (cap <= 64), or
+// separate hi and lo M=128 operands (cap <= 128)
+inline int sel_a_bytes(int cap) { return cap <= 32 ? 64 * 256 : (cap <= 64 ? 128 * 256 : 2 * 128 * 256); }
 
 }  // namespace
 
@@ -409,18 +429,16 @@ bool select_tc_supported(const Geo& g) {
   if (R != 64 && R != 128 && R != 256) return false;
   if (g.q_offset % g.b != 0) return false;
   if (g.s0 >= kMaxLevels) return false;
-  const int NT = sel_tiles(g.cap), MC = sel_mc(g.cap);
-  if (NT * R > 512) return false;  // tensor-memory columns
-  return sel_plan(R, NT * MC * 256, g.s0 + 1, 128).total <= 227 * 1024;
+  return sel_plan(R, sel_a_bytes(g.cap), g.s0 + 1, 128).total <= 227 * 1024;
 }
 
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
                              int* status, cudaStream_t st) {
   CUtensorMap mq;
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq)) return cudaErrorInvalidValue;
-  if (g.cap <= 32) return launch_mc<64, 1>(g, mq, pyr, idx, gap, status, st);
-  if (g.cap <= 64) return launch_mc<128, 1>(g, mq, pyr, idx, gap, status, st);
-  return launch_mc<128, 2>(g, mq, pyr, idx, gap, status, st);
+  if (g.cap <= 32) return launch_mc<64, 1, true>(g, mq, pyr, idx, gap, status, st);
+  if (g.cap <= 64) return launch_mc<128, 1, true>(g, mq, pyr, idx, gap, status, st);
+  return launch_mc<128, 1, false>(g, mq, pyr, idx, gap, status, st);
 }
 
 }  // namespace pyr

@@ -46,6 +46,12 @@ CASES = [
               dtype=BF16, seed=29, n_needle=4, needle_mode=synth.NEEDLE_DECODE),
     W0.scaled(name="cap_covers_all", B=1, Hq=2, Hkv=2, N=1024, Nq=1024, d=64, b=64, topk=4, cap=16, dtype=F32,
               seed=21),
+    # tensor-core selection layouts: candidates stacked in M=128 rows (32 < cap <= 64), and separate
+    # hi / lo operands (cap > 64)
+    W0.scaled(name="cap48_stacked_m128", B=1, Hq=2, Hkv=2, N=8192 + 30, Nq=8192 + 30, d=128, b=64, topk=20, cap=48,
+              dtype=BF16, seed=31, n_needle=6),
+    W0.scaled(name="cap100_separate", B=1, Hq=4, Hkv=2, N=16384, Nq=16384, d=128, b=64, topk=40, cap=100,
+              dtype=BF16, seed=32, n_needle=6),
 ]
 
 
