@@ -31,8 +31,8 @@ PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = ran
 PYR_F32, PYR_BF16 = 0, 1
 
 ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_update", "pyr_select",
-               "bsa_forward", "dense_forward", "bsa_route_invert", "bsa_backward", "pyr_selftest_wait",
-               "pyr_strerror")
+               "bsa_forward", "dense_forward", "bsa_route_invert", "bsa_backward", "bsa_backward_noalloc",
+               "pyr_selftest_wait", "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -76,6 +76,8 @@ def _load_lib():
     lib.bsa_route_invert.restype = ctypes.c_int
     lib.bsa_backward.argtypes = [sp] + [vp] * 15
     lib.bsa_backward.restype = ctypes.c_int
+    lib.bsa_backward_noalloc.argtypes = [sp] + [vp] * 14
+    lib.bsa_backward_noalloc.restype = ctypes.c_int
     lib.pyr_selftest_wait.argtypes = [vp, vp]
     lib.pyr_selftest_wait.restype = ctypes.c_int
     lib.pyr_strerror.argtypes = [ctypes.c_int]
@@ -180,6 +182,15 @@ def bsa_backward(s: PyrShape, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, 
                                     (offset, "offset"), (rho, "rho"), (delta, "delta"), (dQ, "dQ"), (dK, "dK"),
                                     (dV, "dV"))]
     _check(_L().bsa_backward(ctypes.byref(s), *args, _dev(status, "status", True), _stream(stream)), "bsa_backward")
+
+
+def bsa_backward_noalloc(s: PyrShape, Q, K, V, O, lse, dO, idx, offset, rho, dQ, dK, dV, status=None,
+                         stream=None):
+    """bsa_backward without the delta workspace: the library keeps it in a fixed device array."""
+    args = [_dev(t, n) for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (O, "O"), (lse, "lse"), (dO, "dO"), (idx, "idx"),
+                                    (offset, "offset"), (rho, "rho"), (dQ, "dQ"), (dK, "dK"), (dV, "dV"))]
+    _check(_L().bsa_backward_noalloc(ctypes.byref(s), *args, _dev(status, "status", True), _stream(stream)),
+           "bsa_backward_noalloc")
 
 
 def selftest_wait(status, stream=None):

@@ -1,0 +1,63 @@
+// bsa_backward_noalloc: the backward pass for callers that cannot allocate
+// device memory.
+//
+// bsa_backward needs a workspace of one fp32 per query row (D_t = dO_t . O_t),
+// which its caller allocates. Some callers cannot: code that runs while a
+// stream is being captured into a CUDA graph (cudaMalloc is not a stream
+// operation and may synchronise the device), plugins whose host framework owns
+// every byte of device memory and hands out only the tensors it knows about,
+// and serving loops that must never block on the allocator. This entry point
+// keeps that workspace in a fixed array in the library's own device memory
+// instead, so the caller passes only inputs and outputs.
+//
+// The array is a file-scope __device__ variable of kMaxRows floats (16 MiB):
+// every GPU that loads the library holds it until the process exits. Host
+// code must not pass the array's name to a kernel (on the host that name is a
+// stand-in, not a device address); its device address is looked up once per
+// device with cudaGetSymbolAddress, with that device current, on the first
+// call made on it, and cached.
+#include <mutex>
+
+#include "pyr_common.cuh"
+
+namespace pyr {
+namespace {
+
+constexpr int64_t kMaxRows = 4 * 1024 * 1024;  // B * Hq * Nq query rows
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_delta_scratch[kMaxRows];
+
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxDevices] = {};
+
+// The device address of g_delta_scratch on the current device, or nullptr.
+float* scratch_for_current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_delta_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  return g_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace pyr
+
+extern "C" int bsa_backward_noalloc(const pyr_shape* s, const void* Q, const void* K, const void* V, const void* O,
+                                    const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
+                                    const int32_t* rho, void* dQ, void* dK, void* dV, int* dev_status,
+                                    void* stream) {
+  if (!s) return PYR_EINVAL;
+  const int64_t rows = (int64_t)s->B * s->Hq * s->Nq;
+  if (rows <= 0) return PYR_EINVAL;
+  if (rows > pyr::kMaxRows) return PYR_EUNSUPPORTED;  // beyond the fixed workspace
+  float* delta = pyr::scratch_for_current_device();
+  if (!delta) return PYR_ECUDA;
+  // the workspace is written in full (one value per query row) before it is read, so it needs no
+  // clearing between calls
+  return bsa_backward(s, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV, dev_status, stream);
+}

@@ -229,6 +229,31 @@ PYR_API int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const
                          void* stream);
 
 /*
+ * bsa_backward_noalloc - bsa_backward for callers that cannot allocate device
+ * memory: code running while a stream is captured into a CUDA graph (cudaMalloc
+ * is not a stream operation and may synchronise the device), plugins whose host
+ * framework owns all device memory, serving loops that must not block on an
+ * allocator. The pages have no counterpart: this is a deployment variant of
+ * bsa_backward, not part of the method.
+ * Arguments and results are those of bsa_backward without `delta`: the
+ * per-row workspace lives in a fixed array in the library's own device memory
+ * (16 MiB per GPU that loads the library, held until the process exits), so
+ * the call allocates nothing.
+ *   Limit: B * Hq * Nq <= 4194304 query rows; larger shapes return
+ *   PYR_EUNSUPPORTED without launching anything.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current) and caches it; make that first call before any stream
+ *   capture on the device.
+ *   Every call on a device shares the one array. The workspace is written in
+ *   full before it is read, so nothing needs clearing between calls, but calls
+ *   that overlap on the GPU (on different streams, or from several threads
+ *   without ordering) race on it: order them on one stream.
+ */
+PYR_API int bsa_backward_noalloc(const pyr_shape* s, const void* Q, const void* K, const void* V, const void* O,
+                                 const float* lse, const void* dO, const int32_t* idx, const int32_t* offset,
+                                 const int32_t* rho, void* dQ, void* dK, void* dV, int* dev_status, void* stream);
+
+/*
  * pyr_selftest_wait - exercise the bounded waits the kernels rely on: one
  * kernel waits on an mbarrier that nothing arrives on and must give up after
  * its limit (about a second), store PYR_ETIMEOUT in *dev_status (device, must
