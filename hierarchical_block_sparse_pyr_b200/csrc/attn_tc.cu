@@ -325,16 +325,29 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     float s[kKeys];
     for (int t = 0; t < T; t++) {
       const int sb = t & 1;
+      int key0, mode;
+      tile_info(t, &key0, &mode);
+      const int md = row_ok ? (mode >> (2 * qsub)) & 3 : 0;
       ok = warp_wait(bar_s_full + sb, (t >> 1) & 1, abort_flag);
       if (!ok) break;
       tc_fence_after();
+      if (__all_sync(0xffffffffu, md == 0)) {
+        // no row of this warp attends the tile (with two query blocks per CTA, the tile may be
+        // routed for the other block only): P = 0, without reading S or touching the softmax state
+        uint32_t zero[32];
+#pragma unroll
+        for (int c = 0; c < 32; c++) zero[c] = 0u;
+        tmem_st32u(tS_row + sb * 64, zero);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p_full + sb);
+        continue;
+      }
       tmem_ld32(tS_row + sb * 64, s);
       tmem_ld32(tS_row + sb * 64 + 32, s + 32);
       tmem_wait_ld();
 
-      int key0, mode;
-      tile_info(t, &key0, &mode);
-      const int md = row_ok ? (mode >> (2 * qsub)) & 3 : 0;
       // valid keys: full -> every key < N; causal -> keys <= p
       const int lim = md == 0 ? 0 : (md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1));
       if (lim < kKeys) {
