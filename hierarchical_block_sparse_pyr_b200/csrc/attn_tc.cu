@@ -33,6 +33,7 @@
 
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
+#include "tile_list.cuh"
 
 namespace pyr {
 
@@ -95,7 +96,6 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   uint64_t* bar_done = bar_drain + 1;  // every MMA of the CTA finished (one phase)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
-  int* s_ntiles = reinterpret_cast<int*>(smem + PL::kMisc + 8);
   int* tiles = reinterpret_cast<int*>(smem + PL::kTiles);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,16 +105,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   const int i_first = g.i0 + qb0;
   const int nq_here = min(QB, g.nqb - qb0);  // query blocks present in this tile
 
-  // ---- setup: barriers; the routed blocks of the tile's query blocks ----
-  // The raw idx rows are staged in the K/V area, which no copy touches before
-  // the tile list is built.
-  int* s_idx = reinterpret_cast<int*>(smem + PL::kKV);  // the K ring, before any copy
-  if (!dense) {
-    for (int x = threadIdx.x; x < QB * g.topk; x += PL::kThreads) {
-      const int q = x / g.topk, k = x - q * g.topk;
-      s_idx[x] = q < nq_here ? idx[((size_t)unit * g.nqb + (qb0 + q)) * g.topk + k] : -1;
-    }
-  }
+  // ---- setup: barriers; the tile's key-block list (built in the K ring, before any copy) ----
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < NS; s++) {
@@ -133,55 +124,10 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     fence_mbar_init();
     *abort_flag = 0;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int n = 0;
-    if (!dense) {
-      // merge the ascending lists sel(i_q) + [i_q] of the tile's query blocks
-      int pos[QB], prev[QB];
-      for (int q = 0; q < QB; q++) {
-        pos[q] = 0;
-        prev[q] = -1;
-      }
-      while (n < kMaxTiles / TPB) {
-        int cand[QB];
-        int best = 0x7fffffff;
-        for (int q = 0; q < QB; q++) {
-          cand[q] = 0x7fffffff;
-          if (q >= nq_here) continue;
-          const int iq = i_first + q;
-          const int* row = s_idx + q * g.topk;
-          while (pos[q] < g.topk) {
-            const int j = row[pos[q]];
-            if (j < 0) {
-              pos[q]++;
-              continue;
-            }
-            if (j >= iq || j <= prev[q]) {
-              report(status, PYR_EBADIDX);
-              pos[q]++;
-              continue;
-            }
-            break;
-          }
-          if (pos[q] < g.topk) cand[q] = row[pos[q]];
-          else if (pos[q] == g.topk) cand[q] = iq;  // the diagonal block comes last
-          best = min(best, cand[q]);
-        }
-        if (best == 0x7fffffff) break;
-        int mode = 0;
-        for (int q = 0; q < QB; q++) {
-          if (cand[q] == best) {
-            mode |= (pos[q] == g.topk ? 2 : 1) << (2 * q);
-            prev[q] = best;
-            pos[q]++;
-          }
-        }
-        tiles[n++] = (best << 4) | mode;
-      }
-    }
-    *s_ntiles = n;
-  }
+  int n_entries = 0;
+  if (!dense)
+    n_entries = build_tile_list<QB>(idx + ((size_t)unit * g.nqb + qb0) * g.topk, g.topk, i_first, nq_here,
+                                    reinterpret_cast<int*>(smem + PL::kKV), tiles, status);
   const int softmax_warps = 4 * MT;
   if (warp == softmax_warps + 1) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
@@ -193,7 +139,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem;             // S[mt][sb] at column (mt*2 + sb)*64; P over its first 32
   const uint32_t tO = tmem + 128 * MT;  // O[mt] at column 128*MT + mt*128
-  const int nblk = dense ? (i_first + nq_here) : *s_ntiles;  // dense: blocks 0 .. last diagonal
+  const int nblk = dense ? (i_first + nq_here) : n_entries;  // dense: blocks 0 .. last diagonal
   const int T = nblk * TPB;
 
   // tile t -> (first key, modes)

@@ -38,6 +38,7 @@
 
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
+#include "tile_list.cuh"
 
 namespace pyr {
 
@@ -73,58 +74,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// The ascending union of the key blocks that query blocks i_first .. i_first+nq-1
-// attend (each one's routed blocks, then its own block), as entries
-// (block << 4) | modes with 2 bits per query block: 1 full, 2 causal, 0 skip.
-// Routes are used with the forward kernels' rule (>= 0, < i, ascending).
-template <int QB>
-__device__ int merge_tiles(const int* rows, int topk, int i_first, int nq, int max_entries, int* tiles,
-                           int* status) {
-  int pos[QB], prev[QB];
-  for (int q = 0; q < QB; q++) {
-    pos[q] = 0;
-    prev[q] = -1;
-  }
-  int n = 0;
-  while (n < max_entries) {
-    int cand[QB];
-    int best = 0x7fffffff;
-    for (int q = 0; q < QB; q++) {
-      cand[q] = 0x7fffffff;
-      if (q >= nq) continue;
-      const int iq = i_first + q;
-      const int* row = rows + q * topk;
-      while (pos[q] < topk) {
-        const int j = row[pos[q]];
-        if (j < 0) {
-          pos[q]++;
-          continue;
-        }
-        if (j >= iq || j <= prev[q]) {
-          report(status, PYR_EBADIDX);
-          pos[q]++;
-          continue;
-        }
-        break;
-      }
-      if (pos[q] < topk) cand[q] = row[pos[q]];
-      else if (pos[q] == topk) cand[q] = iq;  // the own block comes last
-      best = min(best, cand[q]);
-    }
-    if (best == 0x7fffffff) break;
-    int mode = 0;
-    for (int q = 0; q < QB; q++) {
-      if (cand[q] == best) {
-        mode |= (pos[q] == topk ? 2 : 1) << (2 * q);
-        prev[q] = best;
-        pos[q]++;
-      }
-    }
-    tiles[n++] = (best << 4) | mode;
-  }
-  return n;
-}
-
 template <int QB, int KB>
 __global__ void __launch_bounds__(DqPlan::kThreads, 1)
     bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -148,7 +97,6 @@ __global__ void __launch_bounds__(DqPlan::kThreads, 1)
   uint64_t* bar_drain = bars + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
-  int* s_ntiles = reinterpret_cast<int*>(smem + PL::kMisc + 8);
   int* tiles = reinterpret_cast<int*>(smem + PL::kTiles);
   unsigned char* sQ = smem + PL::kQ;
   unsigned char* sDO = smem + PL::kDO;
@@ -165,12 +113,6 @@ __global__ void __launch_bounds__(DqPlan::kThreads, 1)
   const int i_first = g.i0 + qb0;
   const int nq_here = min(QB, g.nqb - qb0);
 
-  // the raw idx rows, staged in the K ring before any copy lands there
-  int* s_idx = reinterpret_cast<int*>(sK);
-  for (int x = threadIdx.x; x < QB * g.topk; x += PL::kThreads) {
-    const int q = x / g.topk, k = x - q * g.topk;
-    s_idx[x] = q < nq_here ? idx[((size_t)unit * g.nqb + (qb0 + q)) * g.topk + k] : -1;
-  }
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < 3; s++) {
@@ -188,8 +130,9 @@ __global__ void __launch_bounds__(DqPlan::kThreads, 1)
     fence_mbar_init();
     *abort_flag = 0;
   }
-  __syncthreads();
-  if (threadIdx.x == 0) *s_ntiles = merge_tiles<QB>(s_idx, g.topk, i_first, nq_here, kMaxTiles / TPB, tiles, status);
+  // the tile's key-block list, built in the K ring before any copy lands there
+  const int n_entries = build_tile_list<QB>(idx + ((size_t)unit * g.nqb + qb0) * g.topk, g.topk, i_first, nq_here,
+                                            reinterpret_cast<int*>(sK), tiles, status);
   if (warp == 5) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
@@ -199,7 +142,7 @@ __global__ void __launch_bounds__(DqPlan::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tP = tmem + 128, tDQ = tmem + 256;
-  const int T = *s_ntiles * TPB;
+  const int T = n_entries * TPB;
 
   auto tile_info = [&](int t, int* key0, int* mode) {
     const int e = t / TPB, h = t - e * TPB;

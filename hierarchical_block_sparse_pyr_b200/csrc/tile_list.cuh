@@ -1,0 +1,125 @@
+// The key-block list of a query tile: the ascending union of the key blocks
+// that QB (1 or 2) consecutive query blocks attend (PHBA summary, A.1.3: one
+// loaded block serves every row of the tile that routes to it). Query block
+// i attends its routed blocks (its idx row) and its own block. Entries are
+// (block << 4) | modes, 2 bits per query block q at bit 2q: 1 routed (every
+// key), 2 own block (keys up to the row's position), 0 not attended.
+//
+// A route of row i is used only if it is >= 0, < i and greater than every
+// earlier in-range route of the row (the rule every kernel of the library
+// applies); other non-negative entries are skipped and reported as
+// PYR_EBADIDX. Built by the whole CTA in parallel: one warp per query block
+// compacts its row (a prefix-max scan reproduces the sequential rule), then
+// every element finds its place in the union by binary search, duplicates
+// (blocks routed by both query blocks) folded into one entry.
+#pragma once
+
+#include "pyr_common.cuh"
+
+namespace pyr {
+
+constexpr int kTileListPitch = 132;  // >= topk + 1 for topk <= 128, multiple of 4
+// shared-memory ints build_tile_list needs as scratch: two lists, the duplicate
+// flags and their prefix counts, two counts
+constexpr int kTileListScratch = 4 * kTileListPitch + 4;
+
+__device__ __forceinline__ int lower_bound_smem(const int* a, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < v) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Call from every thread of the CTA (it contains block-wide barriers).
+// rows: the QB idx rows in global memory (row q = query block i_first + q);
+// nq: query blocks present (1..QB). Returns the number of entries in tiles.
+template <int QB>
+__device__ int build_tile_list(const int32_t* __restrict__ rows, int topk, int i_first, int nq, int* scratch,
+                               int* tiles, int* status) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* cnt = scratch + 4 * kTileListPitch;  // [0], [1]: list lengths
+  if (warp < nq) {
+    // compact the accepted routes of row `warp`, then append its own block
+    const int iq = i_first + warp;
+    const int32_t* row = rows + (size_t)warp * topk;
+    int* L = scratch + warp * kTileListPitch;
+    int base = 0, pmax = -1;
+    for (int k0 = 0; k0 < topk; k0 += 32) {
+      const int k = k0 + lane;
+      const int j = k < topk ? row[k] : -1;
+      const bool in_range = j >= 0 && j < iq;
+      int incl = in_range ? j : -1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl = max(incl, y);
+      }
+      int before = __shfl_up_sync(0xffffffffu, incl, 1);
+      before = max(lane == 0 ? -1 : before, pmax);
+      const bool acc = in_range && j > before;
+      if (j >= 0 && !acc) report(status, PYR_EBADIDX);
+      const unsigned m = __ballot_sync(0xffffffffu, acc);
+      if (acc) L[base + __popc(m & ((1u << lane) - 1u))] = j;
+      base += __popc(m);
+      pmax = max(pmax, __shfl_sync(0xffffffffu, incl, 31));
+    }
+    if (lane == 0) {
+      L[base] = iq;
+      cnt[warp] = base + 1;
+    }
+  }
+  __syncthreads();
+  const int na = cnt[0];
+  const int* A = scratch;
+  if (QB == 1 || nq == 1) {
+    for (int k = tid; k < na; k += blockDim.x) tiles[k] = (A[k] << 4) | (k == na - 1 ? 2 : 1);
+    __syncthreads();
+    return na;
+  }
+  const int nb = cnt[1];
+  const int* B = scratch + kTileListPitch;
+  int* inA = scratch + 2 * kTileListPitch;  // [k]: B[k] is also in A
+  int* dup = scratch + 3 * kTileListPitch;  // [k]: duplicates among B[0 .. k-1]
+  if (warp == 0) {
+    int run = 0;
+    for (int k0 = 0; k0 <= nb; k0 += 32) {
+      const int k = k0 + lane;
+      int f = 0;
+      if (k < nb) {
+        const int la = lower_bound_smem(A, na, B[k]);
+        f = (la < na && A[la] == B[k]) ? 1 : 0;
+        inA[k] = f;
+      }
+      int incl = f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (k <= nb) dup[k] = run + incl - f;  // exclusive
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  __syncthreads();
+  for (int k = tid; k < na; k += blockDim.x) {
+    const int a = A[k];
+    const int lb = lower_bound_smem(B, nb, a);
+    const bool inB = lb < nb && B[lb] == a;
+    const int mode = (k == na - 1 ? 2 : 1) | (inB ? (lb == nb - 1 ? 2 : 1) << 2 : 0);
+    tiles[k + lb - dup[lb]] = (a << 4) | mode;
+  }
+  for (int k = tid; k < nb; k += blockDim.x) {
+    if (inA[k]) continue;
+    const int b = B[k];
+    const int la = lower_bound_smem(A, na, b);
+    tiles[la + k - dup[k]] = (b << 4) | ((k == nb - 1 ? 2 : 1) << 2);
+  }
+  const int n = na + nb - dup[nb];
+  __syncthreads();
+  return n;
+}
+
+}  // namespace pyr
