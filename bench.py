@@ -426,15 +426,27 @@ def run_ours(args, w, rank, world, local_rank):
         per["attention"].append(ev[2].elapsed_time(ev[3]))
     ms_max = max_over_ranks(ms_total, world, dev)
 
-    # end to end through the binding: pinned host inputs -> device -> path -> O back to pinned host
+    # end to end through the binding: pinned host inputs -> device -> path -> O back to pinned host.
+    # Prefill: a step's inputs are Q, K and V. Decode: they are the new token's q, k and v; k and v
+    # are written into the device-resident cache at the last position (the cache is state, not input).
     O_host = torch.empty(buf.O.shape, dtype=buf.O.dtype, pin_memory=True)
-    h2d = Qh.numel() * Qh.element_size() + Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
+    if w.decode:
+        Kn_h = Kh[:, :, w.N - 1].contiguous().pin_memory()
+        Vn_h = Vh[:, :, w.N - 1].contiguous().pin_memory()
+        h2d = (Qh.numel() * Qh.element_size() + Kn_h.numel() * Kn_h.element_size() +
+               Vn_h.numel() * Vn_h.element_size())
+    else:
+        h2d = Qh.numel() * Qh.element_size() + Kh.numel() * Kh.element_size() + Vh.numel() * Vh.element_size()
     d2h = O_host.numel() * O_host.element_size()
 
     def e2e_step():
         Q.copy_(Qh, non_blocking=True)
-        K.copy_(Kh, non_blocking=True)
-        V.copy_(Vh, non_blocking=True)
+        if w.decode:
+            K[:, :, w.N - 1].copy_(Kn_h, non_blocking=True)
+            V[:, :, w.N - 1].copy_(Vn_h, non_blocking=True)
+        else:
+            K.copy_(Kh, non_blocking=True)
+            V.copy_(Vh, non_blocking=True)
         step()
         O_host.copy_(buf.O, non_blocking=True)
 

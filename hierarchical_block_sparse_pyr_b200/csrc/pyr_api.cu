@@ -110,6 +110,8 @@ int pyr_select(const pyr_shape* s, const void* Q, const void* pyr_v, int32_t* id
   if (!Q || !pyr || !idx || !aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PYR_EINVAL;
   if (pyr::select_tc_supported(g))
     return launch_status(pyr::launch_select_tc(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
+  if (pyr::select_decode_supported(g))
+    return launch_status(pyr::launch_select_decode(g, Q, pyr, idx, gap, (cudaStream_t)stream));
   if (pyr::select_smem_bytes(g) > 227 * 1024) return PYR_EUNSUPPORTED;
   return launch_status(pyr::launch_select(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
 }

@@ -68,6 +68,9 @@ cudaError_t launch_attn_decode(const Geo& g, const void* Q, const void* K, const
 cudaError_t launch_select(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                           cudaStream_t st);
 bool select_tc_supported(const Geo& g);
+bool select_decode_supported(const Geo& g);
+cudaError_t launch_select_decode(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
+                                 cudaStream_t st);
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                              cudaStream_t st);
 bool attn_tc_supported(const Geo& g);
