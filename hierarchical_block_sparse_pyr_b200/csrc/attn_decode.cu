@@ -16,6 +16,7 @@
 
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
+#include "tile_list.cuh"
 
 namespace pyr {
 
@@ -94,31 +95,24 @@ __global__ void __launch_bounds__(kThreads) attn_decode_kernel(const __nv_bfloat
   const int pos = g.q_offset;  // the single query row's position
   const int i = pos / g.b;     // its (diagonal) block
 
-  // ---- block list: routed blocks (ascending, validated), then the diagonal block
+  // ---- block list: routed blocks (ascending, validated), then the diagonal block; built by the
+  // whole CTA (one warp loads and compacts the idx row)
+  __shared__ int tl_scratch[kTileListScratch];
+  __shared__ int tl_entries[kTileListPitch];
   if (tid == 0) {
-    int n = 0;
-    if (!dense) {
-      const int32_t* row = idx + (size_t)unit * g.nqb * g.topk;  // nqb == 1 in decode
-      int prev = -1;
-      for (int k = 0; k < g.topk; k++) {
-        const int j = row[k];
-        if (j < 0) continue;
-        if (j >= i || j <= prev) {
-          if (rank == 0) report(status, PYR_EBADIDX);
-          continue;
-        }
-        prev = j;
-        list[n++] = j;
-      }
-      list[n++] = i;
-    } else {
-      n = i + 1;
-    }
-    s_n = n;
     s_abort = 0;
     mbar_init(bars + 0, 1);
     mbar_init(bars + 1, 1);
     fence_mbar_init();
+  }
+  if (!dense) {
+    // nqb == 1 in decode; the cluster's other CTAs see the same routes, so only rank 0 reports
+    const int n = build_tile_list<1>(idx + (size_t)unit * g.nqb * g.topk, g.topk, i, 1, tl_scratch, tl_entries,
+                                     rank == 0 ? status : nullptr);
+    for (int e = tid; e < n; e += kThreads) list[e] = tl_entries[e] >> 4;
+    if (tid == 0) s_n = n;
+  } else if (tid == 0) {
+    s_n = i + 1;
   }
   for (int x = tid; x < G * D; x += kThreads) {
     const int gg = x / D, e = x - gg * D;
