@@ -101,11 +101,15 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
       const int e0 = my_h * DPT;
       if (m == ms) {
         const float* pr = part + l * D + e0;
-        for (int e = 0; e < DPT; e++) {
-          const float kv = pr[e];
+        for (int e = 0; e < DPT; e += 4) {
+          const float4 kv = *reinterpret_cast<const float4*>(pr + e);
 #pragma unroll
-          for (int gg = 0; gg < kMaxG; gg++)
-            if (gg < G) acc[gg] = fmaf(q_s[gg * D + e0 + e], kv, acc[gg]);
+          for (int gg = 0; gg < kMaxG; gg++) {
+            if (gg < G) {
+              const float4 qa = *reinterpret_cast<const float4*>(q_s + gg * D + e0 + e);
+              acc[gg] = fmaf(qa.x, kv.x, fmaf(qa.y, kv.y, fmaf(qa.z, kv.z, fmaf(qa.w, kv.w, acc[gg]))));
+            }
+          }
         }
       } else {
         const __nv_bfloat16* row = pu + (size_t)(g.lvl_off[l] + m) * 2 * D;
@@ -113,16 +117,29 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
         const uint4* lo4 = reinterpret_cast<const uint4*>(row + D + e0);
 #pragma unroll 2
         for (int v = 0; v < DPT / 8; v++) {
-          float hf[8], lf[8];
+          float hf[8], lf[8], kv[8];
           bf16x8_to_f32(hi4[v], hf);
           bf16x8_to_f32(lo4[v], lf);
 #pragma unroll
-          for (int k = 0; k < 8; k++) {
-            const float kv = hf[k] + lf[k];
-            const int e = e0 + v * 8 + k;
+          for (int k = 0; k < 8; k++) kv[k] = hf[k] + lf[k];
+          const int e = e0 + v * 8;
 #pragma unroll
-            for (int gg = 0; gg < kMaxG; gg++)
-              if (gg < G) acc[gg] = fmaf(q_s[gg * D + e], kv, acc[gg]);
+          for (int gg = 0; gg < kMaxG; gg++) {
+            if (gg < G) {
+              // the 8 query elements of row gg as two 16-byte loads (the same for every candidate: broadcast)
+              const float4 qa = *reinterpret_cast<const float4*>(q_s + gg * D + e);
+              const float4 qb = *reinterpret_cast<const float4*>(q_s + gg * D + e + 4);
+              float a = acc[gg];
+              a = fmaf(qa.x, kv[0], a);
+              a = fmaf(qa.y, kv[1], a);
+              a = fmaf(qa.z, kv[2], a);
+              a = fmaf(qa.w, kv[3], a);
+              a = fmaf(qb.x, kv[4], a);
+              a = fmaf(qb.y, kv[5], a);
+              a = fmaf(qb.z, kv[6], a);
+              a = fmaf(qb.w, kv[7], a);
+              acc[gg] = a;
+            }
           }
         }
       }
