@@ -12,7 +12,10 @@
 //                     the warp splits rows), reduces with shuffles, and the
 //                     CTA then pools the chunk's subtree in shared memory.
 //   pyr_top_kernel    the levels above the chunk level, one CTA per
-//                     (unit, 16-element slice of d), entirely in shared memory.
+//                     (unit, 16-element slice of d), entirely in shared memory;
+//                     launched as a programmatic dependent of the chunk kernel,
+//                     so its CTAs are resident before the chunk kernel ends and
+//                     wait (griddepcontrol.wait) for the chunk kernel's writes.
 #include "pyr_common.cuh"
 
 namespace pyr {
@@ -159,6 +162,8 @@ __global__ void __launch_bounds__(kChunkThreads) pyr_chunk_kernel(const T* __res
     cur = nxt;
     nxt = t;
   }
+  // this CTA's nodes are written: the top-level kernel may start launching
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Levels t+1 .. L from level t, for one unit and a 16-wide slice of d.
@@ -170,6 +175,8 @@ __global__ void __launch_bounds__(kTopThreads) pyr_top_kernel(__nv_bfloat16* __r
   const int nt = g.lvl_n[t];
   float* cur = sm;
   float* nxt = sm + (size_t)nt * kTopSlice;
+  // the chunk kernel's level-t nodes are complete and visible past this point
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // load level t as sums
   for (int x = threadIdx.x; x < nt * kTopSlice; x += kTopThreads) {
     const int m = x / kTopSlice, e = x - m * kTopSlice;
@@ -294,9 +301,17 @@ cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int*
     e = cudaFuncSetAttribute(pyr_top_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(g.d / kTopSlice, g.B * g.Hkv);
-  pyr_top_kernel<<<grid, kTopThreads, smem, st>>>(pyr, g, t);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(g.d / kTopSlice, g.B * g.Hkv, 1);
+  cfg.blockDim = dim3(kTopThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, pyr_top_kernel, pyr, g, t);
 }
 
 }  // namespace pyr
