@@ -129,3 +129,44 @@ def test_backward_full_32k_sampled():
     do = dO.float().numpy().reshape(w.B * w.Hkv, -1, w.d).astype(np.float64)
     assert (np.abs(sv.sum(1) - do.sum(1)) <= 0.05 * np.linalg.norm(sv, axis=1)).all()
     assert (np.abs(sk.sum(1)) <= 0.25 * np.linalg.norm(sk, axis=1)).all()
+
+
+
+@pytest.mark.parametrize("name", ["gqa_bf16_64k", "mha_bf16_1m"])
+def test_backward_full_size_sampled(name):
+    """The larger workloads at full size: route inversion bit-exact, sampled dQ rows, and dK/dV of
+    sampled key blocks (chosen among blocks routed by at most 12 query blocks, so that the oracle,
+    which recomputes every attending row in double, finishes in seconds). Only the sampled pieces
+    are copied back to the host."""
+    w = [x for x in synth.WORKLOADS if x.name == name][0]
+    s = P.shape_of(w)
+    Q, K, V, _ = synth.generate(w)
+    dO = synth.grad_output(w)
+    Qd, Kd, Vd, dOd = (t.cuda() for t in (Q, K, V, dO))
+    fwd = P.Buffers(s)
+    bwd = P.BackwardBuffers(s)
+    P.run(s, Qd, Kd, Vd, fwd)
+    P.run_backward(s, Qd, Kd, Vd, dOd, fwd, bwd)
+    torch.cuda.synchronize()
+    assert int(fwd.status.item()) == 0
+    idx = fwd.idx.cpu().numpy()
+    off_g, rho_g = bwd.offset.cpu().numpy(), bwd.rho.cpu().numpy()
+    off, rho = oracle.route_invert(w, idx)
+    assert (off_g == off).all() and (rho_g == rho).all()
+    rng = np.random.default_rng(11)
+    total = w.B * w.Hq * w.Nq
+    rows = np.unique(np.concatenate([rng.choice(total, 48, replace=False), [0, total - 1]]))
+    dQ_g = bwd.dQ.reshape(-1, w.d)[torch.as_tensor(rows).cuda()].float().cpu().numpy()
+    _close(w, dQ_g, oracle.attend_bwd_q(w, Q, K, V, dO, idx, rows), "dQ")
+    nb = (w.N + w.b - 1) // w.b
+    counts = np.diff(off, axis=1)  # query blocks routing to each key block
+    U = w.B * w.Hkv
+    pool = [(u, j) for u in (0, U // 2, U - 1) for j in range(nb) if counts[u, j] <= 12]
+    pick = [pool[k] for k in rng.choice(len(pool), size=min(4, len(pool)), replace=False)] + [(U - 1, nb - 1)]
+    dK, dV = oracle.attend_bwd_kv(w, Q, K, V, dO, idx, pick)
+    gk = bwd.dK.reshape(U, nb, w.b, w.d)
+    gv = bwd.dV.reshape(U, nb, w.b, w.d)
+    _close(w, np.stack([gk[u, j].float().cpu().numpy() for u, j in pick]), dK, "dK")
+    _close(w, np.stack([gv[u, j].float().cpu().numpy() for u, j in pick]), dV, "dV")
+    del fwd, bwd, Qd, Kd, Vd, dOd
+    torch.cuda.empty_cache()
