@@ -262,8 +262,11 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
       }
       umma_commit(bar_mma);
     }
-    // this thread's slot (rank phase: slot = tid) and its node, read before any slot is rewritten
+    // this thread's slot (rank phase: slot = tid) and its node, read before any slot is rewritten;
+    // with at most 32 slots (M = 64, stacked rows) four threads share slot tid / 4 in the rank count
+    constexpr bool kSplit = (MC == 64 && STACK);
     const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
+    const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
     ok = mbar_wait(bar_mma, nphase & 1, abort_flag);
     ok = __syncthreads_and(ok);  // block-uniform: the loop below has block-wide barriers
     nphase++;
@@ -341,13 +344,37 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     }
     tc_fence_before();
     const int nc8 = (nc + 7) & ~7;
-    if (tid >= nc && tid < nc8) keys[tid] = 0ull;  // zero pad for the 8-wide reads
+    if (tid >= nc && tid < (kSplit ? 32 : nc8)) keys[tid] = 0ull;  // zero pad for the 8-wide reads
     const int n_valid = __syncthreads_count(slot_m >= 0);
     // ---- keep the best: rank = number of strictly larger keys; a kept node of rank r puts its
     // children (those that exist and start before block i; -1 otherwise) in slots 2r, 2r + 1
     const int want = l > 0 ? g.cap / 2 : g.topk;
     const int keep = min(want, n_valid);
-    if (slot_m >= 0) {
+    if (kSplit) {
+      // slot tid / 4: each of its four threads counts the larger keys among 8 of the 32
+      const int sl = tid >> 2, part = tid & 3;
+      const unsigned long long my_key = keys[sl];
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys) + part * 4;
+      const ulonglong2 a0 = k2[0], a1 = k2[1], a2 = k2[2], a3 = k2[3];
+      int rank = split_m >= 0 ? (a0.x > my_key) + (a0.y > my_key) + (a1.x > my_key) + (a1.y > my_key) +
+                                    (a2.x > my_key) + (a2.y > my_key) + (a3.x > my_key) + (a3.y > my_key)
+                              : 0;
+      rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+      rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+      if (split_m >= 0 && part == 0) {
+        if (rank < keep) {
+          if (l > 0) {
+            const int c1 = 2 * split_m + 1;
+            cand[2 * rank] = 2 * split_m;
+            cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+          } else {
+            kept[rank] = split_m;
+          }
+        }
+        if (rank == keep - 1) s_edge[0] = key_score(my_key);
+        if (rank == keep) s_edge[1] = key_score(my_key);
+      }
+    } else if (slot_m >= 0) {
       const unsigned long long my_key = keys[tid];
       int rank = 0;
       const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
