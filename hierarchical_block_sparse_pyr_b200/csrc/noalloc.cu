@@ -2,11 +2,10 @@
 // device memory.
 //
 // bsa_backward needs a workspace of one fp32 per query row (D_t = dO_t . O_t),
-// which its caller allocates. Some callers cannot: code that runs while a
-// stream is being captured into a CUDA graph (cudaMalloc is not a stream
-// operation and may synchronise the device), plugins whose host framework owns
-// every byte of device memory and hands out only the tensors it knows about,
-// and serving loops that must never block on the allocator. This entry point
+// which its caller allocates. Some callers cannot: plugins whose host framework
+// owns every byte of device memory and hands out only the tensors it knows
+// about, and serving or real-time loops that must never call cudaMalloc (it can
+// synchronise the device and block on the allocator). This entry point
 // keeps that workspace in a fixed array in the library's own device memory
 // instead, so the caller passes only inputs and outputs.
 //

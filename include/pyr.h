@@ -230,11 +230,11 @@ PYR_API int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const
 
 /*
  * bsa_backward_noalloc - bsa_backward for callers that cannot allocate device
- * memory: code running while a stream is captured into a CUDA graph (cudaMalloc
- * is not a stream operation and may synchronise the device), plugins whose host
- * framework owns all device memory, serving loops that must not block on an
- * allocator. The pages have no counterpart: this is a deployment variant of
- * bsa_backward, not part of the method.
+ * memory: plugins whose host framework owns all device memory and hands out
+ * only the tensors it knows about, and serving or real-time loops that must not
+ * call cudaMalloc (it can synchronise the device and block on the allocator).
+ * The paper has no counterpart: this is a deployment variant of bsa_backward,
+ * not part of the method.
  * Arguments and results are those of bsa_backward without `delta`: the
  * per-row workspace lives in a fixed array in the library's own device memory
  * (16 MiB per GPU that loads the library, held until the process exits), so

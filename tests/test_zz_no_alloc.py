@@ -1,7 +1,7 @@
 """bsa_backward_noalloc: the backward pass for callers that cannot allocate device memory.
 
-Callers that capture streams into CUDA graphs, plugins whose host owns all device
-memory, and serving loops that must not block on an allocator cannot hand
+Plugins whose host framework owns all device memory, and serving or real-time
+loops that must not call cudaMalloc (it can synchronise the device), cannot hand
 bsa_backward its per-row workspace. The no-allocation entry point keeps that
 workspace in a fixed array inside the library. Here it is called through the C
 ABI, twice in a row, and each result is compared with bsa_backward's on the same
