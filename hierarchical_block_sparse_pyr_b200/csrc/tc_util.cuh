@@ -180,23 +180,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 64: Cody-Waite reduction x = j + f with j the
-// nearest integer (the 1.5 * 2^23 rounding trick) and f in [-0.5, 0.5], then a
-// degree-4 polynomial fitted here to minimise the relative error of 2^f on
-// that interval (max 2.7e-6 in fp32 Horner form); 2^j enters through the
-// exponent bits. Inputs below -126 (and -inf) give a value below 2^-126.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.5f);
-  const float r = x + 12582912.0f;  // 1.5 * 2^23: r's low mantissa bits hold round(x)
-  const float f = x - (r - 12582912.0f);
-  float p = fmaf(0.009570610709488392f, f, 0.055917903780937195f);
-  p = fmaf(p, f, 0.24024732410907745f);
-  p = fmaf(p, f, 0.6931217908859253f);
-  p = fmaf(p, f, 0.9999992847442627f);
-  // round(x) << 23 == bits(r) << 23 (mod 2^32): the offset bits of 1.5 * 2^23 shift out
-  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
