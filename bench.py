@@ -63,7 +63,12 @@ def level_sizes(w):
 
 
 def work_counts(w):
-    """Algorithmic bytes / FLOPs of one step (exact counts from the method's definition)."""
+    """Algorithmic bytes / FLOPs of one step from the method's definition.
+
+    Attention pairs are exact; selection counts every node that can be a candidate
+    at each level, an upper bound on the nodes the walk actually scores (a few
+    percent above it: a kept node whose second child starts at or after the
+    query block contributes one child, not two)."""
     elt = 4 if w.dtype == synth.F32 else 2
     lv = level_sizes(w)
     P = sum(lv)

@@ -97,3 +97,35 @@ def test_python_binding_refuses_cpu_tensors():
     K = torch.zeros((1, 2, 256, 64))
     with pytest.raises(TypeError):
         P.pyr_build(s, K, torch.zeros((1, 2, P.num_nodes(s), 64)))
+
+
+def test_backward_entry_points_validate_on_the_host():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    lib = P._L()
+    s = P.shape_of(synth.WORKLOADS[0].scaled(N=1024, Nq=1024))
+    ok = [16] * 13
+    # route inversion: idx must be 16-byte aligned, offset and rho 4-byte aligned, none null
+    assert lib.bsa_route_invert(ctypes.byref(s), None, 16, 16, None, None) == P.PYR_EINVAL
+    assert lib.bsa_route_invert(ctypes.byref(s), 24, 16, 16, None, None) == P.PYR_EINVAL
+    assert lib.bsa_route_invert(ctypes.byref(s), 16, 18, 16, None, None) == P.PYR_EINVAL
+    assert lib.bsa_route_invert(ctypes.byref(s), 16, 16, None, None, None) == P.PYR_EINVAL
+    assert lib.bsa_route_invert(None, 16, 16, 16, None, None) == P.PYR_EINVAL
+    # backward: every operand present; tensors 16-byte aligned, lse/delta/offset/rho 4-byte aligned
+    for k in range(13):
+        args = list(ok)
+        args[k] = None
+        assert lib.bsa_backward(ctypes.byref(s), *args, None, None) == P.PYR_EINVAL, k
+    for k in range(13):
+        args = list(ok)
+        args[k] = 16 + 2  # misaligned for every operand
+        assert lib.bsa_backward(ctypes.byref(s), *args, None, None) == P.PYR_EINVAL, k
+    # shape errors come first, as in the forward entry points
+    bad = P.shape_of(synth.WORKLOADS[0].scaled(N=1024, Nq=1024))
+    bad.cap = 7
+    assert lib.bsa_backward(ctypes.byref(bad), *ok, None, None) == P.PYR_EINVAL
+    # the backward pass covers whole sequences only: a chunk or a decode step is refused
+    chunk = P.shape_of(synth.WORKLOADS[0].scaled(N=1024, Nq=512, q_offset=512))
+    assert lib.bsa_backward(ctypes.byref(chunk), *ok, None, None) == P.PYR_EUNSUPPORTED
+    dec = P.shape_of(synth.WORKLOADS[1].scaled(N=100, Nq=1, q_offset=99))
+    assert lib.bsa_backward(ctypes.byref(dec), *ok, None, None) == P.PYR_EUNSUPPORTED
