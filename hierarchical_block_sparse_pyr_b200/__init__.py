@@ -31,8 +31,8 @@ PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = ran
 PYR_F32, PYR_BF16 = 0, 1
 
 ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_update", "pyr_select",
-               "bsa_forward", "dense_forward", "bsa_route_invert", "bsa_backward", "bsa_backward_noalloc",
-               "pyr_selftest_wait", "pyr_strerror")
+               "bsa_forward", "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes", "bsa_route_invert",
+               "bsa_backward", "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -72,6 +72,10 @@ def _load_lib():
     lib.bsa_forward.restype = ctypes.c_int
     lib.dense_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
     lib.dense_forward.restype = ctypes.c_int
+    lib.bsa_forward_host.argtypes = [sp, vp, vp, vp, vp, vp, ctypes.c_int, vp, ctypes.c_size_t, vp, vp]
+    lib.bsa_forward_host.restype = ctypes.c_int
+    lib.pyr_host_workspace_bytes.argtypes = [sp, ctypes.c_int, ctypes.c_int]
+    lib.pyr_host_workspace_bytes.restype = ctypes.c_size_t
     lib.bsa_route_invert.argtypes = [sp, vp, vp, vp, vp, vp]
     lib.bsa_route_invert.restype = ctypes.c_int
     lib.bsa_backward.argtypes = [sp] + [vp] * 15
@@ -170,6 +174,34 @@ def dense_forward(s: PyrShape, Q, K, V, O, lse=None, status=None, stream=None):
     _check(_L().dense_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(O, "O"),
                               _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)),
            "dense_forward")
+
+
+def _host(t, name, nullable=False):
+    if t is None:
+        if nullable:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise TypeError(f"{name} must be a CPU tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def host_workspace_bytes(s: PyrShape, units_per_chunk: int = 0, with_lse: bool = False) -> int:
+    return _L().pyr_host_workspace_bytes(ctypes.byref(s), int(units_per_chunk), int(bool(with_lse)))
+
+
+def bsa_forward_host(s: PyrShape, Q, K, V, O, lse=None, units_per_chunk: int = 0, workspace=None, status=None,
+                     stream=None):
+    """The whole forward path for host (CPU, ideally pinned) Q, K, V; writes host O and lse.
+
+    workspace: a CUDA uint8 tensor of at least host_workspace_bytes(s, units_per_chunk, lse is not None)
+    bytes. The results are ready once `stream` (default: the current stream) has been synchronised."""
+    _check(_L().bsa_forward_host(ctypes.byref(s), _host(Q, "Q"), _host(K, "K"), _host(V, "V"), _host(O, "O"),
+                                 _host(lse, "lse", True), int(units_per_chunk), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _dev(status, "status", True),
+                                 _stream(stream)), "bsa_forward_host")
 
 
 def bsa_route_invert(s: PyrShape, idx, offset, rho, status=None, stream=None):

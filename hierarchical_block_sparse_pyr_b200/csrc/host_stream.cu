@@ -1,0 +1,192 @@
+// bsa_forward_host: the forward path for inputs and outputs in host memory.
+//
+// The (batch, kv head) units are independent through all three steps (pyramid,
+// selection, attention), so they stream through the device in chunks of
+// consecutive units: while chunk c is computed on the caller's stream, chunk
+// c + 1 is copied in on one copy stream and chunk c - 1's output is copied out
+// on another. PCIe moves data in both directions at once, so a step costs
+// about the host-to-device copy of Q, K and V plus the compute and copy-out
+// of the last chunk, instead of the sum of all three.
+//
+// A chunk of n consecutive units is itself a valid shape: B = n, Hq = G,
+// Hkv = 1. Unit u = bi * Hkv + hk owns query heads hk G .. hk G + G - 1 of
+// batch bi, which lie next to each other in [B][Hq][Nq][d], so unit u's query
+// rows start at u G Nq d and its keys at u N d. Every kernel computes a unit
+// the same way whatever the other units of its launch are, so the result is
+// bit-identical to pyr_build + pyr_select + bsa_forward over the whole batch.
+//
+// Device workspace (caller-owned): two slots of {Q, K, V, O, lse} for one
+// chunk each, and one pyramid and one idx array for a chunk (the compute
+// stream is in order, so those are reused chunk after chunk). Each part
+// starts on a 256-byte boundary relative to the workspace base.
+#include <mutex>
+
+#include "pyr_common.cuh"
+
+namespace {
+
+constexpr int kSlots = 2;
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct ChunkLayout {
+  size_t q, kv, o, lse, pyr, idx;  // bytes of each part for one chunk, rounded up
+  size_t slot;                     // q + 2 kv + o + lse
+  size_t total;                    // kSlots * slot + pyr + idx
+};
+
+ChunkLayout layout_for(const pyr_shape* s, int64_t P, int64_t nqb, int upc, bool with_lse) {
+  const size_t elt = s->dtype == PYR_F32 ? 4 : 2;
+  const size_t G = (size_t)(s->Hq / s->Hkv);
+  ChunkLayout c;
+  c.q = round_up((size_t)upc * G * s->Nq * s->d * elt);
+  c.kv = round_up((size_t)upc * s->N * s->d * elt);
+  c.o = c.q;
+  c.lse = with_lse ? round_up((size_t)upc * G * s->Nq * sizeof(float)) : 0;
+  c.pyr = round_up((size_t)upc * P * 2 * s->d * 2);
+  c.idx = round_up((size_t)upc * nqb * s->topk * sizeof(int32_t));
+  c.slot = c.q + 2 * c.kv + c.o + c.lse;
+  c.total = kSlots * c.slot + c.pyr + c.idx;
+  return c;
+}
+
+// Chunk size when the caller passes 0: about 16 chunks per call, so that the
+// last chunk (whose compute and copy-out are not hidden) is small.
+int auto_units(const pyr_shape* s) {
+  const int U = s->B * s->Hkv;
+  return U <= 16 ? 1 : (U + 15) / 16;
+}
+
+// Two copy streams and the events that order the slots, made once per device
+// and kept until the process exits. The mutex serialises the enqueueing of
+// calls on one device, so that an event is re-recorded only after every wait
+// on its previous record has been enqueued.
+struct DeviceStreams {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry, in_done[kSlots], compute_done[kSlots], out_done[kSlots], h2d_exit, d2h_exit;
+};
+
+DeviceStreams g_dev[kMaxDevices];
+
+cudaError_t init_streams(DeviceStreams& ds) {
+  if (ds.ready) return cudaSuccess;
+  cudaError_t e = cudaStreamCreateWithFlags(&ds.h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ds.d2h, cudaStreamNonBlocking);
+  cudaEvent_t* evs[] = {&ds.entry, &ds.h2d_exit, &ds.d2h_exit};
+  for (cudaEvent_t* ev : evs)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  for (int k = 0; k < kSlots && e == cudaSuccess; k++) {
+    e = cudaEventCreateWithFlags(&ds.in_done[k], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ds.compute_done[k], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ds.out_done[k], cudaEventDisableTiming);
+  }
+  // on failure the streams and events made so far are kept and the next call
+  // makes the rest again; a failure here means the device is unusable anyway
+  if (e == cudaSuccess) ds.ready = true;
+  return e;
+}
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? PYR_OK : PYR_ECUDA; }
+
+}  // namespace
+
+extern "C" size_t pyr_host_workspace_bytes(const pyr_shape* s, int units_per_chunk, int with_lse) {
+  if (units_per_chunk < 0 || pyr::validate_shape(s) != PYR_OK) return 0;
+  const int64_t P = pyr_num_nodes(s), nqb = pyr_num_qblocks(s);
+  const int U = s->B * s->Hkv;
+  int upc = units_per_chunk ? units_per_chunk : auto_units(s);
+  if (upc > U) upc = U;
+  return layout_for(s, P, nqb, upc, with_lse != 0).total;
+}
+
+extern "C" int bsa_forward_host(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                                int units_per_chunk, void* workspace, size_t workspace_bytes, int* dev_status,
+                                void* stream) {
+  const int rc0 = pyr::validate_shape(s);
+  if (rc0 != PYR_OK) return rc0;
+  const int64_t P = pyr_num_nodes(s), nqb = pyr_num_qblocks(s);
+  if (!Q || !K || !V || !O || !workspace || ((uintptr_t)workspace & 15u) || units_per_chunk < 0) return PYR_EINVAL;
+  const int U = s->B * s->Hkv;
+  int upc = units_per_chunk ? units_per_chunk : auto_units(s);
+  if (upc > U) upc = U;
+  const ChunkLayout c = layout_for(s, P, nqb, upc, lse != nullptr);
+  if (workspace_bytes < c.total) return PYR_EINVAL;
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PYR_ECUDA;
+  DeviceStreams& ds = g_dev[dev];
+  std::lock_guard<std::mutex> lock(ds.mu);
+  if (init_streams(ds) != cudaSuccess) return PYR_ECUDA;
+
+  const cudaStream_t st = (cudaStream_t)stream;
+  const size_t elt = s->dtype == PYR_F32 ? 4 : 2;
+  const int G = s->Hq / s->Hkv;
+  const size_t q_unit = (size_t)G * s->Nq * s->d * elt, kv_unit = (size_t)s->N * s->d * elt;
+  const size_t lse_unit = (size_t)G * s->Nq * sizeof(float);
+  char* base = static_cast<char*>(workspace);
+  char* pyr = base + kSlots * c.slot;
+  int32_t* idx = reinterpret_cast<int32_t*>(pyr + c.pyr);
+
+  // nothing on the copy streams may start before the caller's earlier work on
+  // its stream (which may still be using the workspace)
+  cudaError_t e = cudaEventRecord(ds.entry, st);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ds.h2d, ds.entry, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(ds.d2h, ds.entry, 0);
+  int rc = status_of(e);
+
+  const int nchunks = (U + upc - 1) / upc;
+  for (int ch = 0; ch < nchunks && rc == PYR_OK; ch++) {
+    const int u0 = ch * upc, n = U - u0 < upc ? U - u0 : upc;
+    const int k = ch % kSlots;
+    char* slot = base + k * c.slot;
+    char *dq = slot, *dk = slot + c.q, *dv = dk + c.kv, *dout = dv + c.kv;
+    float* dlse = lse ? reinterpret_cast<float*>(dout + c.o) : nullptr;
+    pyr_shape cs = *s;
+    cs.B = n;
+    cs.Hq = G;
+    cs.Hkv = 1;
+
+    // in: the slot's inputs are free once the chunk that used it two chunks ago has been computed
+    if (ch >= kSlots) e = cudaStreamWaitEvent(ds.h2d, ds.compute_done[k], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dq, static_cast<const char*>(Q) + u0 * q_unit, n * q_unit, cudaMemcpyHostToDevice, ds.h2d);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dk, static_cast<const char*>(K) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
+                          ds.h2d);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(dv, static_cast<const char*>(V) + u0 * kv_unit, n * kv_unit, cudaMemcpyHostToDevice,
+                          ds.h2d);
+    if (e == cudaSuccess) e = cudaEventRecord(ds.in_done[k], ds.h2d);
+    // compute: after the inputs arrived and the slot's previous output left
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ds.in_done[k], 0);
+    if (e == cudaSuccess && ch >= kSlots) e = cudaStreamWaitEvent(st, ds.out_done[k], 0);
+    rc = status_of(e);
+    if (rc == PYR_OK) rc = pyr_build(&cs, dk, pyr, dev_status, st);
+    if (rc == PYR_OK) rc = pyr_select(&cs, dq, pyr, idx, nullptr, dev_status, st);
+    if (rc == PYR_OK) rc = bsa_forward(&cs, dq, dk, dv, idx, dout, dlse, dev_status, st);
+    if (rc != PYR_OK) break;
+    e = cudaEventRecord(ds.compute_done[k], st);
+    // out
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds.d2h, ds.compute_done[k], 0);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(O) + u0 * q_unit, dout, n * q_unit, cudaMemcpyDeviceToHost, ds.d2h);
+    if (e == cudaSuccess && lse)
+      e = cudaMemcpyAsync(lse + (size_t)u0 * (lse_unit / sizeof(float)), dlse, n * lse_unit, cudaMemcpyDeviceToHost,
+                          ds.d2h);
+    if (e == cudaSuccess) e = cudaEventRecord(ds.out_done[k], ds.d2h);
+    rc = status_of(e);
+  }
+
+  // the caller's stream ends after everything enqueued above, on error too:
+  // its later work may free or reuse the workspace and the host buffers
+  cudaError_t e2 = cudaEventRecord(ds.h2d_exit, ds.h2d);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, ds.h2d_exit, 0);
+  if (e2 == cudaSuccess) e2 = cudaEventRecord(ds.d2h_exit, ds.d2h);
+  if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, ds.d2h_exit, 0);
+  if (rc == PYR_OK) rc = status_of(e2);
+  return rc;
+}

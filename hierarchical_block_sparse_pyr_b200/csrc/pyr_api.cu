@@ -66,6 +66,11 @@ int launch_status(cudaError_t e) { return e == cudaSuccess ? PYR_OK : PYR_ECUDA;
 
 }  // namespace
 
+int pyr::validate_shape(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g);
+}
+
 extern "C" {
 
 int pyr_num_levels(const pyr_shape* s) {

@@ -58,6 +58,10 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Host-side shape check of every entry point: PYR_OK or the error code the
+// entry points return for this shape.
+int validate_shape(const pyr_shape* s);
+
 // Launchers (one per kernel family). Each returns cudaSuccess or the launch error.
 cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int* status, cudaStream_t st);
 cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,

@@ -40,7 +40,8 @@
  *   non-zero (a ragged last block).
  *   Ownership: the caller allocates and owns every buffer; the library
  *   allocates nothing, keeps no state between calls beyond cached kernel
- *   attributes, and never frees caller memory.
+ *   attributes (and the copy streams of bsa_forward_host and the workspace
+ *   array of bsa_backward_noalloc), and never frees caller memory.
  *   Streams: `stream` is a cudaStream_t passed as void* (NULL = the legacy
  *   default stream). Calls only enqueue work and return; results are ready
  *   once the stream has been synchronised.
@@ -181,6 +182,48 @@ PYR_API int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const 
  */
 PYR_API int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
                   int* dev_status, void* stream);
+
+/*
+ * bsa_forward_host - the whole forward path (pyr_build, pyr_select and
+ * bsa_forward) for inputs and outputs in host memory. The pages state the
+ * problem with Q, K and V as inputs and O and the log-sum-exp as outputs
+ * (PHBA summary, 3.1 and A.1.3); this entry point takes them where a caller
+ * without device copies of them holds them.
+ * The (batch, kv head) units are independent through all three steps, so
+ * they stream through the device in chunks of `units_per_chunk` consecutive
+ * units (0: about 16 chunks per call): chunk c is computed on `stream` while
+ * chunk c + 1 is copied in and chunk c - 1's output copied out on two copy
+ * streams the library keeps per device (made on the first call on a device,
+ * held until the process exits). O and lse are bit-identical to the three
+ * device calls over the whole batch.
+ *   Q, K, V   host, layouts as above (read).
+ *   O         host, [B][Hq][Nq][d] in s->dtype (written).
+ *   lse       host, [B][Hq][Nq] fp32, or NULL (written).
+ *   workspace device, 16-byte aligned, at least
+ *             pyr_host_workspace_bytes(s, units_per_chunk, lse != NULL)
+ *             bytes, caller-owned; its contents on return are unspecified.
+ *   dev_status device word, or NULL, as for the other entry points.
+ * Host buffers should be page-locked (cudaHostAlloc, cudaHostRegister) for
+ * the copies to overlap the compute; pageable memory gives the same result
+ * with the copies serialised by the CUDA runtime.
+ * The call enqueues and returns: everything it enqueues, on any stream, ends
+ * before work the caller enqueues on `stream` afterwards, so O and lse are
+ * ready, and the workspace and the host buffers are free, once `stream` has
+ * been synchronised; the host inputs must stay unchanged until then. Work on
+ * `stream` before the call is ordered before it. Calls on one device are
+ * enqueued one at a time (a lock); calls that share a workspace must be
+ * ordered on one stream.
+ * Returns the host-side status; PYR_EINVAL also for a workspace that is too
+ * small or misaligned. After an error part of the output may be written.
+ */
+PYR_API int bsa_forward_host(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,
+                             int units_per_chunk, void* workspace, size_t workspace_bytes, int* dev_status,
+                             void* stream);
+
+/* Device workspace bytes that bsa_forward_host needs for this shape, chunk
+ * size (0 = automatic) and lse output (with_lse != 0); 0 on a bad shape or a
+ * negative chunk size. */
+PYR_API size_t pyr_host_workspace_bytes(const pyr_shape* s, int units_per_chunk, int with_lse);
 
 /*
  * bsa_route_invert - the routes in block-major form, for the backward pass

@@ -129,3 +129,56 @@ def test_backward_entry_points_validate_on_the_host():
     assert lib.bsa_backward(ctypes.byref(chunk), *ok, None, None) == P.PYR_EUNSUPPORTED
     dec = P.shape_of(synth.WORKLOADS[1].scaled(N=100, Nq=1, q_offset=99))
     assert lib.bsa_backward(ctypes.byref(dec), *ok, None, None) == P.PYR_EUNSUPPORTED
+
+
+def _ws_expected(w, upc, with_lse):
+    """Workspace of bsa_forward_host: two slots of one chunk's Q, K, V, O (and lse), one pyramid, one idx."""
+    r = lambda x: -(-x // 256) * 256  # noqa: E731
+    elt = 4 if w.dtype == synth.F32 else 2
+    q = r(upc * w.G * w.Nq * w.d * elt)
+    kv = r(upc * w.N * w.d * elt)
+    lse = r(upc * w.G * w.Nq * 4) if with_lse else 0
+    pyr = r(upc * oracle.num_nodes(w) * 2 * w.d * 2)
+    idx = r(upc * oracle.num_qblocks(w) * w.topk * 4)
+    return 2 * (2 * q + 2 * kv + lse) + pyr + idx
+
+
+def test_host_entry_point_workspace_size():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    w = synth.WORKLOADS[1]
+    s = P.shape_of(w)
+    U = w.B * w.Hkv
+    for upc, with_lse in ((1, False), (1, True), (3, True), (U, False)):
+        assert P.host_workspace_bytes(s, upc, with_lse) == _ws_expected(w, upc, with_lse), (upc, with_lse)
+    # 0 picks about 16 chunks; more units per chunk than there are units means one chunk
+    assert P.host_workspace_bytes(s, 0) == _ws_expected(w, max(1, -(-U // 16)), False)
+    assert P.host_workspace_bytes(s, 10 * U) == _ws_expected(w, U, False)
+    assert P.host_workspace_bytes(s, -1) == 0
+    bad = P.shape_of(w)
+    bad.cap = 7
+    assert P.host_workspace_bytes(bad, 1) == 0
+
+
+def test_host_entry_point_validates_on_the_host():
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    lib = P._L()
+    w = synth.WORKLOADS[1]
+    s = P.shape_of(w)
+    need = P.host_workspace_bytes(s, 1, False)
+    call = lambda sh, q=16, k=16, v=16, o=16, upc=1, ws=256, nbytes=need: lib.bsa_forward_host(  # noqa: E731
+        ctypes.byref(sh) if sh is not None else None, q, k, v, o, None, upc, ws, nbytes, None, None)
+    assert call(None) == P.PYR_EINVAL
+    for kw in ({"q": None}, {"k": None}, {"v": None}, {"o": None}, {"ws": None}, {"ws": 264}, {"upc": -1},
+               {"nbytes": need - 1}):
+        assert call(s, **kw) == P.PYR_EINVAL, kw
+    # shape errors are those of the device entry points
+    for field, value in (("cap", 7), ("d", 96), ("q_offset", 10)):
+        bad = P.shape_of(w)
+        setattr(bad, field, value)
+        assert call(bad) == lib.pyr_build(ctypes.byref(bad), 16, 16, None, None), field
+    with pytest.raises(TypeError):
+        import torch
+        P.bsa_forward_host(s, torch.zeros(4), torch.zeros(4), torch.zeros(4), torch.zeros(4),
+                           workspace=torch.zeros(16, dtype=torch.uint8))
