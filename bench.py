@@ -548,52 +548,73 @@ def run_ours(args, w, rank, world, local_rank):
 
 # -------------------------------------------------------- oracle baseline --
 
-def oracle_sample(w, n_qb, seed=0, Q=None, K=None, V=None):
-    """Time the oracle on one (batch, kv head) unit: its pyramid, n_qb evenly spaced query blocks
-    (selection + attention of all their rows). Returns (seconds, est. seconds for the whole job, desc)."""
+def oracle_sample(w, n_qb, seed=0, Q=None, K=None, V=None, n_units=1):
+    """Time the oracle on n_units consecutive (batch, kv head) units starting at unit `seed`: their
+    pyramids and n_qb evenly spaced query blocks of each (selection + attention of all their rows).
+    Returns (seconds, est. seconds for the whole job, desc); with every unit and every query block in
+    the sample the estimate is the measured time itself."""
     import oracle
 
     if Q is None:
         Q, K, V, _ = synth.generate(w)
     nqb = oracle.num_qblocks(w)
     U = w.B * w.Hkv
-    unit = seed % U
-    bi, hk = divmod(unit, w.Hkv)
+    units = [(seed + k) % U for k in range(min(max(1, n_units), U))]
     qbs = np.unique(np.linspace(0, nqb - 1, num=min(n_qb, nqb)).round().astype(int))
     t0 = time.perf_counter()
-    pyr = oracle.pyramid(w, K, [unit])
+    pyr = oracle.pyramid(w, K, units)
     t1 = time.perf_counter()
-    idx_u, _, _ = oracle.select(w, Q, pyr, [unit], [(0, int(q)) for q in qbs])
+    idx_u, _, _ = oracle.select(w, Q, pyr, units, [(k, int(q)) for k in range(len(units)) for q in qbs])
     t2 = time.perf_counter()
     full_idx = -np.ones((w.B, w.Hkv, nqb, w.topk), dtype=np.int32)
-    full_idx[bi, hk, qbs] = idx_u
     rows = []
     first = w.q_offset // w.b
-    for q in qbs:
-        i = first + int(q)
-        p0, p1 = max(i * w.b, w.q_offset), min((i + 1) * w.b, w.q_offset + w.Nq)
-        for g in range(w.G):
-            hq = hk * w.G + g
-            rows += [((bi * w.Hq + hq) * w.Nq + (p - w.q_offset)) for p in range(p0, p1)]
+    for k, unit in enumerate(units):
+        bi, hk = divmod(unit, w.Hkv)
+        full_idx[bi, hk, qbs] = idx_u[k * len(qbs):(k + 1) * len(qbs)]
+        for q in qbs:
+            i = first + int(q)
+            p0, p1 = max(i * w.b, w.q_offset), min((i + 1) * w.b, w.q_offset + w.Nq)
+            for g in range(w.G):
+                hq = hk * w.G + g
+                rows += [((bi * w.Hq + hq) * w.Nq + (p - w.q_offset)) for p in range(p0, p1)]
     oracle.attend(w, Q, K, V, full_idx, np.array(rows, dtype=np.int64))
     t3 = time.perf_counter()
-    per_qb = ((t2 - t1) + (t3 - t2)) / len(qbs)
-    est = U * ((t1 - t0) + per_qb * nqb)
-    desc = (f"unit {unit} of {U}: pyramid + {len(qbs)} of {nqb} query blocks (evenly spaced; selection + "
-            f"attention of all their rows); whole-job time extrapolated x{U} units")
+    nu = len(units)
+    per_qb = ((t2 - t1) + (t3 - t2)) / (len(qbs) * nu)
+    est = U * ((t1 - t0) / nu + per_qb * nqb)
+    if nu == U and len(qbs) == nqb:
+        desc = f"the whole job: all {U} units, pyramid + selection + attention of all {nqb} query blocks each"
+    else:
+        desc = (f"units {units[0]}..{units[-1]} of {U}: pyramid + {len(qbs)} of {nqb} query blocks each (evenly "
+                f"spaced; selection + attention of all their rows); whole-job time extrapolated")
     return t3 - t0, est, desc
 
 
 def cpu_baseline(w, budget_s=15.0):
+    """The oracle on a sample of about budget_s * 0.4 .. budget_s seconds: more query blocks of one unit
+    first, then more units, up to the whole job."""
     Q, K, V, _ = synth.generate(w)
-    n = 4
+    nqb = oracle_nqb(w)
+    U = w.B * w.Hkv
+    n, nu = 4, 1
     took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V)
-    while took < budget_s * 0.4 and n < 4096:
-        n = min(4096, int(n * max(2.0, budget_s / max(took, 1e-3) * 0.5)))
-        took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V)
+    while took < budget_s * 0.4 and (n < min(nqb, 4096) or nu < U):
+        grow = max(2.0, budget_s / max(took, 1e-3) * 0.9)
+        if n < min(nqb, 4096):
+            n = min(nqb, 4096, int(n * grow))
+        else:
+            nu = min(U, int(nu * grow))
+        took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V, n_units=nu)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": round(w.B * w.Nq / est, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": desc, "sample_seconds": round(took, 2)}
+
+
+def oracle_nqb(w):
+    import oracle
+
+    return oracle.num_qblocks(w)
 
 
 def run_reference(args, w):
