@@ -224,6 +224,23 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
 
   for (int l = g.s0; l >= 0 && ok; l--) {
     const bool start = (l == g.s0);
+    // this thread's slot (rank phase: slot = tid) and its node; with at most 32 slots (M = 64,
+    // stacked rows) four threads share slot tid / 4 in the rank count
+    constexpr bool kSplit = (MC == 64 && STACK);
+    const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
+    const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
+    const int n_valid = __syncthreads_count(slot_m >= 0);
+    const int want = l > 0 ? g.cap / 2 : g.topk;
+    const int keep = min(want, n_valid);
+    if (keep == n_valid) {
+      // every valid candidate survives this level whatever its score: no scoring. Keys that
+      // rank the candidates by node index (a fixed score, index tie-break) hand the same set on
+      for (int c = tid; c < nc; c += kThreads) {
+        const int m = start ? c : cand[c];
+        keys[c] = m >= 0 ? (0x80000000ull << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m) : 0ull;
+      }
+      cp_async_wait_all();  // the start level's gather, if this is the start level
+    } else {
     // ---- gather (levels below the start): every thread copies 16-byte chunks of the
     // candidates' (hi, lo) rows with cp.async straight to their swizzled places in the A
     // operand; the straddling node's row comes from shared memory instead; empty slots (-1)
@@ -262,11 +279,6 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
       }
       umma_commit(bar_mma);
     }
-    // this thread's slot (rank phase: slot = tid) and its node, read before any slot is rewritten;
-    // with at most 32 slots (M = 64, stacked rows) four threads share slot tid / 4 in the rank count
-    constexpr bool kSplit = (MC == 64 && STACK);
-    const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
-    const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
     ok = mbar_wait(bar_mma, nphase & 1, abort_flag);
     ok = __syncthreads_and(ok);  // block-uniform: the loop below has block-wide barriers
     nphase++;
@@ -342,14 +354,13 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
         keys[c] = key;
       }
     }
+    }  // scored level
     tc_fence_before();
     const int nc8 = (nc + 7) & ~7;
     if (tid >= nc && tid < (kSplit ? 32 : nc8)) keys[tid] = 0ull;  // zero pad for the 8-wide reads
-    const int n_valid = __syncthreads_count(slot_m >= 0);
+    __syncthreads();
     // ---- keep the best: rank = number of strictly larger keys; a kept node of rank r puts its
     // children (those that exist and start before block i; -1 otherwise) in slots 2r, 2r + 1
-    const int want = l > 0 ? g.cap / 2 : g.topk;
-    const int keep = min(want, n_valid);
     if (kSplit) {
       // slot tid / 4: each of its four threads counts the larger keys among 8 of the 32
       const int sl = tid >> 2, part = tid & 3;
