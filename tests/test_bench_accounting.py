@@ -9,7 +9,6 @@ it is checked against the oracle's own routes and walk on small workloads:
     be fewer (a straddling node's second child, or the end of a level), so the
     closed form is an upper bound within a few percent.
 """
-import numpy as np
 import pytest
 
 import bench

@@ -3,7 +3,6 @@ import numpy as np
 import torch
 
 import synth
-from synth import BF16, F32
 
 
 def test_draws_are_deterministic_and_seed_dependent():
