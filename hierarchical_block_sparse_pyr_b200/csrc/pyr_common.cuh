@@ -29,8 +29,6 @@ __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
-
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
 template <>
