@@ -30,9 +30,9 @@ LIB_PATH = os.path.join(_PKG, "lib", "libpyr.so")
 PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = range(6)
 PYR_F32, PYR_BF16 = 0, 1
 
-ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_build", "pyr_update", "pyr_select",
-               "bsa_forward", "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes", "bsa_route_invert",
-               "bsa_backward", "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
+ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_pyramid_elems", "pyr_build", "pyr_update",
+               "pyr_select", "bsa_forward", "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes",
+               "bsa_route_invert", "bsa_backward", "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -62,6 +62,8 @@ def _load_lib():
     lib.pyr_num_nodes.restype = ctypes.c_int64
     lib.pyr_num_qblocks.argtypes = [sp]
     lib.pyr_num_qblocks.restype = ctypes.c_int64
+    lib.pyr_pyramid_elems.argtypes = [sp]
+    lib.pyr_pyramid_elems.restype = ctypes.c_size_t
     lib.pyr_build.argtypes = [sp, vp, vp, vp, vp]
     lib.pyr_build.restype = ctypes.c_int
     lib.pyr_update.argtypes = [sp, vp, vp, ctypes.c_int, vp, vp]
@@ -125,6 +127,11 @@ def num_nodes(s: PyrShape) -> int:
 
 def num_qblocks(s: PyrShape) -> int:
     return _L().pyr_num_qblocks(ctypes.byref(s))
+
+
+def pyramid_elems(s: PyrShape) -> int:
+    """bf16 values of the pyr buffer: B * Hkv * P * 2 * d."""
+    return _L().pyr_pyramid_elems(ctypes.byref(s))
 
 
 def _dev(t, name, nullable=False):

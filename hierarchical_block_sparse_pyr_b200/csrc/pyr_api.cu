@@ -88,6 +88,11 @@ int64_t pyr_num_qblocks(const pyr_shape* s) {
   return make_geo(s, &g) == PYR_OK ? g.nqb : 0;
 }
 
+size_t pyr_pyramid_elems(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? (size_t)s->B * s->Hkv * (size_t)g.P * 2 * s->d : 0;
+}
+
 int pyr_build(const pyr_shape* s, const void* K, void* pyr, int* dev_status, void* stream) {
   Geo g;
   int rc = make_geo(s, &g);

@@ -105,6 +105,11 @@ PYR_API int64_t pyr_num_nodes(const pyr_shape* s);
 /* Query blocks per (batch, kv head), nqb; 0 on a bad shape. */
 PYR_API int64_t pyr_num_qblocks(const pyr_shape* s);
 
+/* Elements of the pyr buffer: B * Hkv * P * 2 * d bf16 values (the (hi, lo)
+ * pair of every node mean), which is as many bytes as B * Hkv * P * d fp32
+ * means; 0 on a bad shape. */
+PYR_API size_t pyr_pyramid_elems(const pyr_shape* s);
+
 /*
  * pyr_build - the key pyramid (PISA abstract: pooling builds O(log N) levels;
  * PHBA A.1.2: a centroid is the fp32 average of the block's key rows).

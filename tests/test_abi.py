@@ -44,6 +44,10 @@ def test_geometry_matches_the_oracle():
         assert P.num_levels(s) == oracle.num_levels(w)
         assert P.num_nodes(s) == oracle.num_nodes(w)
         assert P.num_qblocks(s) == oracle.num_qblocks(w)
+        assert P.pyramid_elems(s) == w.B * w.Hkv * oracle.num_nodes(w) * 2 * w.d
+    bad = P.shape_of(synth.WORKLOADS[0])
+    bad.cap = 7
+    assert P.pyramid_elems(bad) == 0
 
 
 @pytest.mark.parametrize("field,value,code", [
