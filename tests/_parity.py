@@ -2,13 +2,16 @@
 
 Acceptance (per the selection/attention contract):
   idx   bit-exact for every (batch, kv head, query block) whose oracle gap is
-        >= GAP_EXEMPT; rows under it may differ and are counted;
+        >= GAP_EXEMPT; a row under it may differ, but then the walk must be able
+        to end in the GPU's result when every comparison of two oracle scores
+        within TIE_EPS of each other may go either way (`walk_reaches`);
   O     bf16: max-abs <= 2e-2 and relative L2 <= 1e-2; fp32: max-abs <= 1e-4;
   lse   bf16: max-abs <= 2e-3; fp32: max-abs <= 1e-4;
   pyr   fp32 accumulation against the double oracle: max-abs <= 2e-5 * (1 + |x|).
 """
 from __future__ import annotations
 
+import itertools
 import math
 
 import numpy as np
@@ -19,6 +22,9 @@ import oracle
 import synth
 
 GAP_EXEMPT = 1e-4
+# comparisons the walk may take either way when a GPU row differs inside the exemption: twice the
+# exemption, i.e. per-score differences up to GAP_EXEMPT between the GPU's fp32 scores and the oracle's
+TIE_EPS = 2 * GAP_EXEMPT
 TOL = {synth.F32: dict(o_abs=1e-4, o_rel=1e-4, lse=1e-4), synth.BF16: dict(o_abs=2e-2, o_rel=1e-2, lse=2e-3)}
 
 
@@ -122,3 +128,134 @@ def fmt(w):
 
 def sqrt_d(w):
     return math.sqrt(w.d)
+
+
+# ---- tie-tolerant walk: which results can the coarse-to-fine walk reach when near-ties go either way --
+
+def walk_reaches(w, Q, pyr_unit: np.ndarray, unit: int, qb: int, target, eps: float, max_states: int = 20000):
+    """Can the walk of (unit, query block qb) end in `target` (one idx row) if each comparison between
+    two oracle node scores that differ by at most `eps` may be decided either way?
+
+    The walk (PISA abstract: coarse-to-fine, a bounded candidate set per level) starts at the finest
+    level s0 with at most `cap` nodes, with every node that begins before query block i; a level
+    above 0 keeps min(cap/2, #candidates) nodes and hands on their children that exist and begin
+    before i; level 0 keeps min(topk, #candidates). A kept set S of candidates C is reachable when
+    min score over S >= max score over C minus S, minus eps. With eps = 0 and no exact ties only the
+    oracle's own result is reachable; when every level's margin exceeds eps it is still the only one.
+    Scores are the oracle's (`oracle.node_score`). Returns True, False, or None when the search
+    visited more than max_states (level, candidate set) states.
+    """
+    first = w.q_offset // w.b
+    i = first + qb
+    lv = [n for _, n in oracle.level_offsets(w)]
+    s0 = 0
+    while lv[s0] > w.cap:
+        s0 += 1
+    T = sorted(int(x) for x in np.asarray(target).reshape(-1) if x >= 0)
+    if len(set(T)) != len(T):
+        return False
+    cache = {}
+
+    def score(l, m):
+        if (l, m) not in cache:
+            cache[(l, m)] = oracle.node_score(w, Q, pyr_unit, unit, qb, l, m)[0]
+        return cache[(l, m)]
+
+    def reachable_sets(cands, sc, keep, required):
+        """Every kept set of size `keep` that holds `required` and meets the eps rule."""
+        if keep == 0:
+            return [frozenset()] if not required else []
+        out = []
+        seen = set()
+        for z in cands:  # z: the lowest-scoring member of the kept set
+            t = sc[z]
+            must = {x for x in cands if sc[x] > t + eps} | set(required) | {z}
+            if any(sc[x] < t for x in must) or len(must) > keep:
+                continue
+            opt = sorted((x for x in cands if x not in must and t <= sc[x] <= t + eps), key=lambda x: (-sc[x], x))
+            need = keep - len(must)
+            if need > len(opt):
+                continue
+            if math.comb(len(opt), need) > 2000:
+                return None
+            for extra in itertools.combinations(opt, need):
+                S = frozenset(must | set(extra))
+                if S in seen:
+                    continue
+                seen.add(S)
+                rest = [sc[x] for x in cands if x not in S]
+                if not rest or min(sc[x] for x in S) >= max(rest) - eps:
+                    out.append(S)
+        # the oracle's own choice (best scores, lower index on ties) first
+        out.sort(key=lambda S: sorted((-sc[x], x) for x in S))
+        return out
+
+    states = [0]
+    visited = {}
+
+    def dfs(l, cands):
+        key = (l, frozenset(cands))
+        if key in visited:
+            return visited[key]
+        states[0] += 1
+        if states[0] > max_states:
+            raise _SearchBound
+        sc = {m: score(l, m) for m in cands}
+        want = w.cap // 2 if l > 0 else w.topk
+        keep = min(want, len(cands))
+        required = sorted({t >> l for t in T})
+        if any(r not in sc for r in required):
+            visited[key] = False
+            return False
+        if l == 0:
+            if len(T) != keep:
+                res = False
+            else:
+                rest = [sc[x] for x in cands if x not in set(T)]
+                res = not rest or min(sc[x] for x in T) >= max(rest) - eps
+            visited[key] = res
+            return res
+        sets = reachable_sets(cands, sc, keep, required)
+        if sets is None:
+            raise _SearchBound
+        res = False
+        for S in sets:
+            nxt = sorted(ch for m in S for ch in (2 * m, 2 * m + 1) if ch < lv[l - 1] and (ch << (l - 1)) < i)
+            if dfs(l - 1, nxt):
+                res = True
+                break
+        visited[key] = res
+        return res
+
+    start = [m for m in range(lv[s0]) if (m << s0) < i]
+    try:
+        return dfs(s0, start)
+    except _SearchBound:
+        return None
+
+
+class _SearchBound(Exception):
+    pass
+
+
+def check_exempt_rows(w, Q, pyr_units: np.ndarray, units, items, idx_gpu: np.ndarray, idx_ora: np.ndarray,
+                      gap_ora: np.ndarray, eps: float = TIE_EPS):
+    """Every row inside the gap exemption whose GPU idx differs from the oracle's must be reachable by
+    the tie-tolerant walk. items[k] = (slot, qb): slot indexes units and pyr_units ([len(units), P, d]).
+    Returns (differing, reached, undecided); undecided rows (search bound) are reported, not failed."""
+    idx_gpu = idx_gpu.reshape(len(items), -1)
+    idx_ora = idx_ora.reshape(len(items), -1)
+    gap_ora = gap_ora.reshape(-1)
+    differing = reached = undecided = 0
+    for k, (slot, qb) in enumerate(items):
+        if gap_ora[k] >= GAP_EXEMPT or (idx_gpu[k] == idx_ora[k]).all():
+            continue
+        differing += 1
+        r = walk_reaches(w, Q, pyr_units[slot], units[slot], qb, idx_gpu[k], eps)
+        if r is None:
+            undecided += 1
+            continue
+        assert r, (f"unit {units[slot]} query block {qb}: GPU idx {idx_gpu[k]} is not reachable by the walk with "
+                   f"near-ties within {eps} (oracle {idx_ora[k]}, gap {gap_ora[k]:.2e})")
+        reached += 1
+    return differing, reached, undecided

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from _parity import (check_out, check_pyramid, check_select, check_valid_idx, fmt, run_gpu)
+from _parity import (check_exempt_rows, check_out, check_pyramid, check_select, check_valid_idx, fmt, run_gpu)
 from synth import BF16, F32
 
 pytestmark = pytest.mark.gpu
@@ -80,12 +80,15 @@ def test_parity_small(w):
     idx_o, gap_o, _ = oracle.select_all(w, Q, K)
     idx_g = g["idx"].numpy().reshape(idx_o.shape)
     checked, exempt, exempt_diff = check_select(idx_g, idx_o, gap_o)
+    items = [(u, q) for u in units for q in range(idx_o.shape[1])]
+    _, reached, undecided = check_exempt_rows(w, Q, pyr_o, units, items, idx_g, idx_o, gap_o)
     check_valid_idx(w, g["idx"].numpy())
     gap_g = g["gap"].double().numpy().reshape(gap_o.shape)
     fin = np.isfinite(gap_o)
     assert (np.isfinite(gap_g) == fin).all()
     np.testing.assert_allclose(gap_g[fin], gap_o[fin], atol=1e-3, rtol=1e-3)
-    print(f"\n{fmt(w)} select: {checked} rows bit-exact, {exempt} exempt ({exempt_diff} differ)")
+    print(f"\n{fmt(w)} select: {checked} rows bit-exact, {exempt} exempt ({exempt_diff} differ: {reached} reachable "
+          f"with near-ties either way, {undecided} undecided)")
 
     rows = _rows_all(w) if w.B * w.Hq * w.Nq <= 16384 else _rows_sample(w)
     # attention given the oracle's idx

@@ -13,8 +13,8 @@ import torch
 
 import oracle
 import synth
-from _parity import (check_out, check_pyramid, check_select, check_valid_idx, fmt, rows_of_qblock, run_gpu,
-                     sample_items)
+from _parity import (check_exempt_rows, check_out, check_pyramid, check_select, check_valid_idx, fmt,
+                     rows_of_qblock, run_gpu, sample_items)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +37,7 @@ def test_workload_full_size(w):
     idx_o, gap_o, _ = oracle.select(w, Q, pyr_o, units, items)
     idx_g = np.stack([idx_all.reshape(w.B * w.Hkv, -1, w.topk)[units[s], q] for s, q in items])
     checked, exempt, exempt_diff = check_select(idx_g, idx_o, gap_o)
+    _, reached, undecided = check_exempt_rows(w, Q, pyr_o, units, items, idx_g, idx_o, gap_o)
 
     # attention for sampled rows, given the oracle's idx: patch those rows into a copy of the GPU idx
     idx_patch = idx_all.copy().reshape(w.B * w.Hkv, -1, w.topk)
@@ -69,7 +70,8 @@ def test_workload_full_size(w):
             if 0 <= i - first < sel.shape[1]:
                 tot += 1
                 hit += int(j in sel[u, i - first])
-    print(f"\n{fmt(w)}: select {checked} rows bit-exact, {exempt} exempt ({exempt_diff} differ); "
+    print(f"\n{fmt(w)}: select {checked} rows bit-exact, {exempt} exempt ({exempt_diff} differ, {reached} reachable "
+          f"with near-ties either way, {undecided} undecided); "
           f"attention on {len(rows)} rows max-abs {e:.2e} rel-L2 {r:.2e}; needle recall {hit}/{tot}")
     del g, g2
     torch.cuda.empty_cache()
