@@ -441,3 +441,25 @@ def test_attend_rejects_non_causal_or_repeated_blocks():
     idx[0, 0, 2] = [1, 1]
     with pytest.raises(ValueError):
         oracle.attend(w, Q, K, V, idx, np.array([70]))
+
+
+def _recall(w):
+    Q, K, V, owner = synth.generate(w)
+    idx, _, _ = oracle.select_all(w, Q, K)
+    own = owner.numpy().reshape(w.B * w.Hkv, -1)
+    first = w.q_offset // w.b
+    hit = tot = 0
+    for u in range(own.shape[0]):
+        for j in np.nonzero(own[u] >= 0)[0]:
+            i = own[u, j]
+            if 0 <= i - first < idx.shape[1]:
+                tot += 1
+                hit += int(j in idx[u, i - first])
+    return hit, tot
+
+
+@pytest.mark.parametrize("name,expect", [("mha_bf16_32k", (6411, 6588)), ("gqa_bf16_64k", (9036, 14591))])
+def test_needle_recall_is_frozen_at_full_size(name, expect):
+    """Regression pins: the oracle's needle recall on the full workloads, as measured on this generator
+    (a property of the method and the data, not a target)."""
+    assert _recall(synth.BY_NAME[name]) == expect
