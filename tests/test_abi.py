@@ -186,3 +186,22 @@ def test_host_entry_point_validates_on_the_host():
         import torch
         P.bsa_forward_host(s, torch.zeros(4), torch.zeros(4), torch.zeros(4), torch.zeros(4),
                            workspace=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_device_memory_grows_linearly_with_the_context():
+    """The score matrix is never formed (PISA abstract): every buffer the path needs, and the host-buffer
+    workspace, grow in proportion to N, never with N^2."""
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    base = synth.WORKLOADS[1]
+    sizes = []
+    for N in (32768, 65536, 131072, 262144, 1 << 20):
+        w = base.scaled(N=N, Nq=N)
+        s = P.shape_of(w)
+        nqb = P.num_qblocks(s)
+        tensors = 4 * w.B * w.Hq * N * w.d * 2                    # Q, K, V, O (bf16, MHA)
+        routes = w.B * w.Hkv * nqb * (w.topk + 1) * 4 + w.B * w.Hq * N * 4  # idx, gap, lse
+        total = tensors + routes + P.pyramid_elems(s) * 2
+        sizes.append((N, total, P.host_workspace_bytes(s, 0, True)))
+    for (n0, t0, h0), (n1, t1, h1) in zip(sizes, sizes[1:]):
+        assert t1 / t0 <= 1.01 * n1 / n0 and h1 / h0 <= 1.01 * n1 / n0, (n0, n1)
