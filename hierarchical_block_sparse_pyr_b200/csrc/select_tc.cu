@@ -6,7 +6,10 @@
 //
 // One CTA (4 warps) per (batch, kv head, query block i). The walk is a chain
 // of dependent levels, so the kernel is built for latency: per level it takes
-// four block-wide barriers and one batch of MMAs.
+// five block-wide barriers and one batch of MMAs. A level that has no more
+// valid candidates than it keeps (cap/2, or topk at level 0) passes all of
+// them on whatever their scores, so it skips gather, score and LogSumExp and
+// ranks the candidates by node index (three barriers).
 //   prologue the G*b query rows are staged once by TMA (the N operand); the
 //            start level's candidates are requested at once; the nodes that
 //            straddle block i (one per level) get the exact means of their
