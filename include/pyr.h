@@ -72,7 +72,7 @@ extern "C" {
 
 #define PYR_OK 0
 #define PYR_EINVAL 1       /* a NULL or misaligned pointer, or an inconsistent shape */
-#define PYR_EUNSUPPORTED 2 /* a shape or dtype this build has no kernel for */
+#define PYR_EUNSUPPORTED 2 /* a shape or dtype the library has no kernel for */
 #define PYR_ECUDA 3        /* the CUDA runtime refused a launch */
 #define PYR_ETIMEOUT 4     /* device: a bounded wait ran out (kernel returned early) */
 #define PYR_EBADIDX 5      /* device: idx held a block that is not strictly before its query block */

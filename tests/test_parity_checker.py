@@ -10,7 +10,7 @@ on the CPU, against the oracle itself:
   - a pyramid perturbed by noise well under eps/2 per score makes the oracle pick
     other rows, and every one of them is reachable (the call the GPU tests make);
   - a perturbation ten times larger yields rows that are not (the check is not vacuous);
-  - an exhausted search reports None instead of a verdict.
+  - an exhausted search reports None instead of an answer.
 """
 import numpy as np
 import pytest
@@ -91,8 +91,8 @@ def test_rows_from_much_larger_score_errors_are_not_all_reachable(w32):
     moved = pyr + rng.normal(0.0, 1e-3, pyr.shape)
     idx2, _, _ = oracle.select(w, Q, moved, units, items)
     rows = np.nonzero(~(idx2 == idx).all(axis=1))[0][:300]
-    verdicts = [walk_reaches(w, Q, pyr[items[k][0]], items[k][0], items[k][1], idx2[k], TIE_EPS) for k in rows]
-    assert verdicts.count(False) >= 20 and verdicts.count(None) == 0
+    answers = [walk_reaches(w, Q, pyr[items[k][0]], items[k][0], items[k][1], idx2[k], TIE_EPS) for k in rows]
+    assert answers.count(False) >= 20 and answers.count(None) == 0
 
 
 def test_search_bound_reports_undecided(w32):
