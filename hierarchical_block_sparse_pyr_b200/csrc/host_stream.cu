@@ -19,6 +19,8 @@
 // chunk each, and one pyramid and one idx array for a chunk (the compute
 // stream is in order, so those are reused chunk after chunk). Each part
 // starts on a 256-byte boundary relative to the workspace base.
+#include <map>
+#include <memory>
 #include <mutex>
 
 #include "pyr_common.cuh"
@@ -26,7 +28,6 @@
 namespace {
 
 constexpr int kSlots = 2;
-constexpr int kMaxDevices = 64;
 constexpr size_t kAlign = 256;
 
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -59,9 +60,12 @@ int auto_units(const pyr_shape* s) {
   return U <= 16 ? 1 : (U + 15) / 16;
 }
 
-// Two copy streams and the events that order the slots, made once per device
+// Two copy streams and the events that order the slots, made once per CUDA
+// context (streams and events belong to the context they were made in, so the
+// primary context of a device, a context the caller made current with the
+// driver API and a context made after a cudaDeviceReset each get their own)
 // and kept until the process exits. The mutex serialises the enqueueing of
-// calls on one device, so that an event is re-recorded only after every wait
+// calls in one context, so that an event is re-recorded only after every wait
 // on its previous record has been enqueued.
 struct DeviceStreams {
   std::mutex mu;
@@ -70,7 +74,17 @@ struct DeviceStreams {
   cudaEvent_t entry, in_done[kSlots], compute_done[kSlots], out_done[kSlots], h2d_exit, d2h_exit;
 };
 
-DeviceStreams g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+std::map<unsigned long long, std::unique_ptr<DeviceStreams>> g_dev;  // context id -> its streams
+
+DeviceStreams* streams_for_current_context() {
+  unsigned long long ctx = 0;
+  if (!pyr::current_context_id(&ctx)) return nullptr;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  std::unique_ptr<DeviceStreams>& ds = g_dev[ctx];
+  if (!ds) ds.reset(new DeviceStreams);
+  return ds.get();
+}
 
 cudaError_t init_streams(DeviceStreams& ds) {
   if (ds.ready) return cudaSuccess;
@@ -116,9 +130,9 @@ extern "C" int bsa_forward_host(const pyr_shape* s, const void* Q, const void* K
   const ChunkLayout c = layout_for(s, P, nqb, upc, lse != nullptr);
   if (workspace_bytes < c.total) return PYR_EINVAL;
 
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PYR_ECUDA;
-  DeviceStreams& ds = g_dev[dev];
+  DeviceStreams* dsp = streams_for_current_context();
+  if (!dsp) return PYR_ECUDA;
+  DeviceStreams& ds = *dsp;
   std::lock_guard<std::mutex> lock(ds.mu);
   if (init_streams(ds) != cudaSuccess) return PYR_ECUDA;
 
