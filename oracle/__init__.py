@@ -34,6 +34,30 @@ class OraShape(ctypes.Structure):
                                              "dtype")]
 
 
+class OraSelectOpts(ctypes.Structure):
+    _fields_ = [("budget", ctypes.c_void_p), ("fcf_tau", ctypes.c_double), ("fcf_extra", ctypes.c_int),
+                ("rcg_lambda", ctypes.c_double)]
+
+
+class SelectOpts:
+    """The PHAROS selection variants (PHAROS page, "Four mechanisms powering PHAROS"); defaults = plain walk.
+
+    budget      DBA: level-0 budget of each (batch, kv head) unit ([B * Hkv] ints, clamped to [0, topk]),
+                or None for topk - fcf_extra everywhere;
+    fcf_tau,    FCF: when the walk's confidence (its smallest margin above level 0 and at the level-0
+    fcf_extra   budget boundary) is below fcf_tau, level 0 keeps fcf_extra more blocks (at most topk);
+    rcg_lambda  RCG: candidates rank by R = S + rcg_lambda * R(parent).
+    """
+
+    def __init__(self, budget=None, fcf_tau=0.0, fcf_extra=0, rcg_lambda=0.0):
+        self.budget = None if budget is None else np.ascontiguousarray(np.asarray(budget, dtype=np.int32))
+        self.fcf_tau, self.fcf_extra, self.rcg_lambda = float(fcf_tau), int(fcf_extra), float(rcg_lambda)
+
+    def c_struct(self):
+        return OraSelectOpts(None if self.budget is None else self.budget.ctypes.data, self.fcf_tau,
+                             self.fcf_extra, self.rcg_lambda)
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle (gcc -O2, OpenMP over independent units)."""
     if force or not os.path.exists(_OUT) or os.path.getmtime(_OUT) < os.path.getmtime(_SRC):
@@ -68,6 +92,13 @@ def _load():
         lib.ora_node_score.restype = ctypes.c_int
         lib.ora_select.argtypes = [sp, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P, _P]
         lib.ora_select.restype = ctypes.c_int
+        lib.ora_select_ex.argtypes = [sp, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P, ctypes.c_int,
+                                      ctypes.POINTER(OraSelectOpts), _P, _P, _P, _P]
+        lib.ora_select_ex.restype = ctypes.c_int
+        lib.ora_trace_levels.argtypes = [sp]
+        lib.ora_trace_levels.restype = ctypes.c_int
+        lib.ora_trace_width.argtypes = [sp]
+        lib.ora_trace_width.restype = ctypes.c_int
         lib.ora_attend.argtypes = [sp, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P]
         lib.ora_attend.restype = ctypes.c_int
         lib.ora_route_invert.argtypes = [sp, _P, ctypes.c_int32, _P, _P]
@@ -138,10 +169,22 @@ def node_score(w, Q, pyr_unit: np.ndarray, unit: int, qb: int, level: int, m: in
     return s.value, n.value
 
 
-def select(w, Q, pyr: np.ndarray, units, items, start_level: int = -1):
+def trace_levels(w) -> int:
+    """Levels of a selection trace: the start level s0 down to 0 (s0 + 1)."""
+    return _load().ora_trace_levels(ctypes.byref(shape_of(w)))
+
+
+def trace_width(w) -> int:
+    """Entries per trace level: max(cap / 2, topk)."""
+    return _load().ora_trace_width(ctypes.byref(shape_of(w)))
+
+
+def select(w, Q, pyr: np.ndarray, units, items, start_level: int = -1, opts: SelectOpts = None,
+           with_trace: bool = False):
     """Selection for items [(slot, qb), ...]; slot indexes ``units`` / ``pyr``.
 
-    Returns (idx [n, topk] int32, gap [n] float64, ncand [n, L+1] int32).
+    Returns (idx [n, topk] int32, gap [n] float64, ncand [n, L+1] int32), plus, with with_trace,
+    trace [n, levels, width] int32: row s0 - l lists the nodes kept at level l, best first, then -1.
     """
     units = np.ascontiguousarray(np.asarray(units, dtype=np.int32))
     items = np.asarray(items, dtype=np.int64).reshape(-1, 2)
@@ -152,21 +195,29 @@ def select(w, Q, pyr: np.ndarray, units, items, start_level: int = -1):
     gap = np.empty(n, dtype=np.float64)
     ncand = np.empty((n, num_levels(w)), dtype=np.int32)
     pyr = np.ascontiguousarray(pyr)
-    rc = _load().ora_select(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(pyr), len(units), _ptr(units), n, _ptr(slot),
-                            _ptr(qb), start_level, _ptr(idx), _ptr(gap), _ptr(ncand))
+    tl = trace_levels(w) if start_level < 0 else min(start_level, num_levels(w) - 1) + 1
+    trace = np.empty((n, tl, trace_width(w)), dtype=np.int32) if with_trace else None
+    if opts is not None and opts.budget is not None:
+        assert len(opts.budget) == w.B * w.Hkv
+    co = opts.c_struct() if opts is not None else None
+    rc = _load().ora_select_ex(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(pyr), len(units), _ptr(units), n,
+                               _ptr(slot), _ptr(qb), start_level, ctypes.byref(co) if co is not None else None,
+                               _ptr(idx), _ptr(gap), _ptr(ncand), None if trace is None else _ptr(trace))
     if rc:
-        raise ValueError(f"ora_select rc={rc}")
+        raise ValueError(f"ora_select_ex rc={rc}")
+    if with_trace:
+        return idx[:, :w.topk], gap, ncand, trace
     return idx[:, :w.topk], gap, ncand
 
 
-def select_all(w, Q, K, units=None, start_level: int = -1):
+def select_all(w, Q, K, units=None, start_level: int = -1, opts: SelectOpts = None):
     """Full selection for the listed units (default: all): idx [U, nqb, topk], gap [U, nqb], ncand."""
     if units is None:
         units = list(range(w.B * w.Hkv))
     pyr = pyramid(w, K, units)
     nqb = num_qblocks(w)
     items = [(s, q) for s in range(len(units)) for q in range(nqb)]
-    idx, gap, ncand = select(w, Q, pyr, units, items, start_level)
+    idx, gap, ncand = select(w, Q, pyr, units, items, start_level, opts)
     return idx.reshape(len(units), nqb, w.topk), gap.reshape(len(units), nqb), ncand.reshape(len(units), nqb, -1)
 
 

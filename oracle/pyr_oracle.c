@@ -273,14 +273,59 @@ static int cmp_i32(const void* a, const void* b) {
 }
 
 /*
+ * Selection variants of the PHAROS page ("Four mechanisms powering PHAROS"),
+ * all off by default (a zeroed struct or NULL gives the plain walk above):
+ *   budget     depth-sounding budget allocation (DBA): token budgets differ
+ *              across heads. budget[unit] (unit = batch * Hkv + kv head) is
+ *              the number of level-0 blocks that unit's walk keeps, clamped
+ *              to [0, topk]; NULL: topk - fcf_extra for every unit. The page
+ *              derives budgets from attention-head entropy but gives no
+ *              formula, so the budgets are an input.
+ *   fcf_tau,   fog-gate confidence fallback (FCF): the budget grows when
+ *   fcf_extra  confidence is low. Confidence is the walk's smallest margin
+ *              between the last kept and the first dropped candidate over the
+ *              levels above 0 and at the level-0 budget boundary; when it is
+ *              below fcf_tau, level 0 keeps min(budget + fcf_extra, topk).
+ *              fcf_extra = 0: off.
+ *   rcg_lambda range-light cross-level guidance (RCG): coarse-level scores
+ *              guide the finer levels. Candidates are ranked by
+ *              R = S + rcg_lambda * R(parent), R = S at the start level;
+ *              0: off (rank by S).
+ */
+typedef struct {
+  const int32_t* budget; /* [B * Hkv] or NULL */
+  double fcf_tau;
+  int fcf_extra;
+  double rcg_lambda;
+} ora_select_opts;
+
+/* Levels a trace holds: the start level s0 (the finest level with at most cap
+ * nodes) down to 0. */
+int ora_trace_levels(const ora_shape* s) {
+  const int64_t nb = num_blocks(s);
+  int s0 = 0;
+  while (level_nodes(nb, s0) > s->cap) s0++;
+  return s0 + 1;
+}
+
+/* Entries per trace level: the most nodes any level keeps. */
+int ora_trace_width(const ora_shape* s) { return s->cap / 2 > s->topk ? s->cap / 2 : s->topk; }
+
+/*
  * Selection for (unit, query block i). Writes idx[0..topk) (ascending, -1
  * padded), *gap, and, when ncand is given, the number of candidates scored at
- * each level (ncand[l], l = 0..L; zero for levels not scored).
+ * each level (ncand[l], l = 0..L; zero for levels not scored). When trace is
+ * given ([s0 + 1][ora_trace_width] entries), row s0 - l lists the nodes kept at
+ * level l, best first, then -1.
  * start_level < 0 starts at s0; otherwise at the given level (used by tests
  * to check that starting at the root gives the same answer).
+ * gap is the smallest margin of any decision the walk took: last kept minus
+ * first dropped at every level that dropped a candidate (at the level-0
+ * boundary actually used) and, when FCF could change the result, the distance
+ * between the confidence and fcf_tau.
  */
 static void select_one(const ora_shape* s, const void* Q, const double* pyr, int64_t unit, int64_t i, int start_level,
-                       int32_t* idx, double* gap, int32_t* ncand) {
+                       const ora_select_opts* opt, int32_t* idx, double* gap, int32_t* ncand, int32_t* trace) {
   const int d = s->d, G = s->Hq / s->Hkv;
   const int64_t nb = num_blocks(s);
   const int L = top_level(nb);
@@ -288,39 +333,83 @@ static void select_one(const ora_shape* s, const void* Q, const double* pyr, int
   double* rows = (double*)malloc(sizeof(double) * (size_t)G * s->b * d);
   double* kbar = (double*)malloc(sizeof(double) * (size_t)d);
   const int nr = gather_rows(s, Q, bi, hk, i, rows);
+  const int extra = opt ? opt->fcf_extra : 0;
+  const double lambda = opt ? opt->rcg_lambda : 0.0;
+  int base = (opt && opt->budget) ? opt->budget[unit] : s->topk - extra;
+  if (base < 0) base = 0;
+  if (base > s->topk) base = s->topk;
 
   int s0 = 0;
   while (level_nodes(nb, s0) > s->cap) s0++;
   if (start_level >= 0) s0 = start_level > L ? L : start_level;
+  const int tw = ora_trace_width(s);
+  if (trace)
+    for (int k = 0; k < (s0 + 1) * tw; k++) trace[k] = -1;
 
-  /* candidate lists hold at most max(cap, n_s0) nodes */
+  /* candidate lists hold at most max(cap, n_s0) nodes; score is the ranking
+   * score R, parent the parent's R (0 at the start level) */
   int64_t room = level_nodes(nb, s0);
   if (room < s->cap) room = s->cap;
   if (room < 2) room = 2;
   cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)room * 2);
   cand_t* next = (cand_t*)malloc(sizeof(cand_t) * (size_t)room * 2);
+  double* parent = (double*)malloc(sizeof(double) * (size_t)room * 2);
+  double* next_parent = (double*)malloc(sizeof(double) * (size_t)room * 2);
   int nc = 0;
   for (int64_t m = 0; m < level_nodes(nb, s0); m++)
-    if ((m << s0) < i) cand[nc++].m = m;
+    if ((m << s0) < i) {
+      parent[nc] = 0.0;
+      cand[nc++].m = m;
+    }
 
   if (ncand)
     for (int l = 0; l <= L; l++) ncand[l] = 0;
-  double g = INFINITY;
+  double g = INFINITY;    /* smallest decision margin */
+  double conf = INFINITY; /* smallest margin above level 0 (FCF confidence) */
   for (int k = 0; k < s->topk; k++) idx[k] = -1;
 
   for (int l = s0; l >= 0; l--) {
     for (int c = 0; c < nc; c++) {
-      double nv;
-      node_score(s, pyr, rows, nr, i, l, cand[c].m, kbar, &cand[c].score, &nv);
+      double nv, sc;
+      node_score(s, pyr, rows, nr, i, l, cand[c].m, kbar, &sc, &nv);
+      cand[c].score = sc + lambda * parent[c];
     }
     if (ncand) ncand[l] = nc;
     sort_candidates(cand, nc);
-    const int want = l > 0 ? s->cap / 2 : s->topk;
-    const int keep = nc < want ? nc : want;
-    if (keep < nc && keep > 0) {
-      const double gl = cand[keep - 1].score - cand[keep].score;
-      if (gl < g) g = gl;
+    int keep;
+    if (l > 0) {
+      const int want = s->cap / 2;
+      keep = nc < want ? nc : want;
+      if (keep < nc && keep > 0) {
+        const double gl = cand[keep - 1].score - cand[keep].score;
+        if (gl < g) g = gl;
+        if (gl < conf) conf = gl;
+      }
+    } else {
+      const int keep_base = nc < base ? nc : base;
+      keep = keep_base;
+      if (extra > 0) {
+        double c0 = conf;
+        if (keep_base < nc && keep_base > 0) {
+          const double gb = cand[keep_base - 1].score - cand[keep_base].score;
+          if (gb < c0) c0 = gb;
+        }
+        int wide = base + extra < s->topk ? base + extra : s->topk;
+        if (wide > nc) wide = nc;
+        if (c0 < opt->fcf_tau) keep = wide;
+        if (wide != keep_base) {
+          /* the fallback decision changes the result: its margin counts */
+          const double gt = fabs(c0 - opt->fcf_tau);
+          if (gt < g) g = gt;
+        }
+      }
+      if (keep < nc && keep > 0) {
+        const double gl = cand[keep - 1].score - cand[keep].score;
+        if (gl < g) g = gl;
+      }
     }
+    if (trace)
+      for (int k = 0; k < keep; k++) trace[(s0 - l) * tw + k] = (int32_t)cand[k].m;
     if (l == 0) {
       for (int k = 0; k < keep; k++) idx[k] = (int32_t)cand[k].m;
       qsort(idx, (size_t)keep, sizeof(int32_t), cmp_i32);
@@ -330,15 +419,23 @@ static void select_one(const ora_shape* s, const void* Q, const double* pyr, int
     int nn = 0;
     for (int k = 0; k < keep; k++)
       for (int64_t ch = 2 * cand[k].m; ch <= 2 * cand[k].m + 1; ch++)
-        if (ch < nchild && (ch << (l - 1)) < i) next[nn++].m = ch;
+        if (ch < nchild && (ch << (l - 1)) < i) {
+          next_parent[nn] = cand[k].score;
+          next[nn++].m = ch;
+        }
     cand_t* t = cand;
     cand = next;
     next = t;
+    double* tp = parent;
+    parent = next_parent;
+    next_parent = tp;
     nc = nn;
   }
   *gap = g;
   free(cand);
   free(next);
+  free(parent);
+  free(next_parent);
   free(rows);
   free(kbar);
 }
@@ -347,28 +444,44 @@ static void select_one(const ora_shape* s, const void* Q, const double* pyr, int
  * Selection for a list of items. Item k is (slot[k], qb[k]): slot indexes
  * units[] and pyr ([nunits][P][d], the pyramids of those units, as written
  * by ora_pyramid); qb is the query block relative to the first query block.
- * idx: [nitems][topk]; gap: [nitems] (nullable); ncand: [nitems][L+1]
- * (nullable).
+ * opt: the PHAROS variants (NULL: plain walk); opt->budget is indexed by the
+ * global unit id units[slot]. idx: [nitems][topk]; gap: [nitems] (nullable);
+ * ncand: [nitems][L+1] (nullable); trace: [nitems][levels][width] with
+ * levels = s0 + 1 of the walk's start level (ora_trace_levels unless
+ * start_level is given) and width = ora_trace_width (nullable).
  */
-int ora_select(const ora_shape* s, const void* Q, const double* pyr, int nunits, const int32_t* units, int nitems,
-               const int32_t* slot, const int64_t* qb, int start_level, int32_t* idx, double* gap,
-               int32_t* ncand) {
+int ora_select_ex(const ora_shape* s, const void* Q, const double* pyr, int nunits, const int32_t* units, int nitems,
+                  const int32_t* slot, const int64_t* qb, int start_level, const ora_select_opts* opt, int32_t* idx,
+                  double* gap, int32_t* ncand, int32_t* trace) {
   if (!s || !Q || !pyr || !units || !slot || !qb || !idx) return ORA_EINVAL;
   if (s->cap < 2 || s->cap % 2 || s->topk < 0 || s->Hq % s->Hkv) return ORA_EINVAL;
+  if (opt && (opt->fcf_extra < 0 || opt->fcf_tau != opt->fcf_tau || opt->rcg_lambda != opt->rcg_lambda))
+    return ORA_EINVAL;
   const int64_t P = ora_num_nodes(s);
   const int nl = ora_num_levels(s);
   const int64_t nqb = ora_num_qblocks(s);
+  int tl = ora_trace_levels(s);
+  if (start_level >= 0) tl = (start_level > nl - 1 ? nl - 1 : start_level) + 1;
+  const int64_t tstride = (int64_t)tl * ora_trace_width(s);
   for (int k = 0; k < nitems; k++)
     if (slot[k] < 0 || slot[k] >= nunits || qb[k] < 0 || qb[k] >= nqb) return ORA_EINVAL;
 #pragma omp parallel for schedule(dynamic)
   for (int k = 0; k < nitems; k++) {
     double gk;
     const int64_t i = ora_first_qblock(s) + qb[k];
-    select_one(s, Q, pyr + (int64_t)slot[k] * P * s->d, units[slot[k]], i, start_level,
-               idx + (int64_t)k * s->topk, &gk, ncand ? ncand + (int64_t)k * nl : NULL);
+    select_one(s, Q, pyr + (int64_t)slot[k] * P * s->d, units[slot[k]], i, start_level, opt,
+               idx + (int64_t)k * s->topk, &gk, ncand ? ncand + (int64_t)k * nl : NULL,
+               trace ? trace + k * tstride : NULL);
     if (gap) gap[k] = gk;
   }
   return ORA_OK;
+}
+
+/* The plain walk (no PHAROS variant, no trace). */
+int ora_select(const ora_shape* s, const void* Q, const double* pyr, int nunits, const int32_t* units, int nitems,
+               const int32_t* slot, const int64_t* qb, int start_level, int32_t* idx, double* gap,
+               int32_t* ncand) {
+  return ora_select_ex(s, Q, pyr, nunits, units, nitems, slot, qb, start_level, NULL, idx, gap, ncand, NULL);
 }
 
 /* ---- step 4: causal block-sparse attention ----------------------------- */
