@@ -101,6 +101,10 @@ def _load():
         lib.ora_trace_width.restype = ctypes.c_int
         lib.ora_attend.argtypes = [sp, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P, _P]
         lib.ora_attend.restype = ctypes.c_int
+        lib.ora_prefix_states.argtypes = [sp, ctypes.c_int, _P, _P, _P, _P, ctypes.c_int, _P, _P, _P]
+        lib.ora_prefix_states.restype = ctypes.c_int
+        lib.ora_attend_states.argtypes = [sp, _P, _P, _P, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P, _P, _P, _P]
+        lib.ora_attend_states.restype = ctypes.c_int
         lib.ora_route_invert.argtypes = [sp, _P, ctypes.c_int32, _P, _P]
         lib.ora_route_invert.restype = ctypes.c_int
         lib.ora_attend_bwd_q.argtypes = [sp, _P, _P, _P, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P]
@@ -240,6 +244,52 @@ def attend(w, Q, K, V, idx, rows, dense: bool = False):
         raise ValueError("ora_attend: idx lists a block that is not strictly before the query block, or repeats")
     if rc:
         raise ValueError(f"ora_attend rc={rc}")
+    return O, lse
+
+
+# ---- PHBA prefix-state branch (PHBA summary, 2.2, 3.2, 3.3, A.1.1, A.1.3) ----
+
+def prefix_states(w, M: int, Ks, V, A, W, units=None):
+    """Prefix states of the listed units (default: all): (PK, PV) [len(units), nb, M, d] float64.
+
+    Ks (state-branch keys) and V: [B, Hkv, N, d] in the workload dtype; A (retention) and W (write):
+    [B, Hkv, N, M] float32. Slot s of the key state follows SK <- A_t[s] SK + W_t[s] k_t (the value
+    state likewise, with v_t), from zero; block j's state is taken after the tokens before j * b."""
+    if units is None:
+        units = list(range(w.B * w.Hkv))
+    units = np.ascontiguousarray(np.asarray(units, dtype=np.int32))
+    nb = (w.N + w.b - 1) // w.b
+    PK = np.empty((len(units), nb, M, w.d), dtype=np.float64)
+    PV = np.empty_like(PK)
+    A = A.contiguous() if isinstance(A, torch.Tensor) else np.ascontiguousarray(A, dtype=np.float32)
+    W = W.contiguous() if isinstance(W, torch.Tensor) else np.ascontiguousarray(W, dtype=np.float32)
+    rc = _load().ora_prefix_states(ctypes.byref(shape_of(w)), M, _ptr(Ks), _ptr(V), _ptr(A), _ptr(W), len(units),
+                                   _ptr(units), _ptr(PK), _ptr(PV))
+    if rc:
+        raise ValueError(f"ora_prefix_states rc={rc}")
+    return PK, PV
+
+
+def attend_states(w, Q, K, V, idx, rows, PK, PV, Qs=None):
+    """Attention of flat query rows over tokens and prefix-state slots: (O [n, d], lse [n]) float64.
+
+    PK, PV: [B * Hkv, nb, M, d] float64 (the states of every unit); Qs: the state branch's query
+    (None: Q)."""
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = len(rows)
+    O = np.empty((n, w.d), dtype=np.float64)
+    lse = np.empty(n, dtype=np.float64)
+    M = 0 if PK is None else PK.shape[2]
+    PK = None if PK is None else np.ascontiguousarray(PK, dtype=np.float64)
+    PV = None if PV is None else np.ascontiguousarray(PV, dtype=np.float64)
+    rc = _load().ora_attend_states(ctypes.byref(shape_of(w)), _ptr(Q), _ptr(K), _ptr(V), _ptr(_idx_arr(idx)), n,
+                                   _ptr(rows), None if Qs is None else _ptr(Qs), M,
+                                   None if PK is None else _ptr(PK), None if PV is None else _ptr(PV), _ptr(O),
+                                   _ptr(lse))
+    if rc == 2:
+        raise ValueError("ora_attend_states: idx lists a block that is not strictly before the query block, or repeats")
+    if rc:
+        raise ValueError(f"ora_attend_states rc={rc}")
     return O, lse
 
 

@@ -496,11 +496,16 @@ int ora_select(const ora_shape* s, const void* Q, const double* pyr, int nunits,
  * idx: [B][Hkv][nqb][topk]. O: [nrows][d]; lse: [nrows] (natural log).
  * Returns ORA_EBADIDX if a listed block is not strictly before i or repeats.
  */
-int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, int nrows,
-               const int64_t* rows, int dense, double* O, double* lse) {
-  if (!s || !Q || !K || !V || !rows || !O || !lse || (!dense && !idx)) return ORA_EINVAL;
+/*
+ * Rows of attention. With M > 0 the prefix states take part too (PHBA
+ * prefix-state branch, below): PK, PV are [B*Hkv][nb][M][d] and Qs (NULL: Q)
+ * is the query the state slots are scored with.
+ */
+static int attend_rows(const ora_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, int nrows,
+                       const int64_t* rows, int dense, const void* Qs, int M, const double* PK, const double* PV,
+                       double* O, double* lse) {
   const int d = s->d, G = s->Hq / s->Hkv;
-  const int64_t nqb = ora_num_qblocks(s), first = ora_first_qblock(s);
+  const int64_t nqb = ora_num_qblocks(s), first = ora_first_qblock(s), nb = num_blocks(s);
   const double scale = 1.0 / sqrt((double)d);
   int bad = 0;
 #pragma omp parallel for schedule(dynamic) reduction(| : bad)
@@ -509,10 +514,11 @@ int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, 
     const int64_t bi = bh / s->Hq, hq = bh % s->Hq, hk = hq / G;
     const int64_t p = s->q_offset + t, i = p / s->b;
     const int64_t qbase = rows[r] * d, kvbase = (bi * s->Hkv + hk) * (int64_t)s->N * d;
-    /* the attended key positions, in any order */
+    /* the attended key positions, in any order; with states, the attended state blocks */
     int64_t cap_keys = dense ? p + 1 : (int64_t)(s->topk + 1) * s->b;
     int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap_keys);
-    int64_t nk = 0;
+    int64_t* sblk = (int64_t*)malloc(sizeof(int64_t) * (size_t)(s->topk + 1));
+    int64_t nk = 0, ns = 0;
     if (dense) {
       for (int64_t k = 0; k <= p; k++) keys[nk++] = k;
     } else {
@@ -527,10 +533,13 @@ int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, 
           continue;
         }
         for (int64_t x = j * s->b; x < (j + 1) * s->b && x < s->N; x++) keys[nk++] = x;
+        if (M > 0 && j >= 1) sblk[ns++] = j; /* the prefix state aligned with routed block j */
       }
       for (int64_t x = i * s->b; x <= p; x++) keys[nk++] = x;
+      if (M > 0 && i >= 1) sblk[ns++] = i; /* the current block's prefix state */
     }
-    double* sc = (double*)malloc(sizeof(double) * (size_t)nk);
+    const int64_t nslot = ns * M;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)(nk + nslot + 1));
     double mx = -INFINITY;
     for (int64_t k = 0; k < nk; k++) {
       double dot = 0.0;
@@ -538,19 +547,113 @@ int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, 
       sc[k] = dot * scale;
       if (sc[k] > mx) mx = sc[k];
     }
+    const void* qs = Qs ? Qs : Q;
+    const int64_t sbase = (bi * s->Hkv + hk) * nb * (int64_t)M * d;
+    for (int64_t c = 0; c < nslot; c++) {
+      const double* key = PK + sbase + (sblk[c / M] * M + c % M) * d;
+      double dot = 0.0;
+      for (int e = 0; e < d; e++) dot += elem(qs, s->dtype, qbase + e) * key[e];
+      sc[nk + c] = dot * scale;
+      if (sc[nk + c] > mx) mx = sc[nk + c];
+    }
     double sum = 0.0;
-    for (int64_t k = 0; k < nk; k++) sum += exp(sc[k] - mx);
+    for (int64_t k = 0; k < nk + nslot; k++) sum += exp(sc[k] - mx);
     const double l = mx + log(sum);
     for (int e = 0; e < d; e++) O[(int64_t)r * d + e] = 0.0;
     for (int64_t k = 0; k < nk; k++) {
       const double w = exp(sc[k] - l);
       for (int e = 0; e < d; e++) O[(int64_t)r * d + e] += w * elem(V, s->dtype, kvbase + keys[k] * d + e);
     }
+    for (int64_t c = 0; c < nslot; c++) {
+      const double w = exp(sc[nk + c] - l);
+      const double* val = PV + sbase + (sblk[c / M] * M + c % M) * d;
+      for (int e = 0; e < d; e++) O[(int64_t)r * d + e] += w * val[e];
+    }
     lse[r] = l;
     free(sc);
     free(keys);
+    free(sblk);
   }
   return bad ? ORA_EBADIDX : ORA_OK;
+}
+
+int ora_attend(const ora_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, int nrows,
+               const int64_t* rows, int dense, double* O, double* lse) {
+  if (!s || !Q || !K || !V || !rows || !O || !lse || (!dense && !idx)) return ORA_EINVAL;
+  return attend_rows(s, Q, K, V, idx, nrows, rows, dense, NULL, 0, NULL, NULL, O, lse);
+}
+
+/* ---- PHBA prefix-state branch ----------------------------------------- */
+/*
+ * PHBA summary, 2.2 "Gated slot memory", 3.2 "Prefix-state construction" and
+ * A.1.1: gated recurrences build a prefix-key and a prefix-value state of M
+ * slots each; the state stored immediately before a block summarises only the
+ * causal context before it; the key and the value recurrence share one
+ * slot-wise retention gate and one write gate; the recurrence starts from a
+ * zero state at the start of a sequence.
+ * Reading (the summary prints no formula): with state-branch key k_t, value
+ * v_t, retention a_t[s] and write w_t[s] of token t (slot s = 0 .. M-1),
+ *   SK[s] <- a_t[s] SK[s] + w_t[s] k_t,    SV[s] <- a_t[s] SV[s] + w_t[s] v_t,
+ * from SK = SV = 0 before position 0, token by token; the prefix state of key
+ * block j is (SK, SV) after the tokens at positions < j b, so block 0's is
+ * zero. Written here as that plain sequential recurrence in double.
+ */
+static void prefix_states_unit(const ora_shape* s, int M, const void* Ks, const void* V, const float* A,
+                               const float* W, int64_t unit, double* PK, double* PV) {
+  const int d = s->d;
+  double* SK = (double*)calloc((size_t)M * d, sizeof(double));
+  double* SV = (double*)calloc((size_t)M * d, sizeof(double));
+  const int64_t xbase = unit * (int64_t)s->N * d, gbase = unit * (int64_t)s->N * M;
+  for (int64_t t = 0; t < s->N; t++) {
+    if (t % s->b == 0) {
+      const int64_t j = t / s->b;
+      memcpy(PK + j * M * d, SK, sizeof(double) * (size_t)M * d);
+      memcpy(PV + j * M * d, SV, sizeof(double) * (size_t)M * d);
+    }
+    for (int m = 0; m < M; m++) {
+      const double a = A[gbase + t * M + m], w = W[gbase + t * M + m];
+      for (int e = 0; e < d; e++) {
+        SK[m * d + e] = a * SK[m * d + e] + w * elem(Ks, s->dtype, xbase + t * d + e);
+        SV[m * d + e] = a * SV[m * d + e] + w * elem(V, s->dtype, xbase + t * d + e);
+      }
+    }
+  }
+  free(SK);
+  free(SV);
+}
+
+/*
+ * Prefix states of the listed units: PK, PV [nunits][nb][M][d] (double).
+ * Ks (state-branch keys) and V: [B][Hkv][N][d] in s->dtype; A (retention)
+ * and W (write): [B][Hkv][N][M] float32.
+ */
+int ora_prefix_states(const ora_shape* s, int M, const void* Ks, const void* V, const float* A, const float* W,
+                      int nunits, const int32_t* units, double* PK, double* PV) {
+  if (!s || !Ks || !V || !A || !W || !units || !PK || !PV || M <= 0) return ORA_EINVAL;
+  const int64_t per = num_blocks(s) * (int64_t)M * s->d;
+#pragma omp parallel for schedule(dynamic)
+  for (int u = 0; u < nunits; u++) prefix_states_unit(s, M, Ks, V, A, W, units[u], PK + u * per, PV + u * per);
+  return ORA_OK;
+}
+
+/*
+ * PHBA summary, 3.3 "Online-softmax token-state attention" and A.1.3: the
+ * output is one softmax over the exact tokens (the routed blocks and the
+ * current block up to the query's position) and the prefix-state slots: the
+ * current block's prefix state and the prefix state aligned with each routed
+ * block. Token scores use the (rotated) query and keys, state scores the raw
+ * query against the raw state keys; the values are V and the value states.
+ * Readings: a slot's score is qs . PK[slot] / sqrt(d), the token branch's
+ * scale; a block whose causal prefix is empty (block 0) brings no state (the
+ * PrefixValid flag of PHBA A.1.2); Qs NULL means the state branch uses Q (the
+ * rotation of the pages' models is outside this library).
+ * PK, PV: [B*Hkv][nb][M][d] double, as ora_prefix_states writes for all units.
+ */
+int ora_attend_states(const ora_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, int nrows,
+                      const int64_t* rows, const void* Qs, int M, const double* PK, const double* PV, double* O,
+                      double* lse) {
+  if (!s || !Q || !K || !V || !idx || !rows || !O || !lse || M < 0 || (M > 0 && (!PK || !PV))) return ORA_EINVAL;
+  return attend_rows(s, Q, K, V, idx, nrows, rows, 0, Qs, M, PK, PV, O, lse);
 }
 
 /* ---- backward: block-major route metadata and gradients ----------------- */
