@@ -10,6 +10,9 @@ every call needs CUDA tensors.
     pyr_build(shape, K, pyr)                  key pyramid (mean pooling)
     pyr_update(shape, K, pyr, from_pos)       refresh the nodes over rewritten key positions
     pyr_select(shape, Q, pyr, idx, gap)       coarse-to-fine LogSumExp top-K
+    pyr_select_ex(shape, Q, pyr, idx, gap, opts)
+                                              the same with the PHAROS variants (per-head budget,
+                                              confidence fallback, cross-level guidance) and a trace
     bsa_forward(shape, Q, K, V, idx, O, lse)  causal block-sparse attention
     dense_forward(shape, Q, K, V, O, lse)     dense causal attention
     bsa_route_invert(shape, idx, offset, rho) routes in block-major form (for the backward)
@@ -31,8 +34,9 @@ PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = ran
 PYR_F32, PYR_BF16 = 0, 1
 
 ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_pyramid_elems", "pyr_build", "pyr_update",
-               "pyr_select", "bsa_forward", "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes",
-               "bsa_route_invert", "bsa_backward", "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
+               "pyr_select", "pyr_select_ex", "pyr_select_trace_levels", "pyr_select_trace_width", "bsa_forward",
+               "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes", "bsa_route_invert", "bsa_backward",
+               "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
 
 
 class PyrShape(ctypes.Structure):
@@ -41,6 +45,11 @@ class PyrShape(ctypes.Structure):
 
     def __repr__(self):
         return "PyrShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class PyrSelectOpts(ctypes.Structure):
+    _fields_ = [("budget", ctypes.c_void_p), ("fcf_tau", ctypes.c_float), ("fcf_extra", ctypes.c_int),
+                ("rcg_lambda", ctypes.c_float), ("trace", ctypes.c_void_p)]
 
 
 class PyrError(RuntimeError):
@@ -70,6 +79,12 @@ def _load_lib():
     lib.pyr_update.restype = ctypes.c_int
     lib.pyr_select.argtypes = [sp, vp, vp, vp, vp, vp, vp]
     lib.pyr_select.restype = ctypes.c_int
+    lib.pyr_select_ex.argtypes = [sp, vp, vp, ctypes.POINTER(PyrSelectOpts), vp, vp, vp, vp]
+    lib.pyr_select_ex.restype = ctypes.c_int
+    lib.pyr_select_trace_levels.argtypes = [sp]
+    lib.pyr_select_trace_levels.restype = ctypes.c_int
+    lib.pyr_select_trace_width.argtypes = [sp]
+    lib.pyr_select_trace_width.restype = ctypes.c_int
     lib.bsa_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.bsa_forward.restype = ctypes.c_int
     lib.dense_forward.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp]
@@ -170,6 +185,31 @@ def pyr_update(s: PyrShape, K, pyr, from_pos: int, status=None, stream=None):
 def pyr_select(s: PyrShape, Q, pyr, idx, gap=None, status=None, stream=None):
     _check(_L().pyr_select(ctypes.byref(s), _dev(Q, "Q"), _dev(pyr, "pyr"), _dev(idx, "idx"),
                            _dev(gap, "gap", True), _dev(status, "status", True), _stream(stream)), "pyr_select")
+
+
+def select_trace_levels(s: PyrShape) -> int:
+    return _L().pyr_select_trace_levels(ctypes.byref(s))
+
+
+def select_trace_width(s: PyrShape) -> int:
+    return _L().pyr_select_trace_width(ctypes.byref(s))
+
+
+def new_trace(s: PyrShape, device="cuda"):
+    """A trace buffer [B, Hkv, nqb, levels, width] int32 for pyr_select_ex."""
+    return torch.empty((s.B, s.Hkv, num_qblocks(s), select_trace_levels(s), select_trace_width(s)),
+                       dtype=torch.int32, device=device)
+
+
+def pyr_select_ex(s: PyrShape, Q, pyr, idx, gap=None, budget=None, fcf_tau: float = 0.0, fcf_extra: int = 0,
+                  rcg_lambda: float = 0.0, trace=None, status=None, stream=None):
+    """pyr_select with the PHAROS variants: budget (int32 CUDA tensor [B, Hkv], DBA), fcf_tau / fcf_extra
+    (FCF), rcg_lambda (RCG), and an optional trace buffer (new_trace)."""
+    o = PyrSelectOpts(_dev(budget, "budget", True), float(fcf_tau), int(fcf_extra), float(rcg_lambda),
+                      _dev(trace, "trace", True))
+    _check(_L().pyr_select_ex(ctypes.byref(s), _dev(Q, "Q"), _dev(pyr, "pyr"), ctypes.byref(o), _dev(idx, "idx"),
+                              _dev(gap, "gap", True), _dev(status, "status", True), _stream(stream)),
+           "pyr_select_ex")
 
 
 def bsa_forward(s: PyrShape, Q, K, V, idx, O, lse=None, status=None, stream=None):

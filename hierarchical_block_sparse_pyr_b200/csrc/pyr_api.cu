@@ -1,9 +1,11 @@
 // C ABI of libpyr: argument validation, geometry, dispatch to the kernels.
 // Every entry point validates on the host, enqueues on the caller's stream
 // and returns; nothing here allocates device memory or synchronises.
+#include <cuda.h>
 #include <stdint.h>
 
 #include "pyr_common.cuh"
+#include "select_opts.cuh"
 
 namespace pyr {
 size_t select_smem_bytes(const Geo& g);
@@ -71,6 +73,37 @@ int pyr::validate_shape(const pyr_shape* s) {
   return make_geo(s, &g);
 }
 
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+}  // namespace
+
+bool pyr::current_context_id(unsigned long long* id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id || !id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) {
+    // no context bound to this thread yet: bind the current device's primary context, as the
+    // first runtime call on the thread would
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return false;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 extern "C" {
 
 int pyr_num_levels(const pyr_shape* s) {
@@ -111,19 +144,46 @@ int pyr_update(const pyr_shape* s, const void* K, void* pyr, int from_pos, int* 
       pyr::launch_pyramid_update(g, K, static_cast<__nv_bfloat16*>(pyr), from_pos, dev_status, (cudaStream_t)stream));
 }
 
-int pyr_select(const pyr_shape* s, const void* Q, const void* pyr_v, int32_t* idx, float* gap, int* dev_status,
-               void* stream) {
+int pyr_select_trace_levels(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? g.s0 + 1 : 0;
+}
+
+int pyr_select_trace_width(const pyr_shape* s) {
+  Geo g;
+  return make_geo(s, &g) == PYR_OK ? (s->cap / 2 > s->topk ? s->cap / 2 : s->topk) : 0;
+}
+
+int pyr_select_ex(const pyr_shape* s, const void* Q, const void* pyr_v, const pyr_select_opts* opts, int32_t* idx,
+                  float* gap, int* dev_status, void* stream) {
   Geo g;
   int rc = make_geo(s, &g);
   if (rc) return rc;
   const __nv_bfloat16* pyr = static_cast<const __nv_bfloat16*>(pyr_v);
   if (!Q || !pyr || !idx || !aligned16(Q) || !aligned16(pyr) || !aligned16(idx)) return PYR_EINVAL;
-  if (pyr::select_tc_supported(g))
-    return launch_status(pyr::launch_select_tc(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
-  if (pyr::select_decode_supported(g))
-    return launch_status(pyr::launch_select_decode(g, Q, pyr, idx, gap, (cudaStream_t)stream));
+  pyr::SelOpts o = {nullptr, 0.f, 0, 0.f, nullptr, 0};
+  if (opts) {
+    // NaN or infinite guidance weights and NaN thresholds have no meaning; tau may be +-inf
+    if (opts->fcf_extra < 0 || opts->fcf_tau != opts->fcf_tau || !(fabsf(opts->rcg_lambda) < INFINITY))
+      return PYR_EINVAL;
+    if (((uintptr_t)opts->budget & 3u) || ((uintptr_t)opts->trace & 3u)) return PYR_EINVAL;
+    o.budget = opts->budget;
+    o.fcf_tau = opts->fcf_tau;
+    o.fcf_extra = opts->fcf_extra;
+    o.rcg_lambda = opts->rcg_lambda;
+    o.trace = opts->trace;
+    o.tw = s->cap / 2 > s->topk ? s->cap / 2 : s->topk;
+  }
+  const cudaStream_t st = (cudaStream_t)stream;
+  if (pyr::select_tc_supported(g)) return launch_status(pyr::launch_select_tc(g, Q, pyr, idx, gap, dev_status, o, st));
+  if (pyr::select_decode_supported(g)) return launch_status(pyr::launch_select_decode(g, Q, pyr, idx, gap, o, st));
   if (pyr::select_smem_bytes(g) > 227 * 1024) return PYR_EUNSUPPORTED;
-  return launch_status(pyr::launch_select(g, Q, pyr, idx, gap, dev_status, (cudaStream_t)stream));
+  return launch_status(pyr::launch_select(g, Q, pyr, idx, gap, dev_status, o, st));
+}
+
+int pyr_select(const pyr_shape* s, const void* Q, const void* pyr, int32_t* idx, float* gap, int* dev_status,
+               void* stream) {
+  return pyr_select_ex(s, Q, pyr, nullptr, idx, gap, dev_status, stream);
 }
 
 int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, void* O,

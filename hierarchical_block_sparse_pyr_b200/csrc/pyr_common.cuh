@@ -60,6 +60,13 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
 // entry points return for this shape.
 int validate_shape(const pyr_shape* s);
 
+// Unique id (for the life of the process) of the CUDA context current on the
+// calling thread; when no context is current, the current device's primary
+// context is made current first, as any runtime call would. Device addresses of
+// __device__ variables, streams and events belong to one context, so caches of
+// them are keyed by this id rather than by device ordinal. False on failure.
+bool current_context_id(unsigned long long* id);
+
 // Launchers (one per kernel family). Each returns cudaSuccess or the launch error.
 cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int* status, cudaStream_t st);
 cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,
@@ -67,14 +74,15 @@ cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* py
 bool attn_decode_supported(const Geo& g);
 cudaError_t launch_attn_decode(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
                                int dense, void* O, float* lse, int* status, cudaStream_t st);
+struct SelOpts;  // selection variants and trace (select_opts.cuh)
 cudaError_t launch_select(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
-                          cudaStream_t st);
+                          const SelOpts& o, cudaStream_t st);
 bool select_tc_supported(const Geo& g);
 bool select_decode_supported(const Geo& g);
 cudaError_t launch_select_decode(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
-                                 cudaStream_t st);
+                                 const SelOpts& o, cudaStream_t st);
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
-                             cudaStream_t st);
+                             const SelOpts& o, cudaStream_t st);
 bool attn_tc_supported(const Geo& g);
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
                            void* O, float* lse, int* status, cudaStream_t st);

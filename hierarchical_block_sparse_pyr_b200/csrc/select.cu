@@ -15,7 +15,11 @@
 //            over the inverted node index, so ties go to the lower index),
 //            keep cap/2 (levels > 0) or topk (level 0), expand children.
 // fp32 throughout; the score matrix never leaves shared memory.
+// The PHAROS variants and the trace follow select_opts.cuh (guidance adds the
+// parent's ranking score; the level-0 keep count comes from the budget and the
+// fallback; the trace lists the kept nodes of every level).
 #include "pyr_common.cuh"
+#include "select_opts.cuh"
 
 namespace pyr {
 
@@ -28,7 +32,7 @@ constexpr int kMaxLevels = 24;
 
 struct SelSmem {
   // offsets in bytes into dynamic shared memory
-  size_t q, mt, st, colm, cols, keys, cand, nval, part, pcnt, total;
+  size_t q, mt, st, colm, cols, keys, cand, nval, part, pcnt, psc, total;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~(size_t)15; }
@@ -51,6 +55,7 @@ __host__ __device__ inline SelSmem sel_layout(int R, int d, int elt, int cap) {
   s.nval = o; o = align16(o + (size_t)kMaxCap * 4);
   s.part = o; o = align16(o + (size_t)kMaxLevels * d * 4);
   s.pcnt = o; o = align16(o + (size_t)kMaxLevels * 4);
+  s.psc = o;  o = align16(o + (size_t)2 * kMaxCap * 4);
   s.total = o;
   return s;
 }
@@ -82,7 +87,7 @@ __device__ void bitonic_desc(unsigned long long* key, int n_pow2) {
 template <typename T>
 __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ Q, const __nv_bfloat16* __restrict__ pyr,
                                                           int32_t* __restrict__ idx, float* __restrict__ gap_out,
-                                                          int* status, Geo g) {
+                                                          int* status, Geo g, SelOpts o) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int qb = blockIdx.x;
   const int unit = blockIdx.y;
@@ -107,8 +112,12 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
   float* nval = reinterpret_cast<float*>(smem + L.nval);
   float* part = reinterpret_cast<float*>(smem + L.part);  // [s0+1][d] partial means
   float* pcnt = reinterpret_cast<float*>(smem + L.pcnt);
+  float* psc = reinterpret_cast<float*>(smem + L.psc);  // parent's ranking score per candidate [2][kMaxCap]
   __shared__ int s_nc;
   __shared__ float s_gap;
+  __shared__ float s_conf;
+  const int base = sel_base_budget(o, g, unit);
+  const bool rcg = o.rcg_lambda != 0.f;
 
   for (int x = threadIdx.x; x < R * d; x += kThreads) {
     const int r = x / d, e = x - r * d;
@@ -135,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
     for (int m = 0; m < g.lvl_n[g.s0]; m++)
       if ((m << g.s0) < i) cand[nc++] = m;
     s_nc = nc;
-    s_gap = __int_as_float(0x7f800000);  // +inf
+    s_gap = s_conf = __int_as_float(0x7f800000);  // +inf
     for (int l = 0; l <= g.s0 && l < kMaxLevels; l++) pcnt[l] = (float)((int64_t)(i - ((i >> l) << l)) * g.b);
   }
   __syncthreads();
@@ -226,7 +235,8 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
     for (int c = threadIdx.x; c < np2; c += kThreads) {
       unsigned long long k = 0ull;
       if (c < nc) {
-        const float sc = colm[c] + logf(cols[c]) + logf(nval[c]);
+        float sc = colm[c] + logf(cols[c]) + logf(nval[c]);
+        if (rcg && l < g.s0) sc = fmaf(o.rcg_lambda, psc[c], sc);
         k = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)cand[c]);
       }
       keys[c] = k;
@@ -234,23 +244,45 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
     __syncthreads();
     bitonic_desc(keys, np2);
 
-    const int want = l > 0 ? g.cap / 2 : g.topk;
-    const int keep = min(want, nc);
+    const int keep_lo = min(l > 0 ? g.cap / 2 : base, nc);
+    int keep = keep_lo;
+    float decision_margin = __int_as_float(0x7f800000);
+    if (l == 0 && o.fcf_extra > 0 && keep_lo < nc) {
+      // the scores by rank, from the sorted keys (colm is free once the keys are made)
+      for (int c = threadIdx.x; c < nc; c += kThreads) colm[c] = key_to_float((uint32_t)(keys[c] >> 32));
+      __syncthreads();
+      keep = sel_fcf_keep(o, g, base, nc, colm, s_conf, &decision_margin);
+    }
+    if (o.trace) {
+      int32_t* trow = sel_trace_row(o, g, unit, qb, l);
+      for (int k = threadIdx.x; k < o.tw; k += kThreads)
+        trow[k] = k < keep ? (int)(0xFFFFFFFFu - (uint32_t)(keys[k] & 0xFFFFFFFFull)) : -1;
+    }
     if (threadIdx.x == 0) {
       if (keep < nc && keep > 0) {
         const float a = key_to_float((uint32_t)(keys[keep - 1] >> 32));
         const float b = key_to_float((uint32_t)(keys[keep] >> 32));
         s_gap = fminf(s_gap, a - b);
+        if (l > 0) s_conf = fminf(s_conf, a - b);
       }
+      s_gap = fminf(s_gap, decision_margin);
       if (l > 0) {
         int nn = 0;
         int* next = cand + kMaxCap;
+        float* next_p = psc + kMaxCap;
         for (int k = 0; k < keep; k++) {
           const int m = (int)(0xFFFFFFFFu - (uint32_t)(keys[k] & 0xFFFFFFFFull));
+          const float r = key_to_float((uint32_t)(keys[k] >> 32));
           for (int ch = 2 * m; ch <= 2 * m + 1; ch++)
-            if (ch < g.lvl_n[l - 1] && (ch << (l - 1)) < i) next[nn++] = ch;
+            if (ch < g.lvl_n[l - 1] && (ch << (l - 1)) < i) {
+              next_p[nn] = r;
+              next[nn++] = ch;
+            }
         }
-        for (int k = 0; k < nn; k++) cand[k] = next[k];
+        for (int k = 0; k < nn; k++) {
+          cand[k] = next[k];
+          psc[k] = next_p[k];
+        }
         s_nc = nn;
       }
     }
@@ -279,13 +311,13 @@ __global__ void __launch_bounds__(kThreads) select_kernel(const T* __restrict__ 
 
 template <typename T>
 cudaError_t launch_t(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
-                     cudaStream_t st) {
+                     const SelOpts& o, cudaStream_t st) {
   const SelSmem L = sel_layout(g.G * min(g.b, g.Nq), g.d, (int)sizeof(T), g.cap);
   auto kern = select_kernel<T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nqb, g.B * g.Hkv);
-  kern<<<grid, kThreads, L.total, st>>>(reinterpret_cast<const T*>(Q), pyr, idx, gap, status, g);
+  kern<<<grid, kThreads, L.total, st>>>(reinterpret_cast<const T*>(Q), pyr, idx, gap, status, g, o);
   return cudaGetLastError();
 }
 
@@ -297,9 +329,9 @@ size_t select_smem_bytes(const Geo& g) {
 }
 
 cudaError_t launch_select(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
-                          cudaStream_t st) {
-  if (g.dtype == PYR_BF16) return launch_t<__nv_bfloat16>(g, Q, pyr, idx, gap, status, st);
-  return launch_t<float>(g, Q, pyr, idx, gap, status, st);
+                          const SelOpts& o, cudaStream_t st) {
+  if (g.dtype == PYR_BF16) return launch_t<__nv_bfloat16>(g, Q, pyr, idx, gap, status, o, st);
+  return launch_t<float>(g, Q, pyr, idx, gap, status, o, st);
 }
 
 }  // namespace pyr

@@ -16,7 +16,11 @@
 // that straddles the query block uses the exact mean of its part before the
 // block, precomputed for every level from the binary decomposition of
 // [m 2^l, i) into whole finer nodes. fp32 throughout.
+// The PHAROS variants and the trace follow select_opts.cuh: guidance adds the
+// parent's ranking score, the level-0 keep count comes from the budget and,
+// with the fallback, from the scores by rank after one more barrier.
 #include "pyr_common.cuh"
+#include "select_opts.cuh"
 
 namespace pyr {
 
@@ -45,7 +49,7 @@ template <typename T, int D, int TPC>
 __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __restrict__ Q,
                                                                  const __nv_bfloat16* __restrict__ pyr,
                                                                  int32_t* __restrict__ idx, float* __restrict__ gap_out,
-                                                                 Geo g) {
+                                                                 Geo g, SelOpts o) {
   constexpr int DPT = D / TPC;  // elements of d per thread
   __shared__ __align__(16) float q_s[kMaxG * D];
   __shared__ __align__(16) float part[kMaxLevels * D];
@@ -54,6 +58,9 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
   __shared__ int kept[kMaxCap];
   __shared__ float s_edge[2];
   __shared__ float s_gap;
+  __shared__ float s_conf;
+  __shared__ float sbr[kMaxCap];  // level-0 ranking scores by rank (fallback decision)
+  __shared__ float psc[kMaxCap];  // parent's ranking score per candidate slot (guidance)
 
   const int tid = threadIdx.x;
   const int unit = blockIdx.x;
@@ -81,8 +88,10 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
       part[l * D + e] = cnt > 0 ? acc / (float)(cnt * g.b) : 0.f;
     }
   }
-  if (tid == 0) s_gap = __int_as_float(0x7f800000);
+  if (tid == 0) s_gap = s_conf = __int_as_float(0x7f800000);
   __syncthreads();
+  const int base = sel_base_budget(o, g, unit);
+  const bool rcg = o.rcg_lambda != 0.f;
 
   const int my_c = tid / TPC, my_h = tid % TPC;  // scoring: candidate slot, part of d
   int nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
@@ -163,7 +172,8 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
         const int j0 = m << l;
         const int j1 = min(min((m + 1) << l, g.nb), i);
         const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
-        const float sc = (mx + __log2f(s)) * 0.6931471805599453f + __logf(nval);
+        float sc = (mx + __log2f(s)) * 0.6931471805599453f + __logf(nval);
+        if (rcg && !start) sc = fmaf(o.rcg_lambda, psc[my_c], sc);
         key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
       }
       keys[my_c] = key;
@@ -172,10 +182,12 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
     if (tid >= nc && tid < nc8) keys[tid] = 0ull;
     const int n_valid = __syncthreads_count(slot_m >= 0);
     // ---- keep the best; a kept node of rank r puts its children in slots 2r, 2r + 1
-    const int want = l > 0 ? g.cap / 2 : g.topk;
-    const int keep = min(want, n_valid);
+    const int keep_lo = min(l > 0 ? g.cap / 2 : base, n_valid);
+    int32_t* trow = o.trace ? sel_trace_row(o, g, unit, 0, l) : nullptr;
+    int my_rank = -1;
+    unsigned long long my_key = 0ull;
     if (slot_m >= 0) {
-      const unsigned long long my_key = keys[tid];
+      my_key = keys[tid];
       int rank = 0;
       const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
       for (int c = 0; c < nc8 / 2; c += 4) {
@@ -183,20 +195,40 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
         rank += (a0.x > my_key) + (a0.y > my_key) + (a1.x > my_key) + (a1.y > my_key) + (a2.x > my_key) +
                 (a2.y > my_key) + (a3.x > my_key) + (a3.y > my_key);
       }
-      if (rank < keep) {
+      my_rank = rank;
+    }
+    int keep = keep_lo;
+    float decision_margin = __int_as_float(0x7f800000);
+    if (l == 0 && o.fcf_extra > 0 && keep_lo < n_valid) {  // block-uniform
+      if (my_rank >= 0) sbr[my_rank] = key_score_d(my_key);
+      __syncthreads();
+      keep = sel_fcf_keep(o, g, base, n_valid, sbr, s_conf, &decision_margin);
+    }
+    if (my_rank >= 0) {
+      if (my_rank < keep) {
         if (l > 0) {
           const int c1 = 2 * slot_m + 1;
-          cand[2 * rank] = 2 * slot_m;
-          cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+          cand[2 * my_rank] = 2 * slot_m;
+          cand[2 * my_rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+          if (rcg) psc[2 * my_rank] = psc[2 * my_rank + 1] = key_score_d(my_key);
         } else {
-          kept[rank] = slot_m;
+          kept[my_rank] = slot_m;
         }
+        if (trow) trow[my_rank] = slot_m;
       }
-      if (rank == keep - 1) s_edge[0] = key_score_d(my_key);
-      if (rank == keep) s_edge[1] = key_score_d(my_key);
+      if (my_rank == keep - 1) s_edge[0] = key_score_d(my_key);
+      if (my_rank == keep) s_edge[1] = key_score_d(my_key);
     }
+    if (trow && tid >= keep && tid < o.tw) trow[tid] = -1;
     __syncthreads();
-    if (tid == 0 && keep < n_valid && keep > 0) s_gap = fminf(s_gap, s_edge[0] - s_edge[1]);
+    if (tid == 0) {
+      if (keep < n_valid && keep > 0) {
+        const float mg = s_edge[0] - s_edge[1];
+        s_gap = fminf(s_gap, mg);
+        if (l > 0) s_conf = fminf(s_conf, mg);
+      }
+      s_gap = fminf(s_gap, decision_margin);
+    }
     nc = 2 * keep;
     if (l == 0) {
       for (int k = tid; k < g.topk; k += kThreads) {
@@ -217,11 +249,11 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
 
 template <typename T, int D>
 cudaError_t launch_dec(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
-                       cudaStream_t st) {
+                       const SelOpts& o, cudaStream_t st) {
   if (g.cap <= 64)
-    select_decode_kernel<T, D, 2><<<g.B * g.Hkv, kThreads, 0, st>>>(static_cast<const T*>(Q), pyr, idx, gap, g);
+    select_decode_kernel<T, D, 2><<<g.B * g.Hkv, kThreads, 0, st>>>(static_cast<const T*>(Q), pyr, idx, gap, g, o);
   else
-    select_decode_kernel<T, D, 1><<<g.B * g.Hkv, kThreads, 0, st>>>(static_cast<const T*>(Q), pyr, idx, gap, g);
+    select_decode_kernel<T, D, 1><<<g.B * g.Hkv, kThreads, 0, st>>>(static_cast<const T*>(Q), pyr, idx, gap, g, o);
   return cudaGetLastError();
 }
 
@@ -232,13 +264,13 @@ bool select_decode_supported(const Geo& g) {
 }
 
 cudaError_t launch_select_decode(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
-                                 cudaStream_t st) {
+                                 const SelOpts& o, cudaStream_t st) {
   if (g.dtype == PYR_F32) {
-    if (g.d == 64) return launch_dec<float, 64>(g, Q, pyr, idx, gap, st);
-    return launch_dec<float, 128>(g, Q, pyr, idx, gap, st);
+    if (g.d == 64) return launch_dec<float, 64>(g, Q, pyr, idx, gap, o, st);
+    return launch_dec<float, 128>(g, Q, pyr, idx, gap, o, st);
   }
-  if (g.d == 64) return launch_dec<__nv_bfloat16, 64>(g, Q, pyr, idx, gap, st);
-  return launch_dec<__nv_bfloat16, 128>(g, Q, pyr, idx, gap, st);
+  if (g.d == 64) return launch_dec<__nv_bfloat16, 64>(g, Q, pyr, idx, gap, o, st);
+  return launch_dec<__nv_bfloat16, 128>(g, Q, pyr, idx, gap, o, st);
 }
 
 }  // namespace pyr

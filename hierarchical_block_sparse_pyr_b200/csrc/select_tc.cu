@@ -33,7 +33,12 @@
 //            (-1 for a child that does not exist or starts at or after block i).
 // q is exactly representable in bf16, so the only rounding beyond fp32
 // accumulation is the hi/lo split of the means.
+// The PHAROS variants (select_opts.cuh) change only the ranking score (RCG:
+// the parent's ranking score is added), the level-0 keep count (DBA budget,
+// FCF fallback: level 0 then publishes the scores by rank and takes one more
+// barrier to decide) and, with a trace, what is written per level.
 #include "pyr_common.cuh"
+#include "select_opts.cuh"
 #include "tc_util.cuh"
 
 namespace pyr {
@@ -63,7 +68,7 @@ struct SelCfg {
 };
 
 struct SelPlan {
-  int q, a, ppair, keys, cand, kept, misc, bars, total;
+  int q, a, ppair, keys, cand, kept, sbr, psc, misc, bars, total;
 };
 
 // R: query rows (N of the MMA); a_bytes: the A tiles; levels: s0 + 1.
@@ -76,7 +81,9 @@ __host__ __device__ inline SelPlan sel_plan(int R, int a_bytes, int levels, int 
   p.keys = o;  o += (kMaxCap + 8) * 8;
   p.cand = o;  o += kMaxCap * 4;
   p.kept = o;  o += kMaxCap * 4;
-  p.misc = o;  o += 64;                  // gap, tmem slot, abort flag, boundary scores
+  p.sbr = o;   o += kMaxCap * 4;         // level-0 ranking scores by rank (fallback decision)
+  p.psc = o;   o += kMaxCap * 4;         // parent's ranking score per candidate slot (guidance)
+  p.misc = o;  o += 64;                  // gap, tmem slot, abort flag, boundary scores, confidence
   p.bars = o;  o += 16;                  // q_full, mma_done
   p.total = o + 1024;                    // + alignment slack
   return p;
@@ -109,7 +116,7 @@ __device__ __forceinline__ int a_chunk_off(int c, int q) {
 template <int MC, int NT, bool STACK>
 __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     select_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __nv_bfloat16* __restrict__ pyr,
-                     int32_t* __restrict__ idx, float* __restrict__ gap_out, int* status, Geo g) {
+                     int32_t* __restrict__ idx, float* __restrict__ gap_out, int* status, Geo g, SelOpts o) {
   using C = SelCfg<MC, NT, STACK>;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -126,6 +133,9 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 8);
   float* s_edge = reinterpret_cast<float*>(smem + L.misc + 16);  // [0]: last kept, [1]: first dropped
+  float* s_conf = reinterpret_cast<float*>(smem + L.misc + 32);  // smallest margin above level 0
+  float* sbr = reinterpret_cast<float*>(smem + L.sbr);
+  float* psc = reinterpret_cast<float*>(smem + L.psc);
   uint64_t* bar_q = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* bar_mma = bar_q + 1;
 
@@ -151,7 +161,10 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     fence_mbar_init();
     *abort_flag = 0;
     *s_gap = __int_as_float(0x7f800000);
+    *s_conf = __int_as_float(0x7f800000);
   }
+  const int base = sel_base_budget(o, g, unit);  // level-0 budget before any fallback
+  const bool rcg = o.rcg_lambda != 0.f;
   // start level s0: every node that begins before block i, node m in slot m
   int nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
   {
@@ -233,9 +246,10 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
     const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
     const int n_valid = __syncthreads_count(slot_m >= 0);
-    const int want = l > 0 ? g.cap / 2 : g.topk;
-    const int keep = min(want, n_valid);
-    if (keep == n_valid) {
+    // keep count, except at level 0 with the fallback on, where it can grow after scoring
+    const int keep_lo = min(l > 0 ? g.cap / 2 : base, n_valid);
+    int32_t* trow = o.trace ? sel_trace_row(o, g, unit, qb, l) : nullptr;
+    if (keep_lo == n_valid && !rcg) {
       // every valid candidate survives this level whatever its score: no scoring. Keys that
       // rank the candidates by node index (a fixed score, index tie-break) hand the same set on
       for (int c = tid; c < nc; c += kThreads) {
@@ -351,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
           const int j0 = m << l;
           const int j1 = min(min((m + 1) << l, g.nb), i);
           const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
-          const float sc = (M + __log2f(S)) * 0.6931471805599453f + __logf(nval);
+          float sc = (M + __log2f(S)) * 0.6931471805599453f + __logf(nval);
+          if (rcg && !start) sc = fmaf(o.rcg_lambda, psc[c], sc);
           key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
         }
         keys[c] = key;
@@ -362,34 +377,29 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     const int nc8 = (nc + 7) & ~7;
     if (tid >= nc && tid < (kSplit ? 32 : nc8)) keys[tid] = 0ull;  // zero pad for the 8-wide reads
     __syncthreads();
-    // ---- keep the best: rank = number of strictly larger keys; a kept node of rank r puts its
-    // children (those that exist and start before block i; -1 otherwise) in slots 2r, 2r + 1
+    // ---- keep the best: rank = number of strictly larger keys (keys are distinct: they hold the
+    // node index); a kept node of rank r puts its children (those that exist and start before
+    // block i; -1 otherwise) in slots 2r, 2r + 1
+    int my_rank = -1, my_node = -1;
+    unsigned long long my_key = 0ull;
     if (kSplit) {
       // slot tid / 4: each of its four threads counts the larger keys among 8 of the 32
       const int sl = tid >> 2, part = tid & 3;
-      const unsigned long long my_key = keys[sl];
+      const unsigned long long k_sl = keys[sl];
       const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys) + part * 4;
       const ulonglong2 a0 = k2[0], a1 = k2[1], a2 = k2[2], a3 = k2[3];
-      int rank = split_m >= 0 ? (a0.x > my_key) + (a0.y > my_key) + (a1.x > my_key) + (a1.y > my_key) +
-                                    (a2.x > my_key) + (a2.y > my_key) + (a3.x > my_key) + (a3.y > my_key)
+      int rank = split_m >= 0 ? (a0.x > k_sl) + (a0.y > k_sl) + (a1.x > k_sl) + (a1.y > k_sl) +
+                                    (a2.x > k_sl) + (a2.y > k_sl) + (a3.x > k_sl) + (a3.y > k_sl)
                               : 0;
       rank += __shfl_xor_sync(0xffffffffu, rank, 1);
       rank += __shfl_xor_sync(0xffffffffu, rank, 2);
       if (split_m >= 0 && part == 0) {
-        if (rank < keep) {
-          if (l > 0) {
-            const int c1 = 2 * split_m + 1;
-            cand[2 * rank] = 2 * split_m;
-            cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
-          } else {
-            kept[rank] = split_m;
-          }
-        }
-        if (rank == keep - 1) s_edge[0] = key_score(my_key);
-        if (rank == keep) s_edge[1] = key_score(my_key);
+        my_rank = rank;
+        my_node = split_m;
+        my_key = k_sl;
       }
     } else if (slot_m >= 0) {
-      const unsigned long long my_key = keys[tid];
+      my_key = keys[tid];
       int rank = 0;
       const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys);
       for (int c = 0; c < nc8 / 2; c += 4) {
@@ -397,20 +407,41 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
         rank += (a0.x > my_key) + (a0.y > my_key) + (a1.x > my_key) + (a1.y > my_key) + (a2.x > my_key) +
                 (a2.y > my_key) + (a3.x > my_key) + (a3.y > my_key);
       }
-      if (rank < keep) {
-        if (l > 0) {
-          const int c1 = 2 * slot_m + 1;
-          cand[2 * rank] = 2 * slot_m;
-          cand[2 * rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
-        } else {
-          kept[rank] = slot_m;
-        }
-      }
-      if (rank == keep - 1) s_edge[0] = key_score(my_key);
-      if (rank == keep) s_edge[1] = key_score(my_key);
+      my_rank = rank;
+      my_node = slot_m;
     }
+    int keep = keep_lo;
+    float decision_margin = __int_as_float(0x7f800000);
+    if (l == 0 && o.fcf_extra > 0 && keep_lo < n_valid) {  // block-uniform
+      if (my_rank >= 0) sbr[my_rank] = key_score(my_key);
+      __syncthreads();
+      keep = sel_fcf_keep(o, g, base, n_valid, sbr, *s_conf, &decision_margin);
+    }
+    if (my_rank >= 0) {
+      if (my_rank < keep) {
+        if (l > 0) {
+          const int c1 = 2 * my_node + 1;
+          cand[2 * my_rank] = 2 * my_node;
+          cand[2 * my_rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+          if (rcg) psc[2 * my_rank] = psc[2 * my_rank + 1] = key_score(my_key);
+        } else {
+          kept[my_rank] = my_node;
+        }
+        if (trow) trow[my_rank] = my_node;
+      }
+      if (my_rank == keep - 1) s_edge[0] = key_score(my_key);
+      if (my_rank == keep) s_edge[1] = key_score(my_key);
+    }
+    if (trow && tid >= keep && tid < o.tw) trow[tid] = -1;
     __syncthreads();
-    if (tid == 0 && keep < n_valid && keep > 0) *s_gap = fminf(*s_gap, s_edge[0] - s_edge[1]);
+    if (tid == 0) {
+      if (keep < n_valid && keep > 0) {
+        const float mg = s_edge[0] - s_edge[1];
+        *s_gap = fminf(*s_gap, mg);
+        if (l > 0) *s_conf = fminf(*s_conf, mg);
+      }
+      *s_gap = fminf(*s_gap, decision_margin);
+    }
     nc = 2 * keep;
     if (l == 0) {
       // the kept blocks in ascending order, then -1
@@ -447,13 +478,13 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
 
 template <int MC, int NT, bool STACK>
 cudaError_t launch_mc(const Geo& g, const CUtensorMap& mq, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
-                      int* status, cudaStream_t st) {
+                      int* status, const SelOpts& o, cudaStream_t st) {
   const SelPlan L = sel_plan(g.G * g.b, NT * SelCfg<MC, NT, STACK>::kATile, g.s0 + 1, 128);
   auto kern = select_tc_kernel<MC, NT, STACK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
   if (e != cudaSuccess) return e;
   dim3 grid(g.nqb, g.B * g.Hkv);
-  kern<<<grid, kThreads, L.total, st>>>(mq, pyr, idx, gap, status, g);
+  kern<<<grid, kThreads, L.total, st>>>(mq, pyr, idx, gap, status, g, o);
   return cudaGetLastError();
 }
 
@@ -474,12 +505,12 @@ bool select_tc_supported(const Geo& g) {
 }
 
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap,
-                             int* status, cudaStream_t st) {
+                             int* status, const SelOpts& o, cudaStream_t st) {
   CUtensorMap mq;
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq)) return cudaErrorInvalidValue;
-  if (g.cap <= 32) return launch_mc<64, 1, true>(g, mq, pyr, idx, gap, status, st);
-  if (g.cap <= 64) return launch_mc<128, 1, true>(g, mq, pyr, idx, gap, status, st);
-  return launch_mc<128, 1, false>(g, mq, pyr, idx, gap, status, st);
+  if (g.cap <= 32) return launch_mc<64, 1, true>(g, mq, pyr, idx, gap, status, o, st);
+  if (g.cap <= 64) return launch_mc<128, 1, true>(g, mq, pyr, idx, gap, status, o, st);
+  return launch_mc<128, 1, false>(g, mq, pyr, idx, gap, status, o, st);
 }
 
 }  // namespace pyr

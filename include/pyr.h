@@ -161,6 +161,61 @@ PYR_API int pyr_select(const pyr_shape* s, const void* Q, const void* pyr, int32
                        int* dev_status, void* stream);
 
 /*
+ * Options of pyr_select_ex: the selection variants the PHAROS page (Zensar,
+ * "Four mechanisms powering PHAROS") proposes as augmentations of
+ * hierarchical selection, and a trace of the walk. All off in a zeroed struct,
+ * which gives pyr_select's plain walk.
+ *   budget     depth-sounding budget allocation (DBA: token budgets differ
+ *              across heads): device [B][Hkv] int32, the number of level-0
+ *              blocks each (batch, kv head) keeps, clamped to [0, topk]; NULL:
+ *              topk - fcf_extra for every unit. The page derives the budgets
+ *              from attention-head entropy without a formula, so they are an
+ *              input here.
+ *   fcf_tau,   fog-gate confidence fallback (FCF: the budget grows when
+ *   fcf_extra  confidence is low): the confidence is the smallest margin
+ *              between the last kept and the first dropped candidate over the
+ *              levels above 0 and at the level-0 budget boundary; when it is
+ *              below fcf_tau, level 0 keeps min(budget + fcf_extra, topk)
+ *              blocks. fcf_extra = 0: off. fcf_tau must not be NaN.
+ *   rcg_lambda range-light cross-level guidance (RCG: coarse levels guide the
+ *              finer ones): candidates rank by R = S + rcg_lambda * R(parent),
+ *              R = S at the start level; margins and gap are taken on R.
+ *              0: off. Must be finite.
+ *   trace      device [B][Hkv][nqb][levels][width] int32 or NULL (written):
+ *              for level l, row levels - 1 - l lists the nodes kept at that
+ *              level (any order), then -1; levels = pyr_select_trace_levels,
+ *              width = pyr_select_trace_width. It records the walk so that it
+ *              can be checked (or explained) level by level.
+ * With a variant on, s->topk is the width of an idx row (the most blocks any
+ * row may keep); rows keep their kept blocks ascending, then -1.
+ */
+typedef struct pyr_select_opts {
+  const int32_t* budget;
+  float fcf_tau;
+  int fcf_extra;
+  float rcg_lambda;
+  int32_t* trace;
+} pyr_select_opts;
+
+/* Levels of a selection trace: the walk's start level (the finest with at
+ * most cap nodes) down to 0; 0 on a bad shape. */
+PYR_API int pyr_select_trace_levels(const pyr_shape* s);
+
+/* Entries per trace level: max(cap / 2, topk); 0 on a bad shape. */
+PYR_API int pyr_select_trace_width(const pyr_shape* s);
+
+/*
+ * pyr_select_ex - pyr_select with the options above (opts may be NULL). The
+ * gap output becomes the smallest margin of any decision the walk took: at
+ * every level the margin at the boundary it used, and, when the fallback
+ * could change the result, the distance between the confidence and fcf_tau.
+ * PYR_EINVAL for a negative fcf_extra, a NaN fcf_tau, a NaN or infinite
+ * rcg_lambda, or a budget or trace pointer that is not 4-byte aligned.
+ */
+PYR_API int pyr_select_ex(const pyr_shape* s, const void* Q, const void* pyr, const pyr_select_opts* opts,
+                          int32_t* idx, float* gap, int* dev_status, void* stream);
+
+/*
  * bsa_forward - causal block-sparse attention (PHBA 3.1, 3.3 and A.1.3:
  * routed blocks plus the current block, one online-softmax merge, output and
  * log-sum-exp; the N x N score matrix is never formed).
