@@ -32,21 +32,34 @@ def to_dev(*ts):
     return [t.cuda() for t in ts]
 
 
-def run_gpu(w, Q, K, V, idx=None, dense=False):
-    """Run the CUDA path on CPU inputs. Returns a dict of CPU tensors."""
+def run_gpu(w, Q, K, V, idx=None, dense=False, opts=None, with_trace=False):
+    """Run the CUDA path on CPU inputs. Returns a dict of CPU tensors.
+
+    opts: an oracle.SelectOpts-like object (budget, fcf_tau, fcf_extra, rcg_lambda) whose values are
+    passed to pyr_select_ex; with_trace adds the selection trace ("trace", [U, nqb, levels, width])."""
     s = P.shape_of(w)
     Qd, Kd, Vd = to_dev(Q, K, V)
     buf = P.Buffers(s)
     P.pyr_build(s, Kd, buf.pyr, buf.status)
-    P.pyr_select(s, Qd, buf.pyr, buf.idx, buf.gap, buf.status)
+    trace = P.new_trace(s) if with_trace else None
+    if opts is None and trace is None:
+        P.pyr_select(s, Qd, buf.pyr, buf.idx, buf.gap, buf.status)
+    else:
+        kw = {}
+        if opts is not None:
+            budget = None if opts.budget is None else torch.as_tensor(np.asarray(opts.budget, dtype=np.int32)).cuda()
+            kw = dict(budget=budget, fcf_tau=opts.fcf_tau, fcf_extra=opts.fcf_extra, rcg_lambda=opts.rcg_lambda)
+        P.pyr_select_ex(s, Qd, buf.pyr, buf.idx, buf.gap, trace=trace, status=buf.status, **kw)
     if dense:
         P.dense_forward(s, Qd, Kd, Vd, buf.O, buf.lse, buf.status)
     else:
         use = buf.idx if idx is None else torch.as_tensor(np.ascontiguousarray(idx), dtype=torch.int32).cuda()
         P.bsa_forward(s, Qd, Kd, Vd, use, buf.O, buf.lse, buf.status)
     torch.cuda.synchronize()
-    out = dict(pyr=P.pyramid_means(buf.pyr).cpu(), idx=buf.idx.cpu(), gap=buf.gap.cpu(), O=buf.O.float().cpu(), lse=buf.lse.cpu(),
-               status=int(buf.status.item()))
+    out = dict(pyr=P.pyramid_means(buf.pyr).cpu(), idx=buf.idx.cpu(), gap=buf.gap.cpu(), O=buf.O.float().cpu(),
+               lse=buf.lse.cpu(), status=int(buf.status.item()))
+    if trace is not None:
+        out["trace"] = trace.reshape(w.B * w.Hkv, trace.shape[2], trace.shape[3], trace.shape[4]).cpu()
     del buf, Qd, Kd, Vd
     return out
 
@@ -236,6 +249,123 @@ def walk_reaches(w, Q, pyr_unit: np.ndarray, unit: int, qb: int, target, eps: fl
 
 class _SearchBound(Exception):
     pass
+
+
+# ---- selection trace: check the GPU's own walk level by level ----------------------------------
+
+def validate_trace(w, Q, pyr_unit: np.ndarray, unit: int, qb: int, trace_rows, idx_row, eps: float,
+                   opts=None, score_cache=None):
+    """Is the GPU's walk of (unit, query block qb), as its trace records it, a valid walk?
+
+    trace_rows [s0 + 1][width]: row s0 - l lists the nodes the GPU kept at level l (any order, -1
+    padded). Following the GPU's own chain of kept sets, with the oracle's scores (oracle.node_score):
+      - level s0's candidates are the nodes that begin before block i; level l - 1's are the children
+        of the nodes kept at level l that exist and begin before block i;
+      - each level keeps the right number of distinct candidates: min(cap/2, #candidates) above level
+        0; at level 0 the budget (opts: DBA budget, FCF expansion), where a confidence within eps of
+        fcf_tau allows either count;
+      - every kept candidate ranks within eps of every dropped one: min R over kept >= max R over
+        dropped - eps (R = S + rcg_lambda * R(parent), R = S without RCG);
+      - idx lists the level-0 kept set, ascending, then -1.
+    With eps = 0 and no exact ties only the oracle's own walk passes. Returns (ok, message).
+    """
+    first = w.q_offset // w.b
+    i = first + qb
+    lv = [n for _, n in oracle.level_offsets(w)]
+    s0 = 0
+    while lv[s0] > w.cap:
+        s0 += 1
+    trace_rows = np.asarray(trace_rows).reshape(s0 + 1, -1)
+    lam = opts.rcg_lambda if opts is not None else 0.0
+    extra = opts.fcf_extra if opts is not None else 0
+    tau = opts.fcf_tau if opts is not None else 0.0
+    if opts is not None and opts.budget is not None:
+        base = int(opts.budget[unit])
+    else:
+        base = w.topk - extra
+    base = min(max(base, 0), w.topk)
+    cache = {} if score_cache is None else score_cache
+
+    def S(l, m):
+        if (l, m) not in cache:
+            cache[(l, m)] = oracle.node_score(w, Q, pyr_unit, unit, qb, l, m)[0]
+        return cache[(l, m)]
+
+    cands = {m: 0.0 for m in range(lv[s0]) if (m << s0) < i}  # node -> parent's R
+    conf = math.inf
+    for k, l in enumerate(range(s0, -1, -1)):
+        kept = [int(x) for x in trace_rows[k] if x >= 0]
+        if len(set(kept)) != len(kept):
+            return False, f"level {l}: a node is kept twice: {kept}"
+        if not set(kept) <= set(cands):
+            return False, f"level {l}: kept {sorted(set(kept) - set(cands))} are not candidates"
+        R = {m: S(l, m) + lam * p for m, p in cands.items()}
+        order = sorted(R, key=lambda m: (-R[m], m))
+        if l > 0:
+            allowed = {min(w.cap // 2, len(R))}
+        else:
+            kb = min(base, len(R))
+            allowed = {kb}
+            if extra > 0:
+                c0 = conf
+                if 0 < kb < len(R):
+                    c0 = min(c0, R[order[kb - 1]] - R[order[kb]])
+                wide = min(base + extra, w.topk, len(R))
+                if c0 < tau + eps:
+                    allowed.add(wide)
+                if c0 < tau - eps:
+                    allowed.discard(kb)
+        if len(kept) not in allowed:
+            return False, f"level {l}: kept {len(kept)} nodes, allowed {sorted(allowed)}"
+        dropped = [m for m in R if m not in set(kept)]
+        if kept and dropped:
+            margin = min(R[m] for m in kept) - max(R[m] for m in dropped)
+            if margin < -eps:
+                return False, (f"level {l}: kept node ranks {-margin:.3e} below a dropped one "
+                               f"(kept {sorted(kept)}, best dropped {max(dropped, key=lambda m: R[m])})")
+            if l > 0:
+                conf = min(conf, margin)
+        if l == 0:
+            want = sorted(kept) + [-1] * (w.topk - len(kept))
+            got = [int(x) for x in np.asarray(idx_row).reshape(-1)]
+            if got != want:
+                return False, f"idx {got} is not the level-0 kept set {want}"
+            return True, ""
+        cands = {ch: R[m] for m in kept for ch in (2 * m, 2 * m + 1) if ch < lv[l - 1] and (ch << (l - 1)) < i}
+    return False, "unreachable"
+
+
+def check_traces(w, Q, pyr_units: np.ndarray, units, items, idx_gpu, trace_gpu, idx_ora, gap_ora, trace_ora,
+                 opts=None, eps: float = TIE_EPS):
+    """Selection acceptance with the GPU's trace: rows with oracle gap >= GAP_EXEMPT must match the
+    oracle bit for bit, trace included (as sets per level); every other row whose idx or trace
+    differs from the oracle's must be a valid walk (validate_trace). Nothing is left undecided.
+    Returns dict(checked, exempt, differing, validated)."""
+    n = len(items)
+    idx_gpu = np.asarray(idx_gpu).reshape(n, -1)
+    idx_ora = np.asarray(idx_ora).reshape(n, -1)
+    trace_gpu = np.asarray(trace_gpu).reshape(n, trace_ora.shape[1], -1)
+    gap_ora = np.asarray(gap_ora).reshape(-1)
+    checked = exempt = differing = validated = 0
+    for k, (slot, qb) in enumerate(items):
+        same_idx = (idx_gpu[k] == idx_ora[k]).all()
+        same_trace = all(set(trace_gpu[k, l][trace_gpu[k, l] >= 0].tolist()) ==
+                         set(trace_ora[k, l][trace_ora[k, l] >= 0].tolist()) for l in range(trace_ora.shape[1]))
+        if gap_ora[k] >= GAP_EXEMPT:
+            checked += 1
+            assert same_idx, (f"unit {units[slot]} query block {qb}: gpu {idx_gpu[k]} oracle {idx_ora[k]} "
+                              f"gap {gap_ora[k]:.3e}")
+            assert same_trace, f"unit {units[slot]} query block {qb}: trace differs with gap {gap_ora[k]:.3e}"
+            continue
+        exempt += 1
+        if same_idx and same_trace:
+            continue
+        differing += int(not same_idx)
+        ok, msg = validate_trace(w, Q, pyr_units[slot], units[slot], qb, trace_gpu[k], idx_gpu[k], eps, opts)
+        assert ok, (f"unit {units[slot]} query block {qb} (oracle gap {gap_ora[k]:.2e}, gpu idx {idx_gpu[k]}, "
+                    f"oracle idx {idx_ora[k]}): {msg}")
+        validated += 1
+    return dict(checked=checked, exempt=exempt, differing=differing, validated=validated)
 
 
 def check_exempt_rows(w, Q, pyr_units: np.ndarray, units, items, idx_gpu: np.ndarray, idx_ora: np.ndarray,

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from _parity import (check_exempt_rows, check_out, check_pyramid, check_select, check_valid_idx, fmt, run_gpu)
+from _parity import check_out, check_pyramid, check_traces, check_valid_idx, fmt, run_gpu
 from synth import BF16, F32
 
 pytestmark = pytest.mark.gpu
@@ -71,24 +71,24 @@ def _rows_sample(w, n=600, seed=0):
 def test_parity_small(w):
     Q, K, V, _ = synth.generate(w)
     units = list(range(w.B * w.Hkv))
-    g = run_gpu(w, Q, K, V)
+    g = run_gpu(w, Q, K, V, with_trace=True)
     assert g["status"] == 0
 
     pyr_o = oracle.pyramid(w, K, units)
     check_pyramid(g["pyr"].double().numpy().reshape(pyr_o.shape), pyr_o)
 
-    idx_o, gap_o, _ = oracle.select_all(w, Q, K)
-    idx_g = g["idx"].numpy().reshape(idx_o.shape)
-    checked, exempt, exempt_diff = check_select(idx_g, idx_o, gap_o)
-    items = [(u, q) for u in units for q in range(idx_o.shape[1])]
-    _, reached, undecided = check_exempt_rows(w, Q, pyr_o, units, items, idx_g, idx_o, gap_o)
+    nqb = oracle.num_qblocks(w)
+    items = [(u, q) for u in units for q in range(nqb)]
+    idx_o, gap_o, _, trace_o = oracle.select(w, Q, pyr_o, units, items, with_trace=True)
+    counts = check_traces(w, Q, pyr_o, units, items, g["idx"].numpy(), g["trace"].numpy(), idx_o, gap_o, trace_o)
     check_valid_idx(w, g["idx"].numpy())
-    gap_g = g["gap"].double().numpy().reshape(gap_o.shape)
+    gap_g = g["gap"].double().numpy().reshape(-1)
     fin = np.isfinite(gap_o)
     assert (np.isfinite(gap_g) == fin).all()
     np.testing.assert_allclose(gap_g[fin], gap_o[fin], atol=1e-3, rtol=1e-3)
-    print(f"\n{fmt(w)} select: {checked} rows bit-exact, {exempt} exempt ({exempt_diff} differ: {reached} reachable "
-          f"with near-ties either way, {undecided} undecided)")
+    print(f"\n{fmt(w)} select: {counts['checked']} rows bit-exact with their trace, {counts['exempt']} exempt "
+          f"({counts['differing']} differ, {counts['validated']} validated level by level, 0 undecided)")
+    idx_o = idx_o.reshape(len(units), nqb, w.topk)
 
     rows = _rows_all(w) if w.B * w.Hq * w.Nq <= 16384 else _rows_sample(w)
     # attention given the oracle's idx
