@@ -109,7 +109,9 @@ def work_counts(w):
     else:
         pyr_bytes = U * (w.N * w.d * elt + P * w.d * 4)
     q_bytes = w.B * w.Hq * w.Nq * w.d * elt
-    sel_bytes = q_bytes + U * sel_nodes * w.d * 4 + U * nqb * w.topk * 4
+    # Q once + the pyramid once (each node a bf16 (hi, lo) pair: 4 bytes per element) + idx; a walk that
+    # touches fewer nodes than the pyramid holds (decode: one query block per unit) reads only those
+    sel_bytes = q_bytes + U * min(P, sel_nodes) * w.d * 4 + U * nqb * w.topk * 4
     # attention: Q + O once; K, V of the selected + diagonal blocks once per query block and kv head
     kv_blocks = 0
     for qb in range(nqb):
@@ -168,7 +170,7 @@ def peak_source(bound, peaks):
         return "derived: 148 SMs x 128 FP32 lanes x 2 FLOP x median SM clock under load"
     tag = "measured" if peaks["source"] == "measured" else "fallback"
     if bound == "tensor":
-        return f"{tag}: dense bf16 cuBLAS, sustained (kernel timed inside a long step loop)"
+        return f"{tag}: dense bf16 cuBLAS, burst (the timed region lasts well under a second)"
     return f"{tag}: HBM copy bandwidth"
 
 
@@ -365,6 +367,148 @@ def count_launches(step):
         return None, [f"profiler unavailable: {ex}"]
 
 
+def make_step(P, s, w, Q, K, V, buf, stream):
+    """One step of the path on resident inputs; ev (4 events) brackets the three calls."""
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        if w.decode:
+            # a decode step refreshes only the nodes over the appended position
+            P.pyr_update(s, K, buf.pyr, w.N - 1, buf.status, stream)
+        else:
+            P.pyr_build(s, K, buf.pyr, buf.status, stream)
+        if ev:
+            ev[1].record(stream)
+        P.pyr_select(s, Q, buf.pyr, buf.idx, buf.gap, buf.status, stream)
+        if ev:
+            ev[2].record(stream)
+        P.bsa_forward(s, Q, K, V, buf.idx, buf.O, buf.lse, buf.status, stream)
+        if ev:
+            ev[3].record(stream)
+    return step
+
+
+def time_steps(step, steps, world, dev, stream, clock_index):
+    """K event-timed steps between barriers + synchronize, clocks sampled meanwhile.
+    Returns (ms per step of this rank, max over ranks, per-kernel ms lists, clocks)."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(clock_index)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for k in range(steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    per = {"pyramid": [], "select": [], "attention": []}
+    for ev in evs:
+        per["pyramid"].append(ev[0].elapsed_time(ev[1]))
+        per["select"].append(ev[1].elapsed_time(ev[2]))
+        per["attention"].append(ev[2].elapsed_time(ev[3]))
+    return ms_total / steps, max_over_ranks(ms_total, world, dev) / steps, per, clk
+
+
+def kernel_report(w, per, ms_step, peaks, sm_clock):
+    """Per-kernel roofline figures from the kernels' average event-timed durations.
+
+    Tensor-core kernels are rated against the burst dense bf16 peak (the timed regions last well
+    under a second); frac_sustained, against the sustained peak, is context. Selection is also
+    rated against HBM with its bytes counted once (Q, the pyramid, idx), and pyramid + selection
+    together against HBM."""
+    wc = work_counts(w)
+    avg = {k: sum(v) / len(v) for k, v in per.items()}
+    alu_peak = 148 * 128 * 2 * sm_clock * 1e6 / 1e12
+    tc_burst, tc_sus = peaks["bf16_tflops"], peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    sel_tc, att_tc = tc_select(w), tc_attention(w)
+    kernels = {
+        "pyramid": dict(ms=avg["pyramid"], bound="hbm", kernel="pyr_update" if w.decode else "pyr_build",
+                        achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9, peak=peaks["hbm_gbs"], unit="GB/s",
+                        algorithmic=wc["pyr_bytes"], traffic=measured_traffic("pyramid", w)),
+        "select": dict(ms=avg["select"], bound="tensor" if sel_tc else "alu",
+                       achieved=wc["sel_flops"] / (avg["select"] * 1e-3) / 1e12,
+                       peak=tc_burst if sel_tc else alu_peak, unit="TFLOP/s", algorithmic=wc["sel_flops"],
+                       hbm_bytes=wc["sel_bytes"], hbm_gbs=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9,
+                       hbm_frac=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                       traffic=measured_traffic("select", w)),
+    }
+    if w.decode:
+        kernels["attention"] = dict(ms=avg["attention"], bound="hbm",
+                                    achieved=wc["att_bytes"] / (avg["attention"] * 1e-3) / 1e9,
+                                    peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["att_bytes"],
+                                    traffic=measured_traffic("attention", w))
+    else:
+        kernels["attention"] = dict(ms=avg["attention"], bound="tensor" if att_tc else "alu",
+                                    achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
+                                    peak=tc_burst if att_tc else alu_peak, unit="TFLOP/s",
+                                    algorithmic=wc["att_flops"], traffic=measured_traffic("attention", w))
+    for name, k in kernels.items():
+        k["frac"] = k["achieved"] / k["peak"]
+        k["share"] = k["ms"] / ms_step
+        if k["bound"] == "tensor":
+            k["frac_sustained"] = k["achieved"] / tc_sus
+    both_ms = avg["pyramid"] + avg["select"]
+    pyr_sel = {"bytes": wc["pyr_bytes"] + wc["sel_bytes"], "ms": both_ms,
+               "achieved_gbs": (wc["pyr_bytes"] + wc["sel_bytes"]) / (both_ms * 1e-3) / 1e9}
+    pyr_sel["hbm_frac"] = pyr_sel["achieved_gbs"] / peaks["hbm_gbs"]
+    return wc, kernels, pyr_sel
+
+
+def rounded(d):
+    return {k: (round(v, 5) if isinstance(v, float) else v) for k, v in d.items()}
+
+
+def roofline_of(kernels, peaks):
+    dom_name = max(kernels, key=lambda k: kernels[k]["ms"])
+    dom = kernels[dom_name]
+    return {"kernel": dom_name, "bound": dom["bound"], "achieved": round(dom["achieved"], 3),
+            "peak": round(dom["peak"], 3), "unit": dom["unit"], "frac": round(dom["frac"], 4),
+            "traffic": dom["traffic"], "peak_source": peak_source(dom["bound"], peaks)}
+
+
+def sub_workload(args, name, dev, stream, local_rank, peaks):
+    """One more workload of the metric's range, timed on the device like the headline one (1 GPU)."""
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    w = synth.BY_NAME[name]
+    t_gen = time.perf_counter()
+    Qh, Kh, Vh, _ = synth.generate(w)
+    t_gen = time.perf_counter() - t_gen
+    s = P.shape_of(w)
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    buf = P.Buffers(s, dev)
+    if w.decode:
+        P.pyr_build(s, K, buf.pyr, buf.status, stream)
+    step = make_step(P, s, w, Q, K, V, buf, stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"{name}: device status {buf.status.item()}")
+    steps = max(3, min(args.steps, 10 if not w.decode else 50))
+    ms_rank, ms_step, per, clk = time_steps(step, steps, 1, dev, stream, local_rank)
+    sm_clock = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    wc, kernels, pyr_sel = kernel_report(w, per, ms_step, peaks, sm_clock)
+    del Q, K, V, buf
+    torch.cuda.empty_cache()
+    out = {"workload": name, "tokens_per_step": wc["tokens"], "steps": steps, "ms_per_step": round(ms_step, 4),
+           "value": round(wc["tokens"] / (ms_step * 1e-3), 1), "unit": "tokens/s",
+           "roofline": roofline_of(kernels, peaks),
+           "kernels": {k: rounded(v) for k, v in kernels.items()}, "pyramid_select_hbm": rounded(pyr_sel),
+           "clocks": clk, "input_generation_s": round(t_gen, 1)}
+    if not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, budget_s=5.0, QKV=(Qh, Kh, Vh))
+    del Qh, Kh, Vh
+    return out
+
+
 def run_ours(args, w, rank, world, local_rank):
     import hierarchical_block_sparse_pyr_b200 as P
 
@@ -381,22 +525,7 @@ def run_ours(args, w, rank, world, local_rank):
     # appended position (the pyramid of the prefilled context is built once, untimed)
     if w.decode:
         P.pyr_build(s, K, buf.pyr, buf.status, stream)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        if w.decode:
-            P.pyr_update(s, K, buf.pyr, w.N - 1, buf.status, stream)
-        else:
-            P.pyr_build(s, K, buf.pyr, buf.status, stream)
-        if ev:
-            ev[1].record(stream)
-        P.pyr_select(s, Q, buf.pyr, buf.idx, buf.gap, buf.status, stream)
-        if ev:
-            ev[2].record(stream)
-        P.bsa_forward(s, Q, K, V, buf.idx, buf.O, buf.lse, buf.status, stream)
-        if ev:
-            ev[3].record(stream)
+    step = make_step(P, s, w, Q, K, V, buf, stream)
 
     for _ in range(args.warmup):
         step()
@@ -406,29 +535,7 @@ def run_ours(args, w, rank, world, local_rank):
     launches_per_step, kernel_names = count_launches(step)
 
     # timed region: K steps, per-kernel events on the launching stream
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local_rank)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    t0.record(stream)
-    for k in range(args.steps):
-        step(evs[k])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    clk = clocks.stop()
-    ms_total = t0.elapsed_time(t1)
-    per = {"pyramid": [], "select": [], "attention": []}
-    for ev in evs:
-        per["pyramid"].append(ev[0].elapsed_time(ev[1]))
-        per["select"].append(ev[1].elapsed_time(ev[2]))
-        per["attention"].append(ev[2].elapsed_time(ev[3]))
-    ms_max = max_over_ranks(ms_total, world, dev)
+    _, ms_step, per, clk = time_steps(step, args.steps, world, dev, stream, local_rank)
 
     # end to end through the binding: pinned host inputs -> device -> path -> O back to pinned host.
     # Prefill: a step's inputs are Q, K and V. Decode: they are the new token's q, k and v; k and v
@@ -487,62 +594,55 @@ def run_ours(args, w, rank, world, local_rank):
     backward = (time_backward(P, s, w, Q, K, V, buf, stream, args.steps, args.warmup)
                 if args.backward and not w.decode else None)
 
-    wc = work_counts(w)
     peaks = load_peaks()
-    ms_step = ms_max / args.steps
-    value = job_throughput(wc["tokens"], world, ms_step)
-    avg = {k: sum(v) / len(v) for k, v in per.items()}
     sm_clock = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    kernels = {
-        "pyramid": dict(ms=avg["pyramid"], bound="hbm", kernel="pyr_update" if w.decode else "pyr_build", achieved=wc["pyr_bytes"] / (avg["pyramid"] * 1e-3) / 1e9,
-                        peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["pyr_bytes"],
-                        traffic=measured_traffic("pyramid", w)),
-        "select": dict(ms=avg["select"], bound="tensor" if tc_select(w) else "alu",
-                       achieved=wc["sel_flops"] / (avg["select"] * 1e-3) / 1e12,
-                       peak=(peaks["bf16_tflops_sustained"] if tc_select(w) else
-                             148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s", algorithmic=wc["sel_flops"],
-                       hbm_gbs=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9,
-                       hbm_frac=wc["sel_bytes"] / (avg["select"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                       traffic=measured_traffic("select", w)),
-        "attention": (dict(ms=avg["attention"], bound="hbm", achieved=wc["att_bytes"] / (avg["attention"] * 1e-3) / 1e9,
-                           peak=peaks["hbm_gbs"], unit="GB/s", algorithmic=wc["att_bytes"],
-                           traffic=measured_traffic("attention", w)) if w.decode else
-                      dict(ms=avg["attention"], bound="tensor" if tc_attention(w) else "alu",
-                           achieved=wc["att_flops"] / (avg["attention"] * 1e-3) / 1e12,
-                           peak=(peaks["bf16_tflops_sustained"] if tc_attention(w) else
-                                 148 * 128 * 2 * sm_clock * 1e6 / 1e12), unit="TFLOP/s",
-                           algorithmic=wc["att_flops"], traffic=measured_traffic("attention", w))),
-    }
-    for k in kernels.values():
-        k["frac"] = k["achieved"] / k["peak"]
-        k["share"] = k["ms"] / ms_step
-    dom_name = max(kernels, key=lambda k: kernels[k]["ms"])
-    dom = kernels[dom_name]
-    roofline = {"kernel": dom_name, "bound": dom["bound"], "achieved": round(dom["achieved"], 3),
-                "peak": round(dom["peak"], 3), "unit": dom["unit"], "frac": round(dom["frac"], 4),
-                "traffic": dom["traffic"], "peak_source": peak_source(dom["bound"], peaks)}
+    wc, kernels, pyr_sel = kernel_report(w, per, ms_step, peaks, sm_clock)
+    value = job_throughput(wc["tokens"], world, ms_step)
+    l2_mib = (Qh.numel() + Kh.numel() + Vh.numel()) * Qh.element_size() >> 20
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == synth.BF16 else "f32", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d, "b": w.b,
-                   "topk": w.topk, "cap": w.cap, "seed": w.seed, "global_batch": w.B * world, "seq_len": w.N,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (Q+K+V %d MiB > 126 MB)" % (
-                       (Qh.numel() + Kh.numel() + Vh.numel()) * Qh.element_size() >> 20)},
+        "config": config_of(w, world, l2_mib),
         "e2e": {"value": round(job_throughput(wc["tokens"], world, e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "call": e2e_call},
         "gpu_launches": None if launches_per_step is None else launches_per_step * args.steps,
-        "roofline": roofline,
-        "kernels": {k: {kk: (round(vv, 5) if isinstance(vv, float) else vv) for kk, vv in v.items()}
-                    for k, v in kernels.items()},
+        "roofline": roofline_of(kernels, peaks),
+        "kernels": {k: rounded(v) for k, v in kernels.items()},
+        "pyramid_select_hbm": rounded(pyr_sel),
         "dense": dict(dense, speedup_of_sparse_step=round(dense["ms"] / ms_step, 3)),
         **({"backward": backward} if backward else {}),
         "kernel_names": kernel_names,
         "clocks": clk,
         "peaks_source": peaks["source"],
     }
+    del Q, K, V, buf, O_host
+    if w.decode:
+        del Kn_h, Vn_h
+    else:
+        del workspace
+    torch.cuda.empty_cache()
+    if world == 1 and rank == 0 and args.sub_workloads:
+        # the rest of the metric's 32K-1M range, each timed like the headline workload
+        out["workloads"] = {}
+        for name in args.sub_workloads:
+            if name != w.name:
+                out["workloads"][name] = sub_workload(args, name, dev, stream, local_rank, peaks)
+    if world == 1 and rank == 0 and args.with_break_even and not w.decode:
+        out["break_even"] = break_even(args, w)
     return out
+
+
+def config_of(w, world, l2_mib=None):
+    """The workload's config dict (the same for both arms)."""
+    c = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d, "b": w.b,
+         "topk": w.topk, "cap": w.cap, "seed": w.seed, "global_batch": w.B * world, "seq_len": w.N,
+         "parallelism": f"replicas{world}" if world > 1 else "single"}
+    if l2_mib is None:
+        elt = 2 if w.dtype == synth.BF16 else 4
+        l2_mib = (w.B * w.Hq * w.Nq + 2 * w.B * w.Hkv * w.N) * w.d * elt >> 20
+    c["l2"] = "inputs larger than L2 (Q+K+V %d MiB > 126 MB)" % l2_mib
+    return c
 
 
 # -------------------------------------------------------- oracle baseline --
@@ -590,10 +690,10 @@ def oracle_sample(w, n_qb, seed=0, Q=None, K=None, V=None, n_units=1):
     return t3 - t0, est, desc
 
 
-def cpu_baseline(w, budget_s=15.0):
+def cpu_baseline(w, budget_s=15.0, QKV=None):
     """The oracle on a sample of about budget_s * 0.4 .. budget_s seconds: more query blocks of one unit
-    first, then more units, up to the whole job."""
-    Q, K, V, _ = synth.generate(w)
+    first, then more units, up to the whole job. QKV: the workload's host tensors, if at hand."""
+    Q, K, V = QKV if QKV is not None else synth.generate(w)[:3]
     nqb = oracle_nqb(w)
     U = w.B * w.Hkv
     n, nu = 4, 1
@@ -607,7 +707,7 @@ def cpu_baseline(w, budget_s=15.0):
         took, est, desc = oracle_sample(w, n, Q=Q, K=K, V=V, n_units=nu)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     return {"value": round(w.B * w.Nq / est, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": desc, "sample_seconds": round(took, 2)}
+            "sample": desc, "sample_seconds": round(took, 2), "extrapolated": "extrapolated" in desc}
 
 
 def oracle_nqb(w):
@@ -617,6 +717,9 @@ def oracle_nqb(w):
 
 
 def run_reference(args, w):
+    """The oracle, as it stands, on the host cores: each step times a bounded sample of the workload
+    (pyramids of one unit and a set of its query blocks). ms_per_step is the time those samples
+    actually took; the whole-job time they extrapolate to is given beside it."""
     Q, K, V, _ = synth.generate(w)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
     n_qb = 8
@@ -631,12 +734,14 @@ def run_reference(args, w):
         ests.append(est)
         tooks.append(took)
     est = statistics.mean(ests)
+    ms_timed = statistics.mean(tooks) * 1e3
     value = w.B * w.Nq / est
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est * 1e3, 1), "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_timed, 1),
+            "ms_per_step_meaning": "host time of one step's sample (timed); value extrapolates it to the whole job",
+            "whole_job_ms_extrapolated": round(est * 1e3, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "Nq": w.Nq, "d": w.d,
-                       "b": w.b, "topk": w.topk, "cap": w.cap, "seed": w.seed},
+            "config": config_of(w, 1),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": desc + f"; {args.steps} steps, mean sample {statistics.mean(tooks):.2f} s"},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -656,15 +761,25 @@ def main():
                     help="also time the backward pass (route inversion + gradients) of the forward step")
     ap.add_argument("--break-even", action="store_true",
                     help="sweep the context length and report where the sparse step beats dense attention")
+    ap.add_argument("--sub-workloads", default="gqa_bf16_64k,mha_bf16_1m,decode_gqa_bf16_128k",
+                    help="comma-separated workloads timed after the headline one and reported under "
+                         "'workloads' (1 GPU only); empty for none")
+    ap.add_argument("--no-break-even", dest="with_break_even", action="store_false",
+                    help="skip the sparse-vs-dense context-length sweep reported under 'break_even'")
     ap.add_argument("--n", type=int, default=None,
                     help="shrink the context length (and query rows) of the workload: for profiling the same "
                          "kernels on a smaller case; the default JSON line always uses the full workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.sub_workloads = [x for x in args.sub_workloads.split(",") if x]
+    for x in args.sub_workloads:
+        if x not in synth.BY_NAME:
+            ap.error(f"unknown workload {x}")
     w = synth.BY_NAME[args.workload]
     if args.n:
         w = w.scaled(name=f"{w.name}@N={args.n}", N=args.n, Nq=1 if w.decode else args.n,
                      q_offset=args.n - 1 if w.decode else 0)
+        args.sub_workloads, args.with_break_even = [], False
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
