@@ -14,6 +14,10 @@ every call needs CUDA tensors.
                                               the same with the PHAROS variants (per-head budget,
                                               confidence fallback, cross-level guidance) and a trace
     bsa_forward(shape, Q, K, V, idx, O, lse)  causal block-sparse attention
+    phba_state_build(shape, M, Ks, V, A, W, PK, PV, workspace)
+                                              PHBA prefix states (gated slot recurrence, chunkwise)
+    phba_forward(shape, Q, K, V, idx, O, lse, Qs, M, PK, PV)
+                                              block-sparse attention over tokens and state slots
     dense_forward(shape, Q, K, V, O, lse)     dense causal attention
     bsa_route_invert(shape, idx, offset, rho) routes in block-major form (for the backward)
     bsa_backward(shape, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV)
@@ -36,7 +40,8 @@ PYR_F32, PYR_BF16 = 0, 1
 ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_pyramid_elems", "pyr_build", "pyr_update",
                "pyr_select", "pyr_select_ex", "pyr_select_trace_levels", "pyr_select_trace_width", "bsa_forward",
                "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes", "bsa_route_invert", "bsa_backward",
-               "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror")
+               "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror", "phba_state_elems",
+               "phba_state_workspace_bytes", "phba_state_build", "phba_forward")
 
 
 class PyrShape(ctypes.Structure):
@@ -99,6 +104,14 @@ def _load_lib():
     lib.bsa_backward.restype = ctypes.c_int
     lib.bsa_backward_noalloc.argtypes = [sp] + [vp] * 14
     lib.bsa_backward_noalloc.restype = ctypes.c_int
+    lib.phba_state_elems.argtypes = [sp, ctypes.c_int]
+    lib.phba_state_elems.restype = ctypes.c_size_t
+    lib.phba_state_workspace_bytes.argtypes = [sp, ctypes.c_int]
+    lib.phba_state_workspace_bytes.restype = ctypes.c_size_t
+    lib.phba_state_build.argtypes = [sp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.phba_state_build.restype = ctypes.c_int
+    lib.phba_forward.argtypes = [sp, vp, vp, vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, vp, vp]
+    lib.phba_forward.restype = ctypes.c_int
     lib.pyr_selftest_wait.argtypes = [vp, vp]
     lib.pyr_selftest_wait.restype = ctypes.c_int
     lib.pyr_strerror.argtypes = [ctypes.c_int]
@@ -215,6 +228,43 @@ def pyr_select_ex(s: PyrShape, Q, pyr, idx, gap=None, budget=None, fcf_tau: floa
 def bsa_forward(s: PyrShape, Q, K, V, idx, O, lse=None, status=None, stream=None):
     _check(_L().bsa_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "idx"), _dev(O, "O"),
                             _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)), "bsa_forward")
+
+
+def phba_state_elems(s: PyrShape, M: int) -> int:
+    return _L().phba_state_elems(ctypes.byref(s), int(M))
+
+
+def phba_state_workspace_bytes(s: PyrShape, M: int) -> int:
+    return _L().phba_state_workspace_bytes(ctypes.byref(s), int(M))
+
+
+class PhbaStates:
+    """Device buffers of the PHBA prefix states (PK, PV [B, Hkv, nb, M, d]) and the build workspace."""
+
+    def __init__(self, s: PyrShape, M: int, device="cuda"):
+        nb = (s.N + s.b - 1) // s.b
+        dt = torch.float32 if s.dtype == PYR_F32 else torch.bfloat16
+        self.M = M
+        self.PK = torch.empty((s.B, s.Hkv, nb, M, s.d), dtype=dt, device=device)
+        self.PV = torch.empty_like(self.PK)
+        self.workspace = torch.empty(phba_state_workspace_bytes(s, M), dtype=torch.uint8, device=device)
+
+
+def phba_state_build(s: PyrShape, M: int, Ks, V, A, W, PK, PV, workspace, status=None, stream=None):
+    """Prefix states of every key block: A (retention), W (write) fp32 CUDA tensors [B, Hkv, N, M]."""
+    _check(_L().phba_state_build(ctypes.byref(s), int(M), _dev(Ks, "Ks"), _dev(V, "V"), _dev(A, "A"), _dev(W, "W"),
+                                 _dev(PK, "PK"), _dev(PV, "PV"), _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _dev(status, "status", True),
+                                 _stream(stream)), "phba_state_build")
+
+
+def phba_forward(s: PyrShape, Q, K, V, idx, O, lse=None, Qs=None, M: int = 0, PK=None, PV=None, status=None,
+                 stream=None):
+    """bsa_forward over the tokens and the M slots of the prefix states (Qs: the state query, None = Q)."""
+    _check(_L().phba_forward(ctypes.byref(s), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "idx"),
+                             _dev(Qs, "Qs", True), int(M), _dev(PK, "PK", M == 0), _dev(PV, "PV", M == 0),
+                             _dev(O, "O"), _dev(lse, "lse", True), _dev(status, "status", True), _stream(stream)),
+           "phba_forward")
 
 
 def dense_forward(s: PyrShape, Q, K, V, O, lse=None, status=None, stream=None):

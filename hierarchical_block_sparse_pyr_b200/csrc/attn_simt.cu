@@ -10,6 +10,10 @@
 // owns 16 query rows. This kernel serves fp32 inputs (where the tolerance
 // leaves no room for reduced-precision tensor-core operands) and is the
 // general fallback for shapes the tensor-core kernels do not take.
+// With PHBA prefix states (M > 0; PHBA summary 3.3 and A.1.3) the same online
+// softmax continues over the M slots of the current block's state and of the
+// state aligned with each routed block (blocks >= 1), scored with the
+// state-branch query against the state keys; the slots carry no causal mask.
 #include "pyr_common.cuh"
 
 namespace pyr {
@@ -25,7 +29,9 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const T* __restr
                                                                 const T* __restrict__ V,
                                                                 const int32_t* __restrict__ idx, int dense,
                                                                 T* __restrict__ O, float* __restrict__ lse,
-                                                                int* status, Geo g) {
+                                                                int* status, Geo g, const T* __restrict__ Qst,
+                                                                const T* __restrict__ PK, const T* __restrict__ PV,
+                                                                int M) {
   constexpr int CPL = D / 32;  // output columns per lane
   extern __shared__ __align__(16) float sm[];
   float* Qs = sm;                          // [64][D]
@@ -101,66 +107,104 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const T* __restr
   const T* Vu = V + (size_t)unit * g.N * D;
   const int nblk = dense ? (i + 1) : s_nblk;
 
+  // one staged sub-tile of up to 32 keys: scores, online softmax, P.V. Lane `lane` owns key `lane`
+  // of the tile, valid when lane < n_keys and, with causal_first >= 0, when its position
+  // causal_first + lane is at most the row's position
+  auto consume_tile = [&](int n_keys, int causal_first) {
+    float s[16];
+#pragma unroll
+    for (int rr = 0; rr < 16; rr++) s[rr] = 0.f;
+    const float* Qw = Qs + warp * 16 * D;
+    for (int e = 0; e < D; e++) {
+      const float kv = Ks[lane * (D + 1) + e];
+#pragma unroll
+      for (int rr = 0; rr < 16; rr++) s[rr] = fmaf(Qw[rr * D + e], kv, s[rr]);
+    }
+#pragma unroll
+    for (int rr = 0; rr < 16; rr++) {
+      const bool ok = pos[rr] >= 0 && lane < n_keys && (causal_first < 0 || causal_first + lane <= pos[rr]);
+      const float x = ok ? s[rr] * scale_log2 : -INFINITY;  // log2 domain
+      float mx = x;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_new = fmaxf(m_run[rr], mx);
+      const float p = (m_new == -INFINITY) ? 0.f : exp2f(x - m_new);
+      float ps = p;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      const float corr = (m_run[rr] == -INFINITY) ? 0.f : exp2f(m_run[rr] - m_new);
+      l_run[rr] = l_run[rr] * corr + ps;
+      m_run[rr] = m_new;
+#pragma unroll
+      for (int c = 0; c < CPL; c++) acc[rr][c] *= corr;
+      Pw[rr * kKeys + lane] = p;
+    }
+    __syncwarp();
+    for (int k = 0; k < kKeys; k++) {
+      float vv[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; c++) vv[c] = Vs[k * D + lane + 32 * c];
+#pragma unroll
+      for (int rr = 0; rr < 16; rr++) {
+        const float p = Pw[rr * kKeys + k];
+#pragma unroll
+        for (int c = 0; c < CPL; c++) acc[rr][c] = fmaf(p, vv[c], acc[rr][c]);
+      }
+    }
+    __syncwarp();
+  };
+  // stage rows [r0, r0 + n) of K-like and V-like tensors (zeros past n)
+  auto stage = [&](const T* Kt, const T* Vt, int n) {
+    __syncthreads();  // previous sub-tile fully consumed
+    for (int x = threadIdx.x; x < kKeys * D; x += kWarps * 32) {
+      const int k = x / D, e = x - k * D;
+      float kv = 0.f, vv = 0.f;
+      if (k < n) {
+        kv = to_f32(Kt[(size_t)k * D + e]);
+        vv = to_f32(Vt[(size_t)k * D + e]);
+      }
+      Ks[k * (D + 1) + e] = kv;
+      Vs[k * D + e] = vv;
+    }
+    __syncthreads();
+  };
+
   for (int bk = 0; bk < nblk; bk++) {
     const int j = dense ? (bk < i ? bk : i) : s_blocks[bk];
     const int kb0 = j * g.b;
     const int kb1 = min(kb0 + g.b, g.N);
     for (int t0 = kb0; t0 < kb1; t0 += kKeys) {
-      __syncthreads();  // previous sub-tile fully consumed
-      for (int x = threadIdx.x; x < kKeys * D; x += kWarps * 32) {
-        const int k = x / D, e = x - k * D;
-        const int t = t0 + k;
-        float kv = 0.f, vv = 0.f;
-        if (t < kb1) {
-          kv = to_f32(Ku[(size_t)t * D + e]);
-          vv = to_f32(Vu[(size_t)t * D + e]);
-        }
-        Ks[k * (D + 1) + e] = kv;
-        Vs[k * D + e] = vv;
-      }
+      const int n = min(kKeys, kb1 - t0);
+      stage(Ku + (size_t)t0 * D, Vu + (size_t)t0 * D, n);
+      consume_tile(n, j < i ? -1 : t0);
+    }
+  }
+
+  if (M > 0 && !dense) {
+    // prefix-state slots: the state-branch query replaces the token query in shared memory
+    if (Qst != Q) {
       __syncthreads();
-      const int t = t0 + lane;  // this lane's key
-      float s[16];
-#pragma unroll
-      for (int rr = 0; rr < 16; rr++) s[rr] = 0.f;
-      const float* Qw = Qs + warp * 16 * D;
-      for (int e = 0; e < D; e++) {
-        const float kv = Ks[lane * (D + 1) + e];
-#pragma unroll
-        for (int rr = 0; rr < 16; rr++) s[rr] = fmaf(Qw[rr * D + e], kv, s[rr]);
-      }
-#pragma unroll
-      for (int rr = 0; rr < 16; rr++) {
-        const bool ok = pos[rr] >= 0 && t < kb1 && (j < i || t <= pos[rr]);
-        const float x = ok ? s[rr] * scale_log2 : -INFINITY;  // log2 domain
-        float mx = x;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const float m_new = fmaxf(m_run[rr], mx);
-        const float p = (m_new == -INFINITY) ? 0.f : exp2f(x - m_new);
-        float ps = p;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-        const float corr = (m_run[rr] == -INFINITY) ? 0.f : exp2f(m_run[rr] - m_new);
-        l_run[rr] = l_run[rr] * corr + ps;
-        m_run[rr] = m_new;
-#pragma unroll
-        for (int c = 0; c < CPL; c++) acc[rr][c] *= corr;
-        Pw[rr * kKeys + lane] = p;
-      }
-      __syncwarp();
-      for (int k = 0; k < kKeys; k++) {
-        float vv[CPL];
-#pragma unroll
-        for (int c = 0; c < CPL; c++) vv[c] = Vs[k * D + lane + 32 * c];
-#pragma unroll
-        for (int rr = 0; rr < 16; rr++) {
-          const float p = Pw[rr * kKeys + k];
-#pragma unroll
-          for (int c = 0; c < CPL; c++) acc[rr][c] = fmaf(p, vv[c], acc[rr][c]);
+      for (int x = threadIdx.x; x < kRows * D; x += kWarps * 32) {
+        const int r = x / D, e = x - r * D;
+        const int ra = r_begin + r;
+        float v = 0.f;
+        if (ra < R) {
+          const int gg = ra / rb, t = p0 - g.q_offset + (ra - gg * rb);
+          v = to_f32(Qst[(((size_t)bi * g.Hq + hk * g.G + gg) * g.Nq + t) * D + e]);
         }
+        Qs[x] = v;
       }
-      __syncwarp();
+    }
+    const T* PKu = PK + (size_t)unit * g.nb * M * D;
+    const T* PVu = PV + (size_t)unit * g.nb * M * D;
+    for (int bk = 0; bk < nblk; bk++) {
+      const int j = s_blocks[bk];  // routed blocks, then the current block
+      if (j < 1) continue;         // block 0 has an empty prefix: no state
+      for (int c0 = 0; c0 < M; c0 += kKeys) {
+        const int n = min(kKeys, M - c0);
+        stage(PKu + ((size_t)j * M + c0) * D, PVu + ((size_t)j * M + c0) * D, n);
+        consume_tile(n, -1);
+      }
     }
   }
 
@@ -185,7 +229,8 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const T* __restr
 
 template <typename T, int D>
 cudaError_t launch_t(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
-                     void* O, float* lse, int* status, cudaStream_t st) {
+                     void* O, float* lse, int* status, cudaStream_t st, const void* Qst, const void* PK,
+                     const void* PV, int M) {
   const size_t smem = sizeof(float) * ((size_t)kRows * D + kKeys * (D + 1) + kKeys * D + kWarps * 16 * kKeys);
   auto kern = attn_simt_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -194,19 +239,21 @@ cudaError_t launch_t(const Geo& g, const void* Q, const void* K, const void* V, 
   dim3 grid(g.nqb, g.B * g.Hkv, ceil_div(rows, kRows));
   kern<<<grid, kWarps * 32, smem, st>>>(reinterpret_cast<const T*>(Q), reinterpret_cast<const T*>(K),
                                          reinterpret_cast<const T*>(V), idx, dense, reinterpret_cast<T*>(O), lse,
-                                         status, g);
+                                         status, g, reinterpret_cast<const T*>(Qst ? Qst : Q),
+                                         reinterpret_cast<const T*>(PK), reinterpret_cast<const T*>(PV), M);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
-                             int dense, void* O, float* lse, int* status, cudaStream_t st) {
+                             int dense, void* O, float* lse, int* status, cudaStream_t st, const void* Qst,
+                             const void* PK, const void* PV, int M) {
   if (g.dtype == PYR_BF16)
-    return g.d == 128 ? launch_t<__nv_bfloat16, 128>(g, Q, K, V, idx, dense, O, lse, status, st)
-                      : launch_t<__nv_bfloat16, 64>(g, Q, K, V, idx, dense, O, lse, status, st);
-  return g.d == 128 ? launch_t<float, 128>(g, Q, K, V, idx, dense, O, lse, status, st)
-                    : launch_t<float, 64>(g, Q, K, V, idx, dense, O, lse, status, st);
+    return g.d == 128 ? launch_t<__nv_bfloat16, 128>(g, Q, K, V, idx, dense, O, lse, status, st, Qst, PK, PV, M)
+                      : launch_t<__nv_bfloat16, 64>(g, Q, K, V, idx, dense, O, lse, status, st, Qst, PK, PV, M);
+  return g.d == 128 ? launch_t<float, 128>(g, Q, K, V, idx, dense, O, lse, status, st, Qst, PK, PV, M)
+                    : launch_t<float, 64>(g, Q, K, V, idx, dense, O, lse, status, st, Qst, PK, PV, M);
 }
 
 }  // namespace pyr

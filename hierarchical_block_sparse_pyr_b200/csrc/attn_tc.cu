@@ -26,7 +26,13 @@
 // commit of QK t+2 (hence PV t) has landed.
 // The K/V tile list is the union of the query blocks' routed blocks and their
 // diagonal blocks, ascending; each entry carries a mode per query block
-// (skip / full / causal). Every mbarrier wait is bounded; a wait that runs out
+// (skip / full / causal). With PHBA prefix states (M > 0; PHBA summary 3.3 and
+// A.1.3: one softmax over tokens and state slots) the tiles of the M-slot
+// states follow the token tiles: each entry j >= 1 of the list brings the
+// state stored before block j (the current block's state for the diagonal,
+// the aligned state for a routed block), with the entry's modes and no causal
+// mask; block 0 has an empty prefix and no state. The state slots are scored
+// with the same Q tile as the tokens. Every mbarrier wait is bounded; a wait that runs out
 // aborts the CTA (PYR_ETIMEOUT), and the CTA still drains its in-flight
 // copies and MMAs and frees its tensor memory before it exits.
 #include <cudaTypedefs.h>
@@ -77,12 +83,12 @@ template <int MT, int QB, int KB, int NS>
 __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBlocks)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx, int dense,
-                   __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* status, Geo g) {
+                   __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* status, Geo g,
+                   const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPV, int M) {
   using PL = Plan<MT, NS>;
   constexpr int TPB = KB / kKeys;  // tiles per key block
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = smem_align<1024>(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
   uint64_t* bar_q = bars;
   uint64_t* bar_k_full = bars + 1;
@@ -140,10 +146,22 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   const uint32_t tS = tmem;             // S[mt][sb] at column (mt*2 + sb)*64; P over its first 32
   const uint32_t tO = tmem + 128 * MT;  // O[mt] at column 128*MT + mt*128
   const int nblk = dense ? (i_first + nq_here) : n_entries;  // dense: blocks 0 .. last diagonal
-  const int T = nblk * TPB;
+  const int T_tok = nblk * TPB;
+  // state tiles: the entries j >= 1 (the list is ascending, so only its first entry can be block 0)
+  const int st_first = (n_entries > 0 && (tiles[0] >> 4) == 0) ? 1 : 0;
+  const int SPB = M / kKeys;  // tiles per state
+  const int T = T_tok + ((M > 0 && !dense) ? (n_entries - st_first) * SPB : 0);
 
-  // tile t -> (first key, modes)
+  // tile t -> (first key row, modes); state tiles: the row in the [nb * M] state rows, full modes
   auto tile_info = [&](int t, int* key0, int* mode) {
+    if (t >= T_tok) {
+      const int k = (t - T_tok) / SPB, h = (t - T_tok) - k * SPB;
+      const int ent = tiles[st_first + k];
+      const int m = ent & 15;
+      *key0 = (ent >> 4) * M + h * kKeys;
+      *mode = (m | (m >> 1)) & 5;  // causal (2) -> full (1) in each query block's two bits
+      return;
+    }
     const int e = t / TPB, h = t - e * TPB;
     int j, m;
     if (dense) {
@@ -186,7 +204,6 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
       uint64_t* full = is_k ? bar_k_full : bar_v_full;
       uint64_t* fre = is_k ? bar_k_free : bar_v_free;
       unsigned char* ring = is_k ? sK : sV;
-      const CUtensorMap* map = is_k ? &tmK : &tmV;
       int t = 0;
       for (; t < T && ok; t++) {
         const int s = t % NS, k = t / NS;
@@ -195,6 +212,7 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
         int key0, mode;
         tile_info(t, &key0, &mode);
         unsigned char* st = ring + s * 16384;
+        const CUtensorMap* map = t < T_tok ? (is_k ? &tmK : &tmV) : (is_k ? &tmPK : &tmPV);
         mbar_expect_tx(full + s, 16384);
         for (int h = 0; h < 2; h++) tma_load_3d(st + h * 8192, map, h * 64, key0, unit, full + s);
       }
@@ -294,8 +312,9 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
       tmem_ld32(tS_row + sb * 64 + 32, s + 32);
       tmem_wait_ld();
 
-      // valid keys: full -> every key < N; causal -> keys <= p
-      const int lim = md == 0 ? 0 : (md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1));
+      // valid keys: full -> every key < N; causal -> keys <= p; state slots -> all of them
+      const int lim = md == 0 ? 0
+                              : (t >= T_tok ? kKeys : (md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1)));
       if (lim < kKeys) {
 #pragma unroll
         for (int c = 0; c < kKeys; c++) s[c] = c < lim ? s[c] : -INFINITY;
@@ -405,14 +424,15 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
 
 template <int MT, int QB, int KB, int NS>
 cudaError_t launch_cfg(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const int32_t* idx, int dense, void* O, float* lse, int* status, cudaStream_t st) {
+                       const int32_t* idx, int dense, void* O, float* lse, int* status, cudaStream_t st,
+                       const CUtensorMap& mpk, const CUtensorMap& mpv, int M) {
   using PL = Plan<MT, NS>;
   auto kern = attn_tc_kernel<MT, QB, KB, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PL::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((g.nqb + QB - 1) / QB, g.B * g.Hkv);
   kern<<<grid, PL::kThreads, PL::kBytes, st>>>(mq, mk, mv, idx, dense, reinterpret_cast<__nv_bfloat16*>(O), lse,
-                                                status, g);
+                                                status, g, mpk, mpv, M);
   return cudaGetLastError();
 }
 
@@ -428,19 +448,29 @@ bool attn_tc_supported(const Geo& g) {
 }
 
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
-                           void* O, float* lse, int* status, cudaStream_t st) {
-  CUtensorMap mq, mk, mv;
+                           void* O, float* lse, int* status, cudaStream_t st, const void* PK, const void* PV,
+                           int M) {
+  CUtensorMap mq, mk, mv, mpk, mpv;
   if (!make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq) || !make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv) ||
       !make_tmap_bf16_3d(&mv, V, g.d, g.N, g.B * g.Hkv))
     return cudaErrorInvalidValue;
+  if (M > 0) {
+    // states [B * Hkv][nb * M][d]: a tile of 64 slots is a 64-row box like a K tile
+    if (M % kKeys || !make_tmap_bf16_3d(&mpk, PK, g.d, g.nb * M, g.B * g.Hkv) ||
+        !make_tmap_bf16_3d(&mpv, PV, g.d, g.nb * M, g.B * g.Hkv))
+      return cudaErrorInvalidValue;
+  } else {
+    mpk = mk;  // unused
+    mpv = mv;
+  }
   const int rows = g.G * g.b;
   if (g.b == 64) {
-    if (rows == 64) return launch_cfg<1, 2, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
-    if (rows == 128) return launch_cfg<1, 1, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
-    return launch_cfg<2, 1, 64, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st);
+    if (rows == 64) return launch_cfg<1, 2, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
+    if (rows == 128) return launch_cfg<1, 1, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
+    return launch_cfg<2, 1, 64, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
   }
-  if (rows == 128) return launch_cfg<1, 1, 128, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st);
-  return launch_cfg<2, 1, 128, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st);
+  if (rows == 128) return launch_cfg<1, 1, 128, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
+  return launch_cfg<2, 1, 128, 3>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
 }
 
 namespace tc {

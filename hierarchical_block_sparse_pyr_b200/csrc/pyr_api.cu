@@ -17,6 +17,8 @@ namespace {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+constexpr int kPhbaMaxSlots = 256;  // prefix-state slots per state
+
 // Shape checks shared by every entry point. Returns PYR_OK and fills g.
 int make_geo(const pyr_shape* s, Geo* g) {
   if (!s) return PYR_EINVAL;
@@ -198,6 +200,52 @@ int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V,
   if (pyr::attn_decode_supported(g))
     return launch_status(pyr::launch_attn_decode(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
+}
+
+size_t phba_state_elems(const pyr_shape* s, int M) {
+  Geo g;
+  if (make_geo(s, &g) != PYR_OK || M < 1 || M > kPhbaMaxSlots) return 0;
+  return (size_t)s->B * s->Hkv * g.nb * M * s->d;
+}
+
+size_t phba_state_workspace_bytes(const pyr_shape* s, int M) {
+  Geo g;
+  if (make_geo(s, &g) != PYR_OK || M < 1 || M > kPhbaMaxSlots) return 0;
+  return pyr::phba_workspace_bytes(g, M);
+}
+
+int phba_state_build(const pyr_shape* s, int M, const void* Ks, const void* V, const float* A, const float* W,
+                     void* PK, void* PV, void* workspace, size_t workspace_bytes, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (M < 1 || M > kPhbaMaxSlots) return PYR_EUNSUPPORTED;
+  if (!Ks || !V || !A || !W || !PK || !PV || !workspace || !aligned16(Ks) || !aligned16(V) || !aligned16(A) ||
+      !aligned16(W) || !aligned16(PK) || !aligned16(PV) || !aligned16(workspace))
+    return PYR_EINVAL;
+  if (workspace_bytes < pyr::phba_workspace_bytes(g, M)) return PYR_EINVAL;
+  (void)dev_status;
+  return launch_status(pyr::launch_phba_states(g, M, Ks, V, A, W, PK, PV, workspace, (cudaStream_t)stream));
+}
+
+int phba_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, const void* Qs,
+                 int M, const void* PK, const void* PV, void* O, float* lse, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (M < 0 || M > kPhbaMaxSlots) return PYR_EUNSUPPORTED;
+  if (!Q || !K || !V || !idx || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) ||
+      (Qs && !aligned16(Qs)))
+    return PYR_EINVAL;
+  if (M > 0 && (!PK || !PV || !aligned16(PK) || !aligned16(PV))) return PYR_EINVAL;
+  const cudaStream_t st = (cudaStream_t)stream;
+  // the tensor-core kernel scores the state slots with its Q tile: it takes the states when the
+  // state branch's query is Q and the states come in whole 64-slot tiles
+  if (pyr::attn_tc_supported(g) && (M == 0 || ((Qs == nullptr || Qs == Q) && M % 64 == 0)))
+    return launch_status(pyr::launch_attn_tc(g, Q, K, V, idx, 0, O, lse, dev_status, st, PK, PV, M));
+  if (M == 0 && pyr::attn_decode_supported(g))
+    return launch_status(pyr::launch_attn_decode(g, Q, K, V, idx, 0, O, lse, dev_status, st));
+  return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, st, Qs, PK, PV, M));
 }
 
 int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, void* O, float* lse,

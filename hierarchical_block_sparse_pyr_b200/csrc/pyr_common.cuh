@@ -24,6 +24,17 @@ struct Geo {
 
 inline int ceil_div(int64_t a, int64_t b) { return (int)((a + b - 1) / b); }
 
+// Dynamic shared memory rounded up to an A-byte boundary of the shared address
+// (A a power of two). The offset is added to the __shared__ array itself, so
+// the compiler still knows the result points to shared memory and accesses it
+// with shared-memory instructions; a round trip through an integer would turn
+// every access through it into a generic one.
+template <int A>
+__device__ __forceinline__ unsigned char* smem_align(unsigned char* raw) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(raw);
+  return raw + ((A - (s & (A - 1))) & (A - 1));
+}
+
 // Device status word: the first error wins.
 __device__ __forceinline__ void report(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
@@ -84,8 +95,10 @@ cudaError_t launch_select_decode(const Geo& g, const void* Q, const __nv_bfloat1
 cudaError_t launch_select_tc(const Geo& g, const void* Q, const __nv_bfloat16* pyr, int32_t* idx, float* gap, int* status,
                              const SelOpts& o, cudaStream_t st);
 bool attn_tc_supported(const Geo& g);
+// PK, PV: PHBA prefix states [B * Hkv][nb][M][d] (M = 0: none; M % 64 == 0 here)
 cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx, int dense,
-                           void* O, float* lse, int* status, cudaStream_t st);
+                           void* O, float* lse, int* status, cudaStream_t st, const void* PK = nullptr,
+                           const void* PV = nullptr, int M = 0);
 cudaError_t launch_route_invert(const Geo& g, const int32_t* idx, int32_t* offset, int32_t* rho, int* status,
                                 cudaStream_t st);
 // parts of the SIMT backward to launch (bit mask)
@@ -101,7 +114,13 @@ cudaError_t launch_backward_dkdv_tc(const Geo& g, const void* Q, const void* K, 
 cudaError_t launch_backward_dq_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
                                   const float* lse, const float* delta, const int32_t* idx, void* dQ, int* status,
                                   cudaStream_t st);
+// Qst: the state branch's query (null: Q); PK, PV, M as for launch_attn_tc (any M)
 cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
-                             int dense, void* O, float* lse, int* status, cudaStream_t st);
+                             int dense, void* O, float* lse, int* status, cudaStream_t st, const void* Qst = nullptr,
+                             const void* PK = nullptr, const void* PV = nullptr, int M = 0);
+// PHBA prefix states: pass A (chunk-local products) and pass B (carry across blocks)
+size_t phba_workspace_bytes(const Geo& g, int M);
+cudaError_t launch_phba_states(const Geo& g, int M, const void* Ks, const void* V, const float* A, const float* W,
+                               void* PK, void* PV, void* ws, cudaStream_t st);
 
 }  // namespace pyr

@@ -235,6 +235,66 @@ PYR_API int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const 
                 float* lse, int* dev_status, void* stream);
 
 /*
+ * PHBA prefix-state branch (PHBA summary, 2.2 "Gated slot memory", 3.2
+ * "Prefix-state construction", 3.3 "Online-softmax token-state attention",
+ * A.1.1 "Chunkwise parallel prefix-state memory construction", A.1.3).
+ * Per (batch, kv head), an M-slot key state and an M-slot value state follow
+ * one slot-wise retention gate a and one write gate w (the summary prints no
+ * formula; the reading taken is)
+ *   SK[s] <- a_t[s] SK[s] + w_t[s] ks_t,   SV[s] <- a_t[s] SV[s] + w_t[s] v_t,
+ * from zero at position 0; the prefix state of key block j is (SK, SV) after
+ * the tokens at positions < j b (block 0's is zero and is never attended:
+ * its causal prefix is empty).
+ * Layouts: PK, PV [B][Hkv][nb][M][d] in s->dtype; gates A (retention) and W
+ * (write) [B][Hkv][N][M] fp32; 1 <= M <= 256.
+ */
+
+/* Elements of PK (and of PV): B * Hkv * nb * M * d; 0 on a bad shape or M. */
+PYR_API size_t phba_state_elems(const pyr_shape* s, int M);
+
+/* Device workspace bytes phba_state_build needs; 0 on a bad shape or M. */
+PYR_API size_t phba_state_workspace_bytes(const pyr_shape* s, int M);
+
+/*
+ * phba_state_build - the prefix states of every key block, computed
+ * chunkwise as the summary describes (A.1.1): within each block, log-A sums
+ * give every token's decay to the block end and the block's writes become
+ * one decay-weighted matrix product; only the block-boundary states are
+ * carried from block to block. fp32 arithmetic.
+ *   Ks        device, [B][Hkv][N][d] in s->dtype: the state branch's keys (the
+ *             pages use un-rotated keys here; pass K when there is no rotation).
+ *   V         device, [B][Hkv][N][d] in s->dtype.
+ *   A, W      device, [B][Hkv][N][M] fp32: retention in [0, 1], write gate.
+ *   PK, PV    device, [B][Hkv][nb][M][d] in s->dtype (written).
+ *   workspace device, 16-byte aligned, >= phba_state_workspace_bytes bytes,
+ *             caller-owned, contents on return unspecified.
+ * s->topk and s->cap are ignored. The whole sequence [0, N) is one sequence
+ * (the recurrence starts from zero at position 0).
+ */
+PYR_API int phba_state_build(const pyr_shape* s, int M, const void* Ks, const void* V, const float* A,
+                             const float* W, void* PK, void* PV, void* workspace, size_t workspace_bytes,
+                             int* dev_status, void* stream);
+
+/*
+ * phba_forward - bsa_forward extended with the prefix states (PHBA 3.3, A.1.3:
+ * one softmax over the exact tokens and the prefix-state slots). Row t of
+ * query block i attends, besides the keys bsa_forward gives it, to the M slots
+ * of the state before block i (if i >= 1) and of the state before each routed
+ * block j >= 1, each slot scored as qs_t . PK[slot] / sqrt(d) and carrying
+ * value PV[slot].
+ *   Q, K, V, idx, O, lse, dev_status: as for bsa_forward.
+ *   Qs     device, [B][Hq][Nq][d] in s->dtype, or NULL (Q): the query the state
+ *          slots are scored with (the pages use the un-rotated query).
+ *   M      slots per state (0: plain bsa_forward); PK, PV as phba_state_build
+ *          writes them.
+ * bf16 prefill with d = 128 and Qs NULL (or Q) and M a multiple of 64 runs on
+ * the tcgen05 tensor cores; every other case on the CUDA cores in fp32.
+ */
+PYR_API int phba_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx,
+                         const void* Qs, int M, const void* PK, const void* PV, void* O, float* lse,
+                         int* dev_status, void* stream);
+
+/*
  * dense_forward - plain causal attention over every key at position <= p
  * (the FlashAttention-style consumer the PHAROS and PHBA pages compare
  * against), for finding the context length at which selection pays off.

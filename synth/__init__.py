@@ -144,6 +144,21 @@ def normal(seed: int, stream: int, shape, dtype=torch.float32, scale: float = 1.
 
 
 STREAM_DO = 6  # the upstream gradient dO of the backward pass (streams 0-5 are the forward inputs)
+STREAM_RET, STREAM_WRITE, STREAM_QS = 7, 8, 9  # prefix-state gates and the state branch's query
+
+
+def phba_gates(w: Workload, M: int, retention_bias: float = 1.5):
+    """Seeded prefix-state gates (A retention, W write), fp32 [B, Hkv, N, M] CPU tensors in (0, 1):
+    sigmoid(N(0,1) + retention_bias) and sigmoid(N(0,1)). The bias keeps most retention gates near
+    0.8, so a state remembers a few dozen tokens."""
+    A = torch.sigmoid(normal(w.seed, STREAM_RET, (w.B, w.Hkv, w.N, M)) + retention_bias).contiguous()
+    W = torch.sigmoid(normal(w.seed, STREAM_WRITE, (w.B, w.Hkv, w.N, M))).contiguous()
+    return A, W
+
+
+def state_query(w: Workload) -> torch.Tensor:
+    """A seeded query for the state branch, distinct from Q: [B, Hq, Nq, d] in the workload dtype."""
+    return normal(w.seed, STREAM_QS, (w.B, w.Hq, w.Nq, w.d), w.torch_dtype)
 
 
 def grad_output(w: Workload, pin: bool = False) -> torch.Tensor:
