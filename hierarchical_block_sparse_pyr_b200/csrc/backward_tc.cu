@@ -83,8 +83,7 @@ __global__ void __launch_bounds__(DqPlan::kThreads, 1)
   using PL = DqPlan;
   constexpr int TPB = KB / kKeys;  // tiles per key block
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = smem_align<1024>(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
   uint64_t* bar_q = bars;               // Q and dO landed
   uint64_t* bar_k_full = bars + 1;      // [3]
@@ -412,8 +411,7 @@ __global__ void __launch_bounds__(KvPlan::kThreads, 1)
   constexpr int TPB = 128 / KB;  // key blocks per tile
   constexpr int NS = kKvStages;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = smem_align<1024>(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
   uint64_t* bar_kv = bars;                   // K and V landed
   uint64_t* bar_full = bars + 1;             // [NS] a chunk's Q, dO, lse, D landed

@@ -119,8 +119,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
                      int32_t* __restrict__ idx, float* __restrict__ gap_out, int* status, Geo g, SelOpts o) {
   using C = SelCfg<MC, NT, STACK>;
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem =
-      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem = smem_align<1024>(smem_raw);
   const int R = g.G * g.b;  // query rows of a full block (N of the MMA)
   const SelPlan L = sel_plan(R, NT * C::kATile, g.s0 + 1, 128);
   unsigned char* sQ = smem + L.q;
