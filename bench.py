@@ -320,6 +320,83 @@ def time_backward(P, s, w, Q, K, V, buf, stream, steps, warmup):
             "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "path": "tcgen05 (bf16, d=128, b in {64, 128}) else fp32 CUDA cores"}
 
 
+def phba_counts(w, M, idx):
+    """Algorithmic bytes of the state build and FLOPs of the state-aware attention (PHBA branch).
+
+    State build: read the state keys and values once, the two fp32 gates once, write the two states
+    (the fp32 workspace between its two passes is not counted). Attention: 4 d FLOPs per token pair
+    (as bsa_forward) plus 4 d per (row, slot) pair, M slots per attended state: the current block's
+    state and each routed block's, blocks >= 1 (block 0 has no state). idx: the routes of the step
+    ([B, Hkv, nqb, topk], numpy), which decide how many routed blocks are >= 1."""
+    elt = 2 if w.dtype == synth.BF16 else 4
+    U = w.B * w.Hkv
+    build_bytes = U * (2 * w.N * w.d * elt + 2 * w.N * M * 4 + 2 * w.nb * M * w.d * elt)
+    first = w.q_offset // w.b
+    nqb = idx.shape[2]
+    qbs = np.arange(nqb)
+    i = first + qbs
+    rows = w.G * (np.minimum((i + 1) * w.b, w.q_offset + w.Nq) - np.maximum(i * w.b, w.q_offset))
+    n_states = (idx >= 1).sum(axis=-1) + (i >= 1)[None, None, :]  # [B, Hkv, nqb]
+    slot_pairs = int((n_states * rows[None, None, :]).sum()) * M
+    return build_bytes, 4 * w.d * slot_pairs
+
+
+def time_phba(args, w, dev, stream, peaks, M=128):
+    """The PHBA prefix-state branch on a workload: pyramid + selection + state build + attention over
+    tokens and state slots, event-timed per call (1 GPU)."""
+    import hierarchical_block_sparse_pyr_b200 as P
+
+    s = P.shape_of(w)
+    Qh, Kh, Vh, _ = synth.generate(w)
+    Ah, Wh = synth.phba_gates(w, M)
+    Q, K, V, A, W = (t.to(dev) for t in (Qh, Kh, Vh, Ah, Wh))
+    buf = P.Buffers(s, dev)
+    st = P.PhbaStates(s, M, dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        P.pyr_build(s, K, buf.pyr, buf.status, stream)
+        P.pyr_select(s, Q, buf.pyr, buf.idx, None, buf.status, stream)
+        if ev:
+            ev[1].record(stream)
+        P.phba_state_build(s, M, K, V, A, W, st.PK, st.PV, st.workspace, buf.status, stream)
+        if ev:
+            ev[2].record(stream)
+        P.phba_forward(s, Q, K, V, buf.idx, buf.O, buf.lse, M=M, PK=st.PK, PV=st.PV, status=buf.status,
+                       stream=stream)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"phba: device status {buf.status.item()}")
+    steps = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    sel = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    bld = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    att = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+    build_bytes, slot_flops = phba_counts(w, M, buf.idx.cpu().numpy())
+    att_flops = work_counts(w)["att_flops"] + slot_flops
+    ms = sel + bld + att
+    del Q, K, V, A, W, buf, st
+    torch.cuda.empty_cache()
+    return {"workload": w.name, "M": M, "ms_per_step": round(ms, 4),
+            "value": round(w.B * w.Nq / (ms * 1e-3), 1), "unit": "tokens/s",
+            "pyramid_select_ms": round(sel, 4),
+            "state_build": {"ms": round(bld, 4), "bound": "hbm", "algorithmic_bytes": build_bytes,
+                            "achieved_gbs": round(build_bytes / (bld * 1e-3) / 1e9, 1),
+                            "frac": round(build_bytes / (bld * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "attention": {"ms": round(att, 4), "bound": "tensor", "algorithmic_tflop": round(att_flops / 1e12, 4),
+                          "achieved_tflops": round(att_flops / (att * 1e-3) / 1e12, 1),
+                          "frac": round(att_flops / (att * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}}
+
+
 def break_even(args, w):
     """Sparse step (pyramid + selection + attention) vs dense causal attention over context lengths."""
     import hierarchical_block_sparse_pyr_b200 as P
@@ -630,6 +707,8 @@ def run_ours(args, w, rank, world, local_rank):
                 out["workloads"][name] = sub_workload(args, name, dev, stream, local_rank, peaks)
     if world == 1 and rank == 0 and args.with_break_even and not w.decode:
         out["break_even"] = break_even(args, w)
+    if world == 1 and rank == 0 and args.phba_slots > 0 and not w.decode and w.dtype == synth.BF16:
+        out["phba"] = time_phba(args, w, dev, stream, peaks, args.phba_slots)
     return out
 
 
@@ -764,6 +843,9 @@ def main():
     ap.add_argument("--sub-workloads", default="gqa_bf16_64k,mha_bf16_1m,decode_gqa_bf16_128k",
                     help="comma-separated workloads timed after the headline one and reported under "
                          "'workloads' (1 GPU only); empty for none")
+    ap.add_argument("--phba-slots", type=int, default=128,
+                    help="also time the PHBA prefix-state branch with this many slots per state, reported under "
+                         "'phba' (0: skip)")
     ap.add_argument("--no-break-even", dest="with_break_even", action="store_false",
                     help="skip the sparse-vs-dense context-length sweep reported under 'break_even'")
     ap.add_argument("--n", type=int, default=None,
@@ -779,7 +861,7 @@ def main():
     if args.n:
         w = w.scaled(name=f"{w.name}@N={args.n}", N=args.n, Nq=1 if w.decode else args.n,
                      q_offset=args.n - 1 if w.decode else 0)
-        args.sub_workloads, args.with_break_even = [], False
+        args.sub_workloads, args.with_break_even, args.phba_slots = [], False, 0
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
