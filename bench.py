@@ -675,6 +675,9 @@ def run_ours(args, w, rank, world, local_rank):
     sm_clock = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
     wc, kernels, pyr_sel = kernel_report(w, per, ms_step, peaks, sm_clock)
     value = job_throughput(wc["tokens"], world, ms_step)
+    if backward:
+        backward["bound"] = "tensor"
+        backward["frac"] = round(backward["tflops"] / peaks["bf16_tflops"], 4)  # burst peak, as the forward
     l2_mib = (Qh.numel() + Kh.numel() + Vh.numel()) * Qh.element_size() >> 20
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -836,8 +839,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--backward", action="store_true",
-                    help="also time the backward pass (route inversion + gradients) of the forward step")
+    ap.add_argument("--no-backward", dest="backward", action="store_false",
+                    help="skip timing the backward pass (route inversion + gradients) of the forward step")
     ap.add_argument("--break-even", action="store_true",
                     help="sweep the context length and report where the sparse step beats dense attention")
     ap.add_argument("--sub-workloads", default="gqa_bf16_64k,mha_bf16_1m,decode_gqa_bf16_128k",
@@ -861,7 +864,7 @@ def main():
     if args.n:
         w = w.scaled(name=f"{w.name}@N={args.n}", N=args.n, Nq=1 if w.decode else args.n,
                      q_offset=args.n - 1 if w.decode else 0)
-        args.sub_workloads, args.with_break_even, args.phba_slots = [], False, 0
+        args.sub_workloads, args.with_break_even, args.phba_slots, args.backward = [], False, 0, False
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
