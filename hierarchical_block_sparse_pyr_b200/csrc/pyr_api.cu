@@ -197,6 +197,8 @@ int bsa_forward(const pyr_shape* s, const void* Q, const void* K, const void* V,
     return PYR_EINVAL;
   if (pyr::attn_tc_supported(g))
     return launch_status(pyr::launch_attn_tc(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
+  if (pyr::attn_decode_warp_supported(g))
+    return launch_status(pyr::launch_attn_decode_warp(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
   if (pyr::attn_decode_supported(g))
     return launch_status(pyr::launch_attn_decode(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, (cudaStream_t)stream));
@@ -224,8 +226,8 @@ int phba_state_build(const pyr_shape* s, int M, const void* Ks, const void* V, c
       !aligned16(W) || !aligned16(PK) || !aligned16(PV) || !aligned16(workspace))
     return PYR_EINVAL;
   if (workspace_bytes < pyr::phba_workspace_bytes(g, M)) return PYR_EINVAL;
-  (void)dev_status;
-  return launch_status(pyr::launch_phba_states(g, M, Ks, V, A, W, PK, PV, workspace, (cudaStream_t)stream));
+  return launch_status(
+      pyr::launch_phba_states(g, M, Ks, V, A, W, PK, PV, workspace, dev_status, (cudaStream_t)stream));
 }
 
 int phba_forward(const pyr_shape* s, const void* Q, const void* K, const void* V, const int32_t* idx, const void* Qs,
@@ -243,6 +245,8 @@ int phba_forward(const pyr_shape* s, const void* Q, const void* K, const void* V
   // state branch's query is Q and the states come in whole 64-slot tiles
   if (pyr::attn_tc_supported(g) && (M == 0 || ((Qs == nullptr || Qs == Q) && M % 64 == 0)))
     return launch_status(pyr::launch_attn_tc(g, Q, K, V, idx, 0, O, lse, dev_status, st, PK, PV, M));
+  if (M == 0 && pyr::attn_decode_warp_supported(g))
+    return launch_status(pyr::launch_attn_decode_warp(g, Q, K, V, idx, 0, O, lse, dev_status, st));
   if (M == 0 && pyr::attn_decode_supported(g))
     return launch_status(pyr::launch_attn_decode(g, Q, K, V, idx, 0, O, lse, dev_status, st));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, idx, 0, O, lse, dev_status, st, Qs, PK, PV, M));
@@ -256,6 +260,8 @@ int dense_forward(const pyr_shape* s, const void* Q, const void* K, const void* 
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return PYR_EINVAL;
   if (pyr::attn_tc_supported(g))
     return launch_status(pyr::launch_attn_tc(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
+  if (pyr::attn_decode_warp_supported(g))
+    return launch_status(pyr::launch_attn_decode_warp(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
   if (pyr::attn_decode_supported(g))
     return launch_status(pyr::launch_attn_decode(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));
   return launch_status(pyr::launch_attn_simt(g, Q, K, V, nullptr, 1, O, lse, dev_status, (cudaStream_t)stream));

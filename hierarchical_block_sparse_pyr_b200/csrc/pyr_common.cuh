@@ -83,6 +83,9 @@ cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int*
 cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,
                                   cudaStream_t st);
 bool attn_decode_supported(const Geo& g);
+bool attn_decode_warp_supported(const Geo& g);  // one warp per 64-key tile, G <= 8
+cudaError_t launch_attn_decode_warp(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
+                                    int dense, void* O, float* lse, int* status, cudaStream_t st);
 cudaError_t launch_attn_decode(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
                                int dense, void* O, float* lse, int* status, cudaStream_t st);
 struct SelOpts;  // selection variants and trace (select_opts.cuh)
@@ -121,6 +124,6 @@ cudaError_t launch_attn_simt(const Geo& g, const void* Q, const void* K, const v
 // PHBA prefix states: pass A (chunk-local products) and pass B (carry across blocks)
 size_t phba_workspace_bytes(const Geo& g, int M);
 cudaError_t launch_phba_states(const Geo& g, int M, const void* Ks, const void* V, const float* A, const float* W,
-                               void* PK, void* PV, void* ws, cudaStream_t st);
+                               void* PK, void* PV, void* ws, int* status, cudaStream_t st);
 
 }  // namespace pyr

@@ -164,14 +164,32 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
   }
   const int base = sel_base_budget(o, g, unit);  // level-0 budget before any fallback
   const bool rcg = o.rcg_lambda != 0.f;
+  // gather targets: thread tid copies 16-byte chunk q = lane of candidate slots c = warp + 4k; with
+  // stacked operands (at most 64 slots) the swizzled destinations depend only on (c, q) and are
+  // computed once here instead of at every level
+  constexpr int kPer = STACK ? NT * C::CPT / 4 : 1;
+  int goff[kPer];
+  if (STACK) {
+#pragma unroll
+    for (int k = 0; k < kPer; k++) goff[k] = a_chunk_off<MC, NT, STACK>(warp + 4 * k, lane);
+  }
   // start level s0: every node that begins before block i, node m in slot m
   int nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
   {
     const int ms = straddler(g.s0);
-    for (int x = tid; x < nc * 32; x += kThreads) {
-      const int c = x >> 5, q = x & 31;
-      if (c == ms) continue;
-      cp_async16(sA + a_chunk_off<MC, NT, STACK>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+    if (STACK) {
+      const __nv_bfloat16* src = pu + (size_t)g.lvl_off[g.s0] * 256 + lane * 8;
+#pragma unroll
+      for (int k = 0; k < kPer; k++) {
+        const int c = warp + 4 * k;
+        if (c < nc && c != ms) cp_async16(sA + goff[k], src + (size_t)c * 256);
+      }
+    } else {
+      for (int x = tid; x < nc * 32; x += kThreads) {
+        const int c = x >> 5, q = x & 31;
+        if (c == ms) continue;
+        cp_async16(sA + a_chunk_off<MC, NT, STACK>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+      }
     }
   }
   __syncthreads();  // barrier init visible before the TMA uses it
@@ -263,15 +281,30 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     // are left as they are: their D rows are never read
     if (!start) {
       const int ms = straddler(l);
-      for (int x = tid; x < nc * 32; x += kThreads) {
-        const int c = x >> 5, q = x & 31;
-        const int m = cand[c];
-        if (m < 0) continue;
-        unsigned char* dst = sA + a_chunk_off<MC, NT, STACK>(c, q);
-        if (m == ms)
-          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
-        else
-          cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
+      if (STACK) {
+        const __nv_bfloat16* src = pu + (size_t)g.lvl_off[l] * 256 + lane * 8;
+        const uint4 strad = *reinterpret_cast<const uint4*>(ppair + l * 512 + lane * 16);
+#pragma unroll
+        for (int k = 0; k < kPer; k++) {
+          const int c = warp + 4 * k;
+          const int m = c < nc ? cand[c] : -1;
+          if (m < 0) continue;
+          if (m == ms)
+            *reinterpret_cast<uint4*>(sA + goff[k]) = strad;
+          else
+            cp_async16(sA + goff[k], src + (size_t)m * 256);
+        }
+      } else {
+        for (int x = tid; x < nc * 32; x += kThreads) {
+          const int c = x >> 5, q = x & 31;
+          const int m = cand[c];
+          if (m < 0) continue;
+          unsigned char* dst = sA + a_chunk_off<MC, NT, STACK>(c, q);
+          if (m == ms)
+            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
+          else
+            cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
+        }
       }
     }
     cp_async_wait_all();
