@@ -16,7 +16,15 @@
 // A zero retention gives log 0 = -inf and exp(-inf) = 0, so no infinity is ever
 // subtracted from another. Arithmetic is fp32; U and D live in a caller-owned
 // workspace.
+// With bf16 inputs, d = 128 and M = 128, pass A runs on the tcgen05 tensor
+// cores: thread s builds slot s's coefficient row w_t[s] exp(R_t[s]) over the
+// block's 64 tokens, split into bf16 hi + lo rows (the pair carries fp32 to
+// about 2^-17), which form the K-major A operands [128 slots][64 tokens]; the
+// block's state keys and values arrive by TMA as MN-major B operands [64 tokens]
+// [128 d]; U_K and U_V accumulate in tensor memory (hi and lo MMAs into one
+// fp32 result) and each thread writes its slot's rows out.
 #include "pyr_common.cuh"
+#include "tc_util.cuh"
 
 namespace pyr {
 
@@ -133,18 +141,176 @@ __global__ void __launch_bounds__(kThreads) phba_scan_kernel(const float* __rest
   }
 }
 
+// Pass A on the tensor cores (bf16, d = 128, M = 128, b = 64: one 64-token box per block).
+struct TcPlan {
+  static constexpr int kXK = 0;               // [2 d-halves][64 tokens][128 B], 128-byte swizzle
+  static constexpr int kXV = 16384;
+  static constexpr int kChi = 32768;          // [128 slots][64 tokens] bf16, K-major, 128-byte swizzle
+  static constexpr int kClo = 49152;
+  static constexpr int kBar = 65536;          // x_full, mma_done
+  static constexpr int kMisc = kBar + 16;     // tmem slot, abort flag
+  static constexpr int kBytes = kMisc + 16 + 1024;  // + alignment slack
+};
+
+__global__ void __launch_bounds__(128) phba_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmKs,
+                                                            const __grid_constant__ CUtensorMap tmV,
+                                                            const float* __restrict__ A, const float* __restrict__ W,
+                                                            float* __restrict__ U, float* __restrict__ Dj,
+                                                            int* status, Geo g) {
+  using namespace tc;
+  constexpr int M = 128, D = 128, BT = 64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_align<1024>(smem_raw);
+  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + TcPlan::kBar);
+  uint64_t* bar_mma = bar_x + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + TcPlan::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + TcPlan::kMisc + 4);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int j = blockIdx.x, unit = blockIdx.y;
+  const int t0 = j * g.b, n = min(g.b, g.N - t0);
+
+  if (tid == 0) {
+    mbar_init(bar_x, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // the block's state keys and values; rows past N arrive as zeros
+    mbar_expect_tx(bar_x, 32768);
+    for (int h = 0; h < 2; h++) {
+      tma_load_3d(smem + TcPlan::kXK + h * 8192, &tmKs, h * 64, t0, unit, bar_x);
+      tma_load_3d(smem + TcPlan::kXV + h * 8192, &tmV, h * 64, t0, unit, bar_x);
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  // slot tid's coefficients over the block's tokens, from the log-A suffix sums (tokens past the
+  // block's end get 0), as bf16 hi + lo rows. Every gate is loaded first, so that all the loads are
+  // in flight together; the scan then runs on registers (c takes the write gates' place)
+  {
+    const int s = tid;
+    const float* As = A + ((size_t)unit * g.N + t0) * M + s;
+    const float* Ws = W + ((size_t)unit * g.N + t0) * M + s;
+    float a[BT], c[BT];
+#pragma unroll
+    for (int t = 0; t < BT; t++) {
+      a[t] = t < n ? __ldg(As + (size_t)t * M) : 1.f;
+      c[t] = t < n ? __ldg(Ws + (size_t)t * M) : 0.f;
+    }
+    float r = 0.f;
+#pragma unroll
+    for (int t = BT - 1; t >= 0; t--) {
+      c[t] *= __expf(r);
+      r += __logf(a[t]);
+    }
+    Dj[((size_t)unit * g.nb + j) * M + s] = __expf(r);
+#pragma unroll
+    for (int ch = 0; ch < 8; ch++) {  // 16-byte chunk ch holds tokens 8 ch .. 8 ch + 7
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        const float a = c[8 * ch + 2 * q], b = c[8 * ch + 2 * q + 1];
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
+        const __nv_bfloat162 l2 =
+            __floats2bfloat162_rn(a - __bfloat162float(h2.x), b - __bfloat162float(h2.y));
+        hi[q] = *reinterpret_cast<const uint32_t*>(&h2);
+        lo[q] = *reinterpret_cast<const uint32_t*>(&l2);
+      }
+      const int off = s * 128 + ((ch ^ (s & 7)) << 4);
+      *reinterpret_cast<uint4*>(smem + TcPlan::kChi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(smem + TcPlan::kClo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+  fence_proxy_async_smem();  // the coefficient rows are read by the tensor cores
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tD = *tmem_slot;
+  bool issued = false;
+  if (tid == 0) {
+    bool ok = mbar_wait(bar_x, 0, abort_flag);
+    if (ok) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // A K-major, B MN-major
+      const uint32_t aH = smem_u32(smem + TcPlan::kChi), aL = smem_u32(smem + TcPlan::kClo);
+      const uint32_t bK = smem_u32(smem + TcPlan::kXK), bV = smem_u32(smem + TcPlan::kXV);
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {  // 16 tokens per step
+        const uint64_t dh = sdesc_sw128(aH + kk * 32, 16, 1024), dl = sdesc_sw128(aL + kk * 32, 16, 1024);
+        const uint64_t dk = sdesc_sw128(bK + kk * 2048, 8192, 1024), dv = sdesc_sw128(bV + kk * 2048, 8192, 1024);
+        umma_bf16(tD, dh, dk, idesc, kk > 0);
+        umma_bf16(tD, dl, dk, idesc, 1);
+        umma_bf16(tD + 128, dh, dv, idesc, kk > 0);
+        umma_bf16(tD + 128, dl, dv, idesc, 1);
+      }
+      umma_commit(bar_mma);
+      issued = true;
+    } else {
+      volatile int no_abort = 0;
+      mbar_wait(bar_x, 0, &no_abort);  // the copies still land in this CTA's shared memory
+    }
+  }
+  issued = __syncthreads_or(issued);
+  bool ok = issued && mbar_wait(bar_mma, 0, abort_flag);
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    tc_fence_after();
+    // thread s holds TMEM lane s: its slot's rows of U_K (columns 0..127) and U_V (128..255)
+    const uint32_t lane_addr = tD + ((uint32_t)(warp * 32) << 16);
+    float* Us = U + ((size_t)unit * g.nb + j) * 2 * M * D;
+    float v[32];
+    for (int which = 0; which < 2; which++) {
+      float* row = Us + ((size_t)which * M + tid) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        tmem_ld32(lane_addr + which * 128 + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 8; q++)
+          *reinterpret_cast<float4*>(row + c0 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+    }
+  } else if (tid == 0 && issued) {
+    // the MMAs may still be in flight after an abort: let them finish before freeing tensor memory
+    umma_commit(bar_mma);
+    volatile int no_abort = 0;
+    mbar_wait(bar_mma, 0, &no_abort);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && tid == 0) report(status, PYR_ETIMEOUT);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tD, 256);
+  }
+}
+
 template <typename T, int D>
 cudaError_t launch_t(const Geo& g, int M, const void* Ks, const void* V, const float* A, const float* W, void* PK,
-                     void* PV, void* ws, cudaStream_t st) {
+                     void* PV, void* ws, int* status, cudaStream_t st) {
   const PhbaWs L = phba_ws(g.B * g.Hkv, g.nb, M, D);
   float* U = static_cast<float*>(ws);
   float* Dj = reinterpret_cast<float*>(static_cast<char*>(ws) + L.u_bytes);
-  const size_t smem = sizeof(float) * ((size_t)g.b * kSlotGroup + (size_t)g.b * D);
-  auto ka = phba_chunk_kernel<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  ka<<<dim3(g.nb, g.B * g.Hkv), kThreads, smem, st>>>(static_cast<const T*>(Ks), static_cast<const T*>(V), A, W, M,
-                                                       U, Dj, g);
+  cudaError_t e;
+  if (sizeof(T) == 2 && D == 128 && M == 128 && g.b == 64) {
+    CUtensorMap mk, mv;
+    if (!tc::make_tmap_bf16_3d(&mk, Ks, D, g.N, g.B * g.Hkv) || !tc::make_tmap_bf16_3d(&mv, V, D, g.N, g.B * g.Hkv))
+      return cudaErrorInvalidValue;
+    e = cudaFuncSetAttribute(phba_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TcPlan::kBytes);
+    if (e != cudaSuccess) return e;
+    phba_chunk_tc_kernel<<<dim3(g.nb, g.B * g.Hkv), 128, TcPlan::kBytes, st>>>(mk, mv, A, W, U, Dj, status, g);
+  } else {
+    const size_t smem = sizeof(float) * ((size_t)g.b * kSlotGroup + (size_t)g.b * D);
+    auto ka = phba_chunk_kernel<T, D>;
+    e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ka<<<dim3(g.nb, g.B * g.Hkv), kThreads, smem, st>>>(static_cast<const T*>(Ks), static_cast<const T*>(V), A, W,
+                                                         M, U, Dj, g);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   phba_scan_kernel<T, D><<<dim3(ceil_div((int64_t)M * D, kThreads), g.B * g.Hkv), kThreads, 0, st>>>(
@@ -157,12 +323,12 @@ cudaError_t launch_t(const Geo& g, int M, const void* Ks, const void* V, const f
 size_t phba_workspace_bytes(const Geo& g, int M) { return phba_ws(g.B * g.Hkv, g.nb, M, g.d).total; }
 
 cudaError_t launch_phba_states(const Geo& g, int M, const void* Ks, const void* V, const float* A, const float* W,
-                               void* PK, void* PV, void* ws, cudaStream_t st) {
+                               void* PK, void* PV, void* ws, int* status, cudaStream_t st) {
   if (g.dtype == PYR_BF16)
-    return g.d == 128 ? launch_t<__nv_bfloat16, 128>(g, M, Ks, V, A, W, PK, PV, ws, st)
-                      : launch_t<__nv_bfloat16, 64>(g, M, Ks, V, A, W, PK, PV, ws, st);
-  return g.d == 128 ? launch_t<float, 128>(g, M, Ks, V, A, W, PK, PV, ws, st)
-                    : launch_t<float, 64>(g, M, Ks, V, A, W, PK, PV, ws, st);
+    return g.d == 128 ? launch_t<__nv_bfloat16, 128>(g, M, Ks, V, A, W, PK, PV, ws, status, st)
+                      : launch_t<__nv_bfloat16, 64>(g, M, Ks, V, A, W, PK, PV, ws, status, st);
+  return g.d == 128 ? launch_t<float, 128>(g, M, Ks, V, A, W, PK, PV, ws, status, st)
+                    : launch_t<float, 64>(g, M, Ks, V, A, W, PK, PV, ws, status, st);
 }
 
 }  // namespace pyr
