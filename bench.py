@@ -148,7 +148,7 @@ def kernel_source(kernel, w):
     if kernel == "select":
         return "select_tc.cu" if tc_select(w) else "select.cu"
     if w.decode:
-        return "attn_decode.cu"
+        return "attn_decode_warp.cu" if w.G <= 8 else "attn_decode.cu"
     return "attn_tc.cu" if tc_attention(w) else "attn_simt.cu"
 
 
