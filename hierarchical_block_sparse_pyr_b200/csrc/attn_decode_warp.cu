@@ -3,28 +3,39 @@
 // the routed blocks plus the current block, one softmax, output and
 // log-sum-exp). HBM-bound: every routed block's keys and values are read once.
 //
-// A cluster of kCluster CTAs per (batch, kv head) splits the unit's 64-key
-// tiles (routed blocks and the current block; a 128-key block is two tiles);
-// within a CTA each of kWarps warps takes whole tiles and runs each by itself,
-// with no block-wide barrier in the loop (the other warps' tiles overlap one
-// warp's loads: two stages per warp with 32-key tiles measured slower, 0.146
-// against 0.117 ms, the per-tile work not amortising over half the keys):
-//   load   lane 0 issues a TMA load of the K tile (two 64 d x 64 key boxes,
-//          128-byte swizzle) and a 1-D bulk copy of the V tile into the warp's
-//          stage, completing on the warp's mbarrier;
-//   score  lane l owns keys l and l + 32: for each 8-element chunk of d it reads
-//          the chunk of both keys (the swizzle puts the chunks of 8 consecutive
-//          keys in 8 different bank groups) and the same chunk of every query
-//          row (one address for the whole warp: a broadcast), fp32 FMAs;
-//   softmax per query row, max and sum over the warp by shuffles; the warp's
-//          running max / sum / output are rescaled lazily per tile;
-//   P.V    lane l owns d-elements 4l .. 4l + 3; probabilities go through the
-//          warp's shared-memory row, values are read as one 256-byte row per key.
-// At the end the warps' partial states merge in shared memory, and CTA 0 of
-// the cluster merges the CTAs' through distributed shared memory. Every
-// mbarrier wait is bounded; an abort still reaches both cluster barriers.
-#include <cooperative_groups.h>
-
+// One CTA per (batch, kv head) takes the unit's 64-key tiles (routed blocks
+// and the current block; a 128-key block is two tiles); each of kWarps warps
+// takes whole tiles and runs each by itself, with no block-wide barrier in
+// the loop (the other warps' tiles overlap one warp's loads):
+//   load   lane 0 issues TMA loads of the K and V tiles (two 64 d x 64 key
+//          boxes each, 128-byte swizzle) into the warp's stage, completing on
+//          the warp's mbarrier;
+//   score  S^T = K q^T per tile on the warp's tensor-core MMAs (m16n8k16, bf16
+//          operands, fp32 accumulation): keys are the M dimension (four
+//          16-key row tiles), the G <= 8 query rows of the kv group the N
+//          dimension, d the K dimension; K fragments come from the swizzled
+//          tile by ldmatrix, q^T fragments stay in registers for the whole
+//          unit (q is used exactly, as bf16);
+//   softmax per query row over the tile's keys: each lane holds 8 keys of two
+//          rows, max and the rescaling by shuffles across the 8 lanes that
+//          share a row; exponentials on the MUFU unit;
+//   P.V    O^T += V^T P^T: V^T fragments by transposing ldmatrix from the
+//          swizzled V tile, P^T fragments by an in-register 8x8 transpose
+//          (movmatrix) of the bf16 probabilities.
+// At the end the warps' partial states (row max, sum, O) merge in shared
+// memory. Every mbarrier wait is bounded; a warp that times out drains its
+// copies in flight and the CTA reports PYR_ETIMEOUT.
+// Why warp MMAs in an HBM-bound kernel: with CUDA-core FMAs (the same loop as
+// packed fp32 FMAs) the tile's G x 64 x 128 products and the matching P.V cost
+// about 2,000 instructions per warp, and with six warps per SM the issue rate,
+// not HBM, set the time (0.104 ms on the 128K GQA decode workload, 40% of
+// HBM); as m16n8k16 MMAs they are 64 MMAs and 64 ldmatrix per tile (0.055 ms,
+// 76%). The tile is a warp-sized product that one warp owns end to end; the
+// CTA-wide tcgen05 path (single-thread issue, accumulators in TMEM lanes that
+// only their own warp can read) would put block-wide synchronisation back in
+// the loop. Splitting each unit over a cluster of 2 or 4 CTAs was slower
+// (0.115 and 0.160 ms with the CUDA-core loop): per-CTA setup and the merge
+// outweigh the extra parallelism.
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
 #include "tile_list.cuh"
@@ -38,63 +49,65 @@ using namespace tc;
 constexpr int kWarps = 6;            // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kTileKeys = 64;        // keys per tile
-constexpr int kStages = 1;           // stages per warp
-constexpr int kCluster = 2;          // CTAs per (batch, kv head)
-constexpr int kMaxGw = 8;            // query rows per kv head
+constexpr int kMaxGw = 8;            // query rows per kv head (the N = 8 of the MMAs)
 constexpr int kMaxListW = 130;
 
 struct WPlan {
-  // per warp and stage: K tile [2 halves][64 keys][128 B] (16 KB), then V tile [64 keys][256 B] (16 KB)
+  // per warp: K tile [2 d-halves][64 keys][128 B] (16 KB), then V tile, same layout (16 KB)
   static constexpr int kStageBytes = 32768;
   static constexpr int kK = 0;
-  static constexpr int kV = kK + kWarps * kStages * kStageBytes;  // (end of the stages)
-  static constexpr int kQ = kV;                            // [kMaxGw][128] fp32, scaled to log2 units
-  static constexpr int kP = kQ + kMaxGw * 128 * 4;         // per warp: [kMaxGw][32] fp32 probabilities
-  static constexpr int kML = kP + kWarps * kMaxGw * kTileKeys * 4;  // per warp: [kMaxGw] max, [kMaxGw] sum
-  static constexpr int kCta = kML + kWarps * 2 * kMaxGw * 4;  // CTA partial: [kMaxGw] max, sum, 1/sum...
-  static constexpr int kPo = kCta + 4 * kMaxGw * 4;        // CTA partial output [kMaxGw][128] fp32
-  static constexpr int kW = kPo + kMaxGw * 128 * 4;        // merge weights [kMaxGw][kCluster]
-  static constexpr int kList = kW + kMaxGw * kCluster * 4;  // the unit's block list
-  static constexpr int kBar = kList + kMaxListW * 4 + 8;   // kWarps mbarriers (8-byte aligned)
-  static constexpr int kBytes = kBar + kWarps * kStages * 8 + 16 + 1024;  // + alignment slack
+  static constexpr int kML = kK + kWarps * kStageBytes;        // per warp: [kMaxGw] max, [kMaxGw] sum
+  static constexpr int kList = kML + kWarps * 2 * kMaxGw * 4;   // the unit's block list
+  static constexpr int kBar = kList + kMaxListW * 4 + 8;        // kWarps mbarriers (8-byte aligned)
+  static constexpr int kBytes = kBar + kWarps * 8 + 16 + 1024;  // + alignment slack
 };
 
-__device__ __forceinline__ void bulk_load_w(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
+// byte offset of 16-byte chunk `ch` (8 d-elements, 0..15) of key row `key` in a tile
+// loaded as two 64 d x 64 key TMA boxes with the 128-byte swizzle
+__device__ __forceinline__ uint32_t tile_off(int key, int ch) {
+  return (uint32_t)((ch >> 3) * 8192 + key * 128 + (((ch & 7) ^ (key & 7)) << 4));
 }
 
-__device__ __forceinline__ void cluster_sync_w() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
-__device__ __forceinline__ uint32_t cluster_rank_w() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
-// bf16 pairs of a 16-byte chunk to 8 floats
-__device__ __forceinline__ void cvt8(const uint4& v, float* f) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int k = 0; k < 4; k++) {
-    f[2 * k] = __uint_as_float(w[k] << 16);
-    f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-  }
+// D += A B for one m16n8k16 tile: A 16 x 16 bf16 (4 registers), B 16 x 8 bf16 (2), D 16 x 8 fp32
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-template <int GM>  // query rows per kv head, rounded up (G <= GM <= 8)
+// transpose of an 8 x 8 matrix of 16-bit elements held one row pair per lane
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_decode_warp_kernel(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16* __restrict__ Q,
-                            const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int dense,
+    attn_decode_warp_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                            const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ idx, int dense,
                             __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* status, Geo g) {
   constexpr int D = 128;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_align<1024>(smem_raw);
-  float* qs = reinterpret_cast<float*>(smem + WPlan::kQ);
   int* list = reinterpret_cast<int*>(smem + WPlan::kList);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WPlan::kBar);
   __shared__ int tl_scratch[kTileListScratch];
@@ -103,25 +116,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t rank = cluster_rank_w();
-  const int CS = gridDim.x;
-  const int unit = blockIdx.y;
+  const int unit = blockIdx.x;
   const int bi = unit / g.Hkv, hk = unit % g.Hkv;
   const int G = g.G;
   const int pos = g.q_offset;  // the query's position
   const int i = pos / g.b;     // its (current) block
+  const int gq = lane >> 2;    // fragment row group: lanes 4gq .. 4gq + 3
+  const int cq = 2 * (lane & 3);  // fragment column pair: the query rows cq, cq + 1 of the accumulators
 
   if (tid == 0) {
     s_abort = 0;
-    for (int w = 0; w < kWarps * kStages; w++) mbar_init(bars + w, 1);
+    for (int w = 0; w < kWarps; w++) mbar_init(bars + w, 1);
     fence_mbar_init();
   }
   // the unit's blocks: routed (ascending, validated), then the current block
   if (!dense) {
-    // every thread of the CTA takes part (the helper has block-wide barriers); rank 0 alone reports
-    // bad routes, the cluster's other CTAs see the same ones
+    // every thread of the CTA takes part (the helper has block-wide barriers)
     const int n = build_tile_list<1>(idx + (size_t)unit * g.nqb * g.topk, g.topk, i, 1, tl_scratch, tl_entries,
-                                     rank == 0 ? status : nullptr);
+                                     status);
     if (warp == 0) {
       for (int e = lane; e < n; e += 32) list[e] = tl_entries[e] >> 4;
       if (lane == 0) s_n = n;
@@ -129,166 +141,166 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (tid == 0) {
     s_n = i + 1;
   }
-  const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
-  for (int x = tid; x < G * D; x += kThreads) {
-    const int gg = x / D, e = x - gg * D;
-    qs[x] = __bfloat162float(Q[((size_t)bi * g.Hq + hk * G + gg) * g.Nq * D + e]) * sl2;
+  // q^T as the B operand of the score MMAs (k = d, n = query row), for the whole unit: lane holds
+  // rows gq (zero past G), d pairs 16 kc + cq .. + 1 (b0) and 16 kc + 8 + cq .. + 1 (b1)
+  uint32_t qb[8][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(Q + ((size_t)bi * g.Hq + hk * G + gq) * g.Nq * D);
+#pragma unroll
+    for (int kc = 0; kc < 8; kc++) {
+      qb[kc][0] = gq < G ? __ldg(qrow + (16 * kc + cq) / 2) : 0u;
+      qb[kc][1] = gq < G ? __ldg(qrow + (16 * kc + 8 + cq) / 2) : 0u;
+    }
   }
   __syncthreads();
 
   const int tpb = g.b / kTileKeys;  // tiles per block
   const int n_tiles = s_n * tpb;
-  const int per = (n_tiles + CS - 1) / CS;
-  const int t_begin = min(n_tiles, (int)rank * per), t_end = min(n_tiles, t_begin + per);
-  unsigned char* stage0 = smem + WPlan::kK + warp * kStages * WPlan::kStageBytes;
-  float* sP = reinterpret_cast<float*>(smem + WPlan::kP) + warp * kMaxGw * kTileKeys;
-  uint64_t* wbar = bars + warp * kStages;
-  const __nv_bfloat16* Vu = V + (size_t)unit * g.N * D;
-  // this warp's tiles: t_begin + warp + kWarps * k, k = 0 .. n_mine - 1
-  const int n_mine = t_begin + warp < t_end ? (t_end - 1 - (t_begin + warp)) / kWarps + 1 : 0;
+  unsigned char* stage = smem + WPlan::kK + warp * WPlan::kStageBytes;
+  uint64_t* wbar = bars + warp;
+  // this warp's tiles: warp + kWarps * k, k = 0 .. n_mine - 1
+  const int n_mine = warp < n_tiles ? (n_tiles - 1 - warp) / kWarps + 1 : 0;
   auto tile_of = [&](int k, int* j, int* key0, int* nk) {
-    const int t = t_begin + warp + kWarps * k;
+    const int t = warp + kWarps * k;
     *j = dense ? t / tpb : list[t / tpb];
     *key0 = *j * g.b + (t % tpb) * kTileKeys;
     *nk = max(0, min(kTileKeys, g.N - *key0));
   };
-  auto issue = [&](int k) {  // lane 0: tile k into stage k % kStages
+  auto issue = [&](int k) {  // lane 0: tile k into the warp's stage; keys past N arrive as zeros
     int j, key0, nk;
     tile_of(k, &j, &key0, &nk);
-    unsigned char* st = stage0 + (k % kStages) * WPlan::kStageBytes;
-    uint64_t* bar = wbar + (k % kStages);
-    // the K boxes always move 16 KB (keys past N arrive as zeros); V moves its nk rows
-    mbar_expect_tx(bar, 16384 + (uint32_t)nk * D * 2);
-    tma_load_3d(st, &tmK, 0, key0, unit, bar);
-    tma_load_3d(st + 8192, &tmK, 64, key0, unit, bar);
-    if (nk > 0) bulk_load_w(st + 16384, Vu + (size_t)key0 * D, (uint32_t)nk * D * 2, bar);
+    mbar_expect_tx(wbar, 32768);
+    tma_load_3d(stage, &tmK, 0, key0, unit, wbar);
+    tma_load_3d(stage + 8192, &tmK, 64, key0, unit, wbar);
+    tma_load_3d(stage + 16384, &tmV, 0, key0, unit, wbar);
+    tma_load_3d(stage + 24576, &tmV, 64, key0, unit, wbar);
   };
-  if (lane == 0)
-    for (int k = 0; k < min(kStages, n_mine); k++) issue(k);
+  if (lane == 0 && n_mine > 0) issue(0);
 
-  float m_run[GM], l_run[GM], acc[GM][4];
+  // ldmatrix row addresses. K (A operand of the scores, m = key, k = d): matrix lane / 8 of a
+  // 16 x 16 fragment is keys + 8 (lane & 8), d-chunk + (lane >> 4). V^T (A operand of P.V,
+  // m = d, k = key, transposing load of V rows): keys + 8 (lane >> 4), d-chunk + ((lane >> 3) & 1).
+  const uint32_t sK = smem_u32(stage), sV = smem_u32(stage + 16384);
+  const int k_key = (lane & 7) + (lane & 8), k_ch = lane >> 4;
+  const int v_key = (lane & 7) + ((lane >> 4) << 3), v_ch = (lane >> 3) & 1;
+
+  const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  float o[8][4];  // O^T: d rows 16 md + gq (+ 8 in [2], [3]), query rows cq, cq + 1
 #pragma unroll
-  for (int r = 0; r < GM; r++) {
-    m_run[r] = -INFINITY;
-    l_run[r] = 0.f;
+  for (int md = 0; md < 8; md++)
 #pragma unroll
-    for (int c = 0; c < 4; c++) acc[r][c] = 0.f;
-  }
+    for (int c = 0; c < 4; c++) o[md][c] = 0.f;
   bool ok = true;
   int k = 0;
   for (; k < n_mine; k++) {
-    ok = mbar_wait(wbar + (k % kStages), (k / kStages) & 1, (volatile int*)&s_abort);
+    ok = mbar_wait(wbar, k & 1, (volatile int*)&s_abort);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     int j, key0, nk;
     tile_of(k, &j, &key0, &nk);
-    const unsigned char* sK = stage0 + (k % kStages) * WPlan::kStageBytes;
-    const __nv_bfloat16* sV = reinterpret_cast<const __nv_bfloat16*>(sK + 16384);
 
-    // ---- scores of keys lane and lane + 32 against every query row (log2 units)
-    float s0[GM], s1[GM];
+    // ---- S^T = K q^T: four 16-key row tiles, eight 16-wide d steps
+    float sc[4][4];
 #pragma unroll
-    for (int r = 0; r < GM; r++) s0[r] = s1[r] = 0.f;
-#pragma unroll 2
-    for (int cc = 0; cc < 16; cc++) {
-      const int h = cc >> 3, c = cc & 7;
-      const int off = h * 8192 + lane * 128 + ((c ^ (lane & 7)) << 4);
-      float k0[8], k1[8];
-      cvt8(*reinterpret_cast<const uint4*>(sK + off), k0);
-      cvt8(*reinterpret_cast<const uint4*>(sK + off + 32 * 128), k1);
+    for (int mt = 0; mt < 4; mt++) {
 #pragma unroll
-      for (int r = 0; r < GM; r++) {
-        if (r < G) {
-          const float4 qa = *reinterpret_cast<const float4*>(qs + r * D + cc * 8);
-          const float4 qb = *reinterpret_cast<const float4*>(qs + r * D + cc * 8 + 4);
-          float a = s0[r], b = s1[r];
-          a = fmaf(qa.x, k0[0], a); b = fmaf(qa.x, k1[0], b);
-          a = fmaf(qa.y, k0[1], a); b = fmaf(qa.y, k1[1], b);
-          a = fmaf(qa.z, k0[2], a); b = fmaf(qa.z, k1[2], b);
-          a = fmaf(qa.w, k0[3], a); b = fmaf(qa.w, k1[3], b);
-          a = fmaf(qb.x, k0[4], a); b = fmaf(qb.x, k1[4], b);
-          a = fmaf(qb.y, k0[5], a); b = fmaf(qb.y, k1[5], b);
-          a = fmaf(qb.z, k0[6], a); b = fmaf(qb.z, k1[6], b);
-          a = fmaf(qb.w, k0[7], a); b = fmaf(qb.w, k1[7], b);
-          s0[r] = a;
-          s1[r] = b;
-        }
+      for (int c = 0; c < 4; c++) sc[mt][c] = 0.f;
+#pragma unroll
+      for (int kc = 0; kc < 8; kc++) {
+        uint32_t a[4];
+        ldsm_x4(sK + tile_off(16 * mt + k_key, 2 * kc + k_ch), a);
+        mma16816(sc[mt], a, qb[kc][0], qb[kc][1]);
       }
     }
-    // ---- online softmax per row: keys past N or past the query's position are masked
-    const bool v0 = lane < nk && (j < i || key0 + lane <= pos);
-    const bool v1 = lane + 32 < nk && (j < i || key0 + lane + 32 <= pos);
+    // ---- online softmax per query row (lane: rows cq + e, keys 16 mt + gq (+ 8)); masked keys:
+    // past N, or past the query's position in its own block
+    float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int r = 0; r < GM; r++) {
-      if (r < G) {
-        const float a = v0 ? s0[r] : -INFINITY, b = v1 ? s1[r] : -INFINITY;
-        float mx = fmaxf(a, b);
+    for (int mt = 0; mt < 4; mt++)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float m_new = fmaxf(m_run[r], mx);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float p0 = ex2(a - m_use), p1 = ex2(b - m_use);
-        float sum = p0 + p1;
+      for (int c = 0; c < 4; c++) {
+        const int key = 16 * mt + gq + ((c >> 1) << 3);
+        const bool valid = key < nk && (j < i || key0 + key <= pos);
+        sc[mt][c] = valid ? sc[mt][c] * sl2 : -INFINITY;
+        mx[c & 1] = fmaxf(mx[c & 1], sc[mt][c]);
+      }
+    float corr[2], m_use[2];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const float corr = m_run[r] == -INFINITY ? 0.f : ex2(m_run[r] - m_use);
-        l_run[r] = l_run[r] * corr + sum;
-        m_run[r] = m_new;
+    for (int e = 0; e < 2; e++) {
 #pragma unroll
-        for (int c = 0; c < 4; c++) acc[r][c] *= corr;
-        sP[r * kTileKeys + lane] = p0;
-        sP[r * kTileKeys + lane + 32] = p1;
+      for (int sh = 4; sh < 32; sh <<= 1) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], sh));
+      const float m_new = fmaxf(m_run[e], mx[e]);
+      m_use[e] = m_new == -INFINITY ? 0.f : m_new;
+      corr[e] = m_run[e] == -INFINITY ? 0.f : ex2(m_run[e] - m_use[e]);
+      m_run[e] = m_new;
+    }
+    float ls[2] = {0.f, 0.f};
+    uint32_t pb[4][2];  // P^T as the B operand of P.V (k = key, n = query row), per 16-key step
+#pragma unroll
+    for (int mt = 0; mt < 4; mt++) {
+      const float p0 = ex2(sc[mt][0] - m_use[0]), p1 = ex2(sc[mt][1] - m_use[1]);
+      const float p2 = ex2(sc[mt][2] - m_use[0]), p3 = ex2(sc[mt][3] - m_use[1]);
+      ls[0] += p0 + p2;
+      ls[1] += p1 + p3;
+      // lane holds (key gq, rows cq, cq + 1): the transpose gives (row gq, keys cq, cq + 1)
+      pb[mt][0] = movmatrix_t(pack_bf16x2(p0, p1));
+      pb[mt][1] = movmatrix_t(pack_bf16x2(p2, p3));
+    }
+#pragma unroll
+    for (int e = 0; e < 2; e++) l_run[e] = l_run[e] * corr[e] + ls[e];
+    if (__any_sync(0xffffffffu, corr[0] != 1.f || corr[1] != 1.f)) {
+#pragma unroll
+      for (int md = 0; md < 8; md++) {
+        o[md][0] *= corr[0];
+        o[md][1] *= corr[1];
+        o[md][2] *= corr[0];
+        o[md][3] *= corr[1];
       }
     }
-    __syncwarp();
-    // ---- P.V: lane owns d-elements 4 lane .. 4 lane + 3
-#pragma unroll 4
-    for (int key = 0; key < nk; key++) {
-      const uint2 w = *reinterpret_cast<const uint2*>(sV + (size_t)key * D + lane * 4);
-      const float x0 = __uint_as_float(w.x << 16), x1 = __uint_as_float(w.x & 0xFFFF0000u);
-      const float x2 = __uint_as_float(w.y << 16), x3 = __uint_as_float(w.y & 0xFFFF0000u);
+    // ---- O^T += V^T P^T: eight 16-wide d row tiles, four 16-key steps
 #pragma unroll
-      for (int r = 0; r < GM; r++) {
-        if (r < G) {
-          const float p = sP[r * kTileKeys + key];
-          acc[r][0] = fmaf(p, x0, acc[r][0]);
-          acc[r][1] = fmaf(p, x1, acc[r][1]);
-          acc[r][2] = fmaf(p, x2, acc[r][2]);
-          acc[r][3] = fmaf(p, x3, acc[r][3]);
-        }
+    for (int md = 0; md < 8; md++)
+#pragma unroll
+      for (int kk = 0; kk < 4; kk++) {
+        uint32_t a[4];
+        ldsm_x4_t(sV + tile_off(16 * kk + v_key, 2 * md + v_ch), a);
+        mma16816(o[md], a, pb[kk][0], pb[kk][1]);
       }
-    }
-    __syncwarp();  // the stage and the probabilities are free again
-    if (lane == 0 && k + kStages < n_mine) issue(k + kStages);
+    __syncwarp();  // every lane's reads of the stage are done before it is refilled
+    if (lane == 0 && k + 1 < n_mine) issue(k + 1);
   }
-  if (!ok) {
-    // drain: this warp's copies still in flight (issued for tiles k .. k + kStages - 1)
-    if (lane == 0) {
-      volatile int no_abort = 0;
-      for (int u = k; u < min(n_mine, k + kStages); u++) mbar_wait(wbar + (u % kStages), (u / kStages) & 1, &no_abort);
-      report(status, PYR_ETIMEOUT);
-    }
+  if (!ok && lane == 0) {
+    // drain: this warp's copy still in flight (issued for tile k)
+    volatile int no_abort = 0;
+    mbar_wait(wbar, k & 1, &no_abort);
+    report(status, PYR_ETIMEOUT);
   }
-  __syncthreads();  // every warp done with its stages: they hold the warps' partial outputs now
+  // the row sums: lanes gq = 0 .. 7 hold parts of the same rows
+#pragma unroll
+  for (int e = 0; e < 2; e++)
+#pragma unroll
+    for (int sh = 4; sh < 32; sh <<= 1) l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], sh);
+  __syncthreads();  // every warp done with its stage: the stages hold the warps' partial outputs now
 
   // ---- merge the warps: per row the max, the rescaled sums and outputs
-  float* wml = reinterpret_cast<float*>(smem + WPlan::kML);    // [warp][2][kMaxGw]
-  float* wacc = reinterpret_cast<float*>(smem + WPlan::kK);    // [warp][kMaxGw][128], over the stages
-  if (lane == 0) {
+  float* wml = reinterpret_cast<float*>(smem + WPlan::kML);  // [warp][2][kMaxGw]
+  float* wacc = reinterpret_cast<float*>(smem + WPlan::kK);  // [warp][kMaxGw][128], over the stages
+  if (gq == 0) {
 #pragma unroll
-    for (int r = 0; r < GM; r++) {
-      wml[(warp * 2) * kMaxGw + r] = m_run[r];
-      wml[(warp * 2 + 1) * kMaxGw + r] = l_run[r];
+    for (int e = 0; e < 2; e++) {
+      wml[(warp * 2) * kMaxGw + cq + e] = m_run[e];
+      wml[(warp * 2 + 1) * kMaxGw + cq + e] = l_run[e];
     }
   }
 #pragma unroll
-  for (int r = 0; r < GM; r++)
-    if (r < G)
-      *reinterpret_cast<float4*>(wacc + ((size_t)warp * kMaxGw + r) * D + lane * 4) =
-          make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+  for (int md = 0; md < 8; md++)
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+      const int r = cq + (c & 1), d = 16 * md + gq + ((c >> 1) << 3);
+      wacc[((size_t)warp * kMaxGw + r) * D + d] = o[md][c];
+    }
   __syncthreads();
-  float* cml = reinterpret_cast<float*>(smem + WPlan::kCta);  // [0]: max, [kMaxGw]: sum
-  float* po = reinterpret_cast<float*>(smem + WPlan::kPo);
   for (int x = tid; x < G * D; x += kThreads) {
     const int r = x / D, e = x - r * D;
     float M = -INFINITY;
@@ -298,76 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int w = 0; w < kWarps; w++) {
       const float mw = wml[(w * 2) * kMaxGw + r];
-      const float sc = mw == -INFINITY ? 0.f : ex2(mw - M);
-      L += sc * wml[(w * 2 + 1) * kMaxGw + r];
-      a += sc * wacc[((size_t)w * kMaxGw + r) * D + e];
+      const float scl = mw == -INFINITY ? 0.f : ex2(mw - M);
+      L += scl * wml[(w * 2 + 1) * kMaxGw + r];
+      a += scl * wacc[((size_t)w * kMaxGw + r) * D + e];
     }
-    po[x] = a;
-    if (e == 0) {
-      cml[r] = M;
-      cml[kMaxGw + r] = L;
-    }
+    const size_t orow = ((size_t)bi * g.Hq + hk * G + r) * g.Nq;
+    O[orow * D + e] = __float2bfloat16_rn(L > 0.f ? a / L : 0.f);
+    if (e == 0 && lse) lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
   }
-  __syncthreads();
-  cluster_sync_w();
-  if (rank == 0) {
-    namespace cg = cooperative_groups;
-    cg::cluster_group cluster = cg::this_cluster();
-    float* wts = reinterpret_cast<float*>(smem + WPlan::kW);  // [kMaxGw][kCluster], then 1/L in cml
-    for (int r = tid; r < G; r += kThreads) {
-      float mr[kCluster], lr[kCluster], M = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kCluster; c++) {
-        mr[c] = c < CS ? *cluster.map_shared_rank(cml + r, c) : -INFINITY;
-        lr[c] = c < CS ? *cluster.map_shared_rank(cml + kMaxGw + r, c) : 0.f;
-        M = fmaxf(M, mr[c]);
-      }
-      float L = 0.f;
-#pragma unroll
-      for (int c = 0; c < kCluster; c++) {
-        const float w = mr[c] == -INFINITY ? 0.f : ex2(mr[c] - M);
-        wts[r * kCluster + c] = w;
-        L += w * lr[c];
-      }
-      cml[2 * kMaxGw + r] = L > 0.f ? 1.f / L : 0.f;
-      const size_t orow = ((size_t)bi * g.Hq + hk * G + r) * g.Nq;
-      if (lse) lse[orow] = (M + log2f(L)) * 0.6931471805599453f;
-    }
-    __syncthreads();
-    for (int x = tid; x < G * D; x += kThreads) {
-      const int r = x / D;
-      float a = 0.f;
-#pragma unroll
-      for (int c = 0; c < kCluster; c++)
-        if (c < CS) a += wts[r * kCluster + c] * *cluster.map_shared_rank(po + x, c);
-      const size_t orow = ((size_t)bi * g.Hq + hk * G + r) * g.Nq;
-      O[orow * D + (x - r * D)] = __float2bfloat16_rn(a * cml[2 * kMaxGw + r]);
-    }
-  }
-  cluster_sync_w();  // no CTA leaves while CTA 0 still reads its shared memory
-}
-
-template <int GM>
-cudaError_t launch_gm(const Geo& g, const CUtensorMap& mk, const void* Q, const void* V, const int32_t* idx, int dense,
-                      void* O, float* lse, int* status, cudaStream_t st) {
-  auto kern = attn_decode_warp_kernel<GM>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WPlan::kBytes);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kCluster, g.B * g.Hkv, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = WPlan::kBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mk, reinterpret_cast<const __nv_bfloat16*>(Q),
-                            reinterpret_cast<const __nv_bfloat16*>(V), idx, dense,
-                            reinterpret_cast<__nv_bfloat16*>(O), lse, status, g);
 }
 
 }  // namespace
@@ -379,10 +329,16 @@ bool attn_decode_warp_supported(const Geo& g) {
 
 cudaError_t launch_attn_decode_warp(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,
                                     int dense, void* O, float* lse, int* status, cudaStream_t st) {
-  CUtensorMap mk;
-  if (!make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv, kTileKeys)) return cudaErrorInvalidValue;
-  if (g.G <= 4) return launch_gm<4>(g, mk, Q, V, idx, dense, O, lse, status, st);
-  return launch_gm<8>(g, mk, Q, V, idx, dense, O, lse, status, st);
+  CUtensorMap mk, mv;
+  if (!make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv, kTileKeys) ||
+      !make_tmap_bf16_3d(&mv, V, g.d, g.N, g.B * g.Hkv, kTileKeys))
+    return cudaErrorInvalidValue;
+  auto kern = attn_decode_warp_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, WPlan::kBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<g.B * g.Hkv, kThreads, WPlan::kBytes, st>>>(mk, mv, reinterpret_cast<const __nv_bfloat16*>(Q), idx, dense,
+                                                     reinterpret_cast<__nv_bfloat16*>(O), lse, status, g);
+  return cudaGetLastError();
 }
 
 }  // namespace pyr

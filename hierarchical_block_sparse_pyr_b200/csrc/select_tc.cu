@@ -337,6 +337,72 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     // halves of every 64-column batch with one shuffle each, so that each holds hi + lo for 32
     // columns; each keeps an online max and sum over its columns, and the pair merges at the end
     const bool full = (rb == g.b);
+    if constexpr (kSplit) {
+      // M = 64 stacked rows: the 16-lane TMEM load hands thread t the hi row (lane t/4) and the lo
+      // row (lane t/4 + 8) of candidate warp*H + t/4 at the same two columns of every eight, so
+      // hi + lo is thread-local and four threads split the candidate's query rows
+      const int c = warp * C::H + (lane >> 2);
+      const int cb = 2 * (lane & 3);
+      float m2 = -INFINITY, s2 = 0.f;
+      if (ntiles > 0 && __any_sync(0xffffffffu, c < nc)) {  // warp-uniform
+#pragma unroll 1
+        for (int c0 = 0; c0 < R; c0 += 64) {
+          uint32_t r[32];
+          tmem_ld16x256b_x8(my_lane_addr + c0, r);
+          tmem_wait_ld();
+          float x[16];
+#pragma unroll
+          for (int k = 0; k < 8; k++) {
+            x[2 * k] = __uint_as_float(r[4 * k]) + __uint_as_float(r[4 * k + 2]);
+            x[2 * k + 1] = __uint_as_float(r[4 * k + 1]) + __uint_as_float(r[4 * k + 3]);
+          }
+          if (!full) {
+#pragma unroll
+            for (int k = 0; k < 16; k++) x[k] = ((c0 + 8 * (k >> 1) + cb + (k & 1)) % g.b) < rb ? x[k] : -INFINITY;
+          }
+          float a[6];
+#pragma unroll
+          for (int k = 0; k < 5; k++) a[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+          a[5] = x[15];
+          const float bm = fmax3(fmax3(a[0], a[1], a[2]), a[3], fmaxf(a[4], a[5])) * sl2;
+          const float mn = fmaxf(m2, bm);
+          if (mn != -INFINITY) {
+            s2 *= ex2(m2 - mn);  // 0 on the first valid batch (m2 = -inf)
+            m2 = mn;
+            const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
+            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int k = 0; k < 8; k++) {
+              const float2 y = __ffma2_rn(make_float2(x[2 * k], x[2 * k + 1]), scl, off);
+              acc[k & 1] = __fadd2_rn(acc[k & 1], make_float2(ex2(y.x), ex2(y.y)));
+            }
+            const float2 sum = __fadd2_rn(acc[0], acc[1]);
+            s2 += sum.x + sum.y;
+          }
+        }
+      }
+      // merge the four threads of the candidate
+#pragma unroll
+      for (int sh = 1; sh <= 2; sh <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m2, sh), so = __shfl_xor_sync(0xffffffffu, s2, sh);
+        const float M = fmaxf(m2, mo);
+        s2 = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
+        m2 = M;
+      }
+      if ((lane & 3) == 0 && c < nc) {
+        const int m = start ? c : cand[c];
+        unsigned long long key = 0ull;  // empty slots rank below every node
+        if (m >= 0) {
+          const int j0 = m << l;
+          const int j1 = min(min((m + 1) << l, g.nb), i);
+          const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
+          float sc = (m2 + __log2f(s2)) * 0.6931471805599453f + __logf(nval);
+          if (rcg && !start) sc = fmaf(o.rcg_lambda, psc[c], sc);
+          key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
+        }
+        keys[c] = key;
+      }
+    } else
 #pragma unroll 1
     for (int t = 0; t < ntiles; t++) {
       const int c = t * C::CPT + my_cq;
