@@ -33,14 +33,15 @@ __device__ __forceinline__ int lower_bound_smem(const int* a, int n, int v) {
   return lo;
 }
 
-// Call from every thread of the CTA (it contains block-wide barriers).
-// rows: the QB idx rows in global memory (row q = query block i_first + q);
-// nq: query blocks present (1..QB). Returns the number of entries in tiles.
-template <int QB>
-__device__ int build_tile_list(const int32_t* __restrict__ rows, int topk, int i_first, int nq, int* scratch,
-                               int* tiles, int* status) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int* cnt = scratch + 4 * kTileListPitch;  // [0], [1]: list lengths
+// Compaction of the routes of nq (1..2) consecutive query blocks, one warp per
+// block: list q (at scratch + q * kTileListPitch) holds row q's accepted routes,
+// ascending, then the block's own index; its length is at
+// scratch[4 * kTileListPitch + q]. Call from every thread of the CTA (it ends
+// with a block-wide barrier).
+__device__ inline void compact_routes(const int32_t* __restrict__ rows, int topk, int i_first, int nq, int* scratch,
+                                      int* status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* cnt = scratch + 4 * kTileListPitch;
   if (warp < nq) {
     // compact the accepted routes of row `warp`, then append its own block
     const int iq = i_first + warp;
@@ -72,6 +73,17 @@ __device__ int build_tile_list(const int32_t* __restrict__ rows, int topk, int i
     }
   }
   __syncthreads();
+}
+
+// Call from every thread of the CTA (it contains block-wide barriers).
+// rows: the QB idx rows in global memory (row q = query block i_first + q);
+// nq: query blocks present (1..QB). Returns the number of entries in tiles.
+template <int QB>
+__device__ int build_tile_list(const int32_t* __restrict__ rows, int topk, int i_first, int nq, int* scratch,
+                               int* tiles, int* status) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int* cnt = scratch + 4 * kTileListPitch;  // [0], [1]: list lengths
+  compact_routes(rows, topk, i_first, nq, scratch, status);
   const int na = cnt[0];
   const int* A = scratch;
   if (QB == 1 || nq == 1) {

@@ -36,6 +36,9 @@ CASES = [
               dtype=BF16, seed=19, n_needle=0),
     W0.scaled(name="chunked_prefill", B=1, Hq=4, Hkv=2, N=2048, Nq=1024, q_offset=1024, d=128, b=64, topk=4, cap=8,
               dtype=BF16, seed=20),
+    # MHA chunked prefill: 64-row query blocks paired from block 16 on, an odd count (the last CTA has one)
+    W0.scaled(name="chunked_prefill_mha", B=1, Hq=3, Hkv=3, N=2100, Nq=1076, q_offset=1024, d=128, b=64, topk=5,
+              cap=10, dtype=BF16, seed=33),
     W0.scaled(name="mha_bf16_odd_qblocks", B=1, Hq=2, Hkv=2, N=2100, Nq=2100, d=128, b=64, topk=5, cap=10,
               dtype=BF16, seed=25),
     W0.scaled(name="gqa2_bf16_b128", B=1, Hq=4, Hkv=2, N=3000, Nq=3000, d=128, b=128, topk=4, cap=8, dtype=BF16,
