@@ -149,6 +149,8 @@ def kernel_source(kernel, w):
         return "select_tc.cu" if tc_select(w) else "select.cu"
     if w.decode:
         return "attn_decode_warp.cu" if w.G <= 8 else "attn_decode.cu"
+    if tc_attention(w) and w.G == 1 and w.b == 64:
+        return "attn_pair.cu"  # 64-row MHA query blocks, two per CTA over their own lists
     return "attn_tc.cu" if tc_attention(w) else "attn_simt.cu"
 
 

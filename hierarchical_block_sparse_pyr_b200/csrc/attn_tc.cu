@@ -227,7 +227,10 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kKeys, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      // operand descriptors: the base of each operand once; a stage and a K step add offsets to the
+      // start-address field (16-byte units, no carry: shared addresses stay below 2^18 bytes)
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024), dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       int issued = 0;
       for (int t = 0; t <= T && ok; t++) {
@@ -236,12 +239,13 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
           ok = mbar_wait(bar_k_full + s, (t / NS) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t dKs = dK + (uint64_t)(s * (16384 >> 4));
+#pragma unroll
           for (int mt = 0; mt < MT; mt++)
-            for (int kk = 0; kk < 8; kk++) {
-              const uint64_t a = sdesc_sw128(aQ + mt * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-              const uint64_t b = sdesc_sw128(aK + s * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-              umma_bf16(tS + (mt * 2 + sb) * 64, a, b, idesc_qk, kk > 0);
-            }
+#pragma unroll
+            for (int kk = 0; kk < 8; kk++)
+              umma_bf16(tS + (mt * 2 + sb) * 64, dQ + (uint64_t)((mt * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                        dKs + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
           umma_commit(bar_s_full + sb);
           umma_commit(bar_k_free + s);
           issued++;
@@ -252,11 +256,14 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
           if (ok) ok = mbar_wait(bar_v_full + s, (u / NS) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
+          const uint64_t dVs = dV + (uint64_t)(s * (16384 >> 4));
+          const uint32_t acc0 = u > 0 ? 1u : 0u;
+#pragma unroll
           for (int mt = 0; mt < MT; mt++)
-            for (int kk = 0; kk < 4; kk++) {
-              const uint64_t b = sdesc_sw128(aV + s * 16384 + kk * 2048, 8192, 1024);
-              umma_bf16_ts(tO + mt * 128, tS + (mt * 2 + pb) * 64 + kk * 8, b, idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
-            }
+#pragma unroll
+            for (int kk = 0; kk < 4; kk++)
+              umma_bf16_ts(tO + mt * 128, tS + (mt * 2 + pb) * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                           kk > 0 ? 1u : acc0);
           umma_commit(bar_v_free + s);
           umma_commit(bar_o);
           issued++;
