@@ -16,13 +16,11 @@
 // A zero retention gives log 0 = -inf and exp(-inf) = 0, so no infinity is ever
 // subtracted from another. Arithmetic is fp32; U and D live in a caller-owned
 // workspace.
-// With bf16 inputs, d = 128 and M = 128, pass A runs on the tcgen05 tensor
-// cores: thread s builds slot s's coefficient row w_t[s] exp(R_t[s]) over the
-// block's 64 tokens, split into bf16 hi + lo rows (the pair carries fp32 to
-// about 2^-17), which form the K-major A operands [128 slots][64 tokens]; the
-// block's state keys and values arrive by TMA as MN-major B operands [64 tokens]
-// [128 d]; U_K and U_V accumulate in tensor memory (hi and lo MMAs into one
-// fp32 result) and each thread writes its slot's rows out.
+// With bf16 inputs, d = 128, b = 64 and M a multiple of 32, a single kernel
+// replaces both passes (phba_carry_tc_kernel below): each CTA carries its part
+// of the state through the blocks in order, the block products run on the
+// tcgen05 tensor cores, and U and D never leave the chip (no workspace
+// traffic, which in the two-pass form was 2 x 4 bytes per state element).
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
 
@@ -141,151 +139,234 @@ __global__ void __launch_bounds__(kThreads) phba_scan_kernel(const float* __rest
   }
 }
 
-// Pass A on the tensor cores (bf16, d = 128, M = 128, b = 64: one 64-token box per block).
-struct TcPlan {
-  static constexpr int kXK = 0;               // [2 d-halves][64 tokens][128 B], 128-byte swizzle
-  static constexpr int kXV = 16384;
-  static constexpr int kChi = 32768;          // [128 slots][64 tokens] bf16, K-major, 128-byte swizzle
-  static constexpr int kClo = 49152;
-  static constexpr int kBar = 65536;          // x_full, mma_done
-  static constexpr int kMisc = kBar + 16;     // tmem slot, abort flag
-  static constexpr int kBytes = kMisc + 16 + 1024;  // + alignment slack
+// One pass on the tensor cores, no workspace (bf16, d = 128, b = 64, M a multiple of 32): one CTA per
+// (unit, state: keys or values, tile of 32 slots) walks the blocks in order and carries its part of the
+// state, P^T [128 d][32 slots] fp32, in registers (thread e of the carry warps holds row e). Per block j:
+//   C^T[s][t] = w_t[s] prod_{t' > t in the block} a_t'[s]  (products, not log sums: a zero retention
+//               gives an exact 0 either way), D_j[s] = prod_t a_t[s], split into bf16 hi + lo rows;
+//   U_j^T = X_j^T C_j^T  on the tensor cores (M = 128 d, N = 32 slots, K = 64 tokens; X_j, the block's
+//               keys or values, arrives by TMA as an MN-major A operand), hi and lo into one fp32 result;
+//   state j = P (written in the input dtype), then P <- D_j P + U_j.
+// Warp roles, each walking the blocks in order, up to kBufs blocks apart:
+//   warps 0-3  coefficients: warp q takes tokens 16q .. 16q + 15, lane s slot s; C_j and D_j go to
+//              buffer j % kBufs once the carry has released it;
+//   warps 4-7  carry: thread e = TMEM lane e; stores state j, reads U_j, updates P;
+//   warp 8     producer: gates and X of block j into a kStages-deep ring (TMA);
+//   warp 9     MMA issuer: U_j into tensor-memory buffer j % kBufs.
+// The carry is the only sequential chain; the buffers let the coefficients and the MMAs of the next
+// blocks run while it works (two buffers measured 0.441 ms on the 32K workload with 128 slots, four
+// buffers and four stages the figure in the design notes).
+struct CarryPlan {
+  static constexpr int kStages = 4;
+  static constexpr int kBufs = 4;                  // coefficient / U / decay buffers
+  static constexpr int kA = 0;                     // per stage: retention gates [64 tokens][32 slots] fp32
+  static constexpr int kW = 8192;                  //            write gates, same layout
+  static constexpr int kX = 16384;                 //            X [2 d-halves][64 tokens][128 B], 128B swizzle
+  static constexpr int kStage = 32768;
+  static constexpr int kC = kStages * kStage;      // [buffer][hi, lo][32 slots][64 tokens] bf16, K-major
+  static constexpr int kDec = kC + kBufs * 8192;   // [buffer][32] block decays
+  static constexpr int kPart = kDec + kBufs * 32 * 4;  // [4 quarters][32] products of a quarter's retentions
+  static constexpr int kBar = kPart + 4 * 32 * 4;  // full, free [stage]; c_full, u_full, u_free [buffer]; drain
+  static constexpr int kNumBars = 2 * kStages + 3 * kBufs + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kBytes = kMisc + 16 + 1024;   // + alignment slack
+  static constexpr int kThreads = 10 * 32;
 };
 
-__global__ void __launch_bounds__(128) phba_chunk_tc_kernel(const __grid_constant__ CUtensorMap tmKs,
-                                                            const __grid_constant__ CUtensorMap tmV,
-                                                            const float* __restrict__ A, const float* __restrict__ W,
-                                                            float* __restrict__ U, float* __restrict__ Dj,
-                                                            int* status, Geo g) {
+// Named barrier 1 over the four coefficient warps, with an AND over their predicates: a wait's outcome
+// becomes the same for all of them before their next named barrier, so an abort never strands a warp.
+__device__ __forceinline__ bool bar_and_128(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(CarryPlan::kThreads, 1)
+    phba_carry_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                         const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmV,
+                         T* __restrict__ PK, T* __restrict__ PV, int M, int* status, Geo g) {
   using namespace tc;
-  constexpr int M = 128, D = 128, BT = 64;
+  using PL = CarryPlan;
+  constexpr int D = 128, BT = 64, NS = 32, NST = PL::kStages, NB = PL::kBufs;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_align<1024>(smem_raw);
-  uint64_t* bar_x = reinterpret_cast<uint64_t*>(smem + TcPlan::kBar);
-  uint64_t* bar_mma = bar_x + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + TcPlan::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + TcPlan::kMisc + 4);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int j = blockIdx.x, unit = blockIdx.y;
-  const int t0 = j * g.b, n = min(g.b, g.N - t0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
+  uint64_t* bar_full = bars;              // [stage] gates and X landed
+  uint64_t* bar_free = bars + NST;        // [stage] the stage's MMA has run
+  uint64_t* bar_c_full = bars + 2 * NST;  // [buffer] coefficients written (4 warp arrivals)
+  uint64_t* bar_u_full = bar_c_full + NB; // [buffer] U in tensor memory
+  uint64_t* bar_u_free = bar_u_full + NB; // [buffer] the carry has read U and D (4 warp arrivals)
+  uint64_t* bar_drain = bar_u_free + NB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
+  float* sdec = reinterpret_cast<float*>(smem + PL::kDec);
+  float* spart = reinterpret_cast<float*>(smem + PL::kPart);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int which = blockIdx.x & 1, s0 = (blockIdx.x >> 1) * NS, unit = blockIdx.y;
+  const int nb = g.nb;
 
   if (tid == 0) {
-    mbar_init(bar_x, 1);
-    mbar_init(bar_mma, 1);
+    for (int b = 0; b < PL::kNumBars; b++) mbar_init(bars + b, 1);
+    for (int b = 0; b < NB; b++) {
+      mbar_init(bar_c_full + b, 4);
+      mbar_init(bar_u_free + b, 4);
+    }
     fence_mbar_init();
     *abort_flag = 0;
   }
-  __syncthreads();
-  if (tid == 0) {
-    // the block's state keys and values; rows past N arrive as zeros
-    mbar_expect_tx(bar_x, 32768);
-    for (int h = 0; h < 2; h++) {
-      tma_load_3d(smem + TcPlan::kXK + h * 8192, &tmKs, h * 64, t0, unit, bar_x);
-      tma_load_3d(smem + TcPlan::kXV + h * 8192, &tmV, h * 64, t0, unit, bar_x);
-    }
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+  if (warp == 9) {
+    tmem_alloc(tmem_slot, 32 * NB);
     tmem_relinquish();
   }
-  // slot tid's coefficients over the block's tokens, from the log-A suffix sums (tokens past the
-  // block's end get 0), as bf16 hi + lo rows. Every gate is loaded first, so that all the loads are
-  // in flight together; the scan then runs on registers (c takes the write gates' place)
-  {
-    const int s = tid;
-    const float* As = A + ((size_t)unit * g.N + t0) * M + s;
-    const float* Ws = W + ((size_t)unit * g.N + t0) * M + s;
-    float a[BT], c[BT];
-#pragma unroll
-    for (int t = 0; t < BT; t++) {
-      a[t] = t < n ? __ldg(As + (size_t)t * M) : 1.f;
-      c[t] = t < n ? __ldg(Ws + (size_t)t * M) : 0.f;
-    }
-    float r = 0.f;
-#pragma unroll
-    for (int t = BT - 1; t >= 0; t--) {
-      c[t] *= __expf(r);
-      r += __logf(a[t]);
-    }
-    Dj[((size_t)unit * g.nb + j) * M + s] = __expf(r);
-#pragma unroll
-    for (int ch = 0; ch < 8; ch++) {  // 16-byte chunk ch holds tokens 8 ch .. 8 ch + 7
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const float a = c[8 * ch + 2 * q], b = c[8 * ch + 2 * q + 1];
-        const __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b);
-        const __nv_bfloat162 l2 =
-            __floats2bfloat162_rn(a - __bfloat162float(h2.x), b - __bfloat162float(h2.y));
-        hi[q] = *reinterpret_cast<const uint32_t*>(&h2);
-        lo[q] = *reinterpret_cast<const uint32_t*>(&l2);
-      }
-      const int off = s * 128 + ((ch ^ (s & 7)) << 4);
-      *reinterpret_cast<uint4*>(smem + TcPlan::kChi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      *reinterpret_cast<uint4*>(smem + TcPlan::kClo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-    }
-  }
-  fence_proxy_async_smem();  // the coefficient rows are read by the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tD = *tmem_slot;
-  bool issued = false;
-  if (tid == 0) {
-    bool ok = mbar_wait(bar_x, 0, abort_flag);
-    if (ok) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 1);  // A K-major, B MN-major
-      const uint32_t aH = smem_u32(smem + TcPlan::kChi), aL = smem_u32(smem + TcPlan::kClo);
-      const uint32_t bK = smem_u32(smem + TcPlan::kXK), bV = smem_u32(smem + TcPlan::kXV);
+  const uint32_t tU = *tmem_slot;  // U_j^T in columns 32 (j % NB) .. + 31, lane = d
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ coefficients
+    const int q = warp;
+    for (int j = 0; j < nb; j++) {
+      const int st = j % NST, b = j % NB;
+      bool ok = mbar_wait(bar_full + st, (j / NST) & 1, abort_flag);
+      if (ok && j >= NB) ok = mbar_wait(bar_u_free + b, (j / NB - 1) & 1, abort_flag);  // buffer b is free
+      if (!bar_and_128(ok)) break;
+      const float* ga = reinterpret_cast<const float*>(smem + st * PL::kStage + PL::kA);
+      const float* gw = reinterpret_cast<const float*>(smem + st * PL::kStage + PL::kW);
+      const int n = min(BT, g.N - j * BT);  // tokens of the block (the rest arrive as zeros)
+      float c[16];
+      float r = 1.f;
+#pragma unroll
+      for (int t = 15; t >= 0; t--) {
+        const int tt = 16 * q + t;
+        const float a = tt < n ? ga[tt * NS + lane] : 1.f;
+        const float w = tt < n ? gw[tt * NS + lane] : 0.f;
+        c[t] = w * r;
+        r *= a;
+      }
+      spart[q * NS + lane] = r;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      float later = 1.f;  // the retentions of the quarters after this one
+      for (int q2 = q + 1; q2 < 4; q2++) later *= spart[q2 * NS + lane];
+      if (q == 0) sdec[b * NS + lane] = r * later;
+      unsigned char* cb = smem + PL::kC + b * 8192;
+#pragma unroll
+      for (int h = 0; h < 2; h++) {  // 16-byte chunk 2q + h holds tokens 16q + 8h .. + 7
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const float x0 = c[8 * h + 2 * e] * later, x1 = c[8 * h + 2 * e + 1] * later;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x0, x1);
+          const __nv_bfloat162 l2 = __floats2bfloat162_rn(x0 - __bfloat162float(h2.x), x1 - __bfloat162float(h2.y));
+          hi[e] = *reinterpret_cast<const uint32_t*>(&h2);
+          lo[e] = *reinterpret_cast<const uint32_t*>(&l2);
+        }
+        const int off = lane * 128 + (((2 * q + h) ^ (lane & 7)) << 4);
+        *reinterpret_cast<uint4*>(cb + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(cb + 4096 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();  // the coefficient rows are read by the tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_c_full + b);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ carry
+    const int e = tid - 128;  // TMEM lane = row d of the state
+    const uint32_t lane_addr = tU + ((uint32_t)((warp - 4) * 32) << 16);
+    T* out = (which ? PV : PK) + (size_t)unit * nb * M * D + (size_t)s0 * D + e;
+    float P[NS];  // the state rows d = e of the slots s0 .. s0 + 31, before block j
+#pragma unroll
+    for (int k = 0; k < NS; k++) P[k] = 0.f;
+    for (int j = 0; j < nb; j++) {
+      const int b = j % NB;
+      T* row = out + (size_t)j * M * D;
+#pragma unroll
+      for (int k = 0; k < NS; k++) {
+        if constexpr (sizeof(T) == 4) row[(size_t)k * D] = P[k];
+        else row[(size_t)k * D] = __float2bfloat16_rn(P[k]);
+      }
+      // U_j is in tensor memory; the wait on the coefficient barrier makes D_j, which the coefficient
+      // warps wrote before their arrival, visible here
+      bool ok = mbar_wait(bar_u_full + b, (j / NB) & 1, abort_flag);
+      if (ok) ok = mbar_wait(bar_c_full + b, (j / NB) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      float u[NS];
+      tmem_ld32(lane_addr + b * 32, u);
+      tmem_wait_ld();
+      const float* dec = sdec + b * NS;
 #pragma unroll
-      for (int kk = 0; kk < 4; kk++) {  // 16 tokens per step
-        const uint64_t dh = sdesc_sw128(aH + kk * 32, 16, 1024), dl = sdesc_sw128(aL + kk * 32, 16, 1024);
-        const uint64_t dk = sdesc_sw128(bK + kk * 2048, 8192, 1024), dv = sdesc_sw128(bV + kk * 2048, 8192, 1024);
-        umma_bf16(tD, dh, dk, idesc, kk > 0);
-        umma_bf16(tD, dl, dk, idesc, 1);
-        umma_bf16(tD + 128, dh, dv, idesc, kk > 0);
-        umma_bf16(tD + 128, dl, dv, idesc, 1);
+      for (int k = 0; k < NS; k++) P[k] = fmaf(dec[k], P[k], u[k]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_u_free + b);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ producer: gates and X of block j
+    if (lane == 0) {
+      const CUtensorMap* tmX = which ? &tmV : &tmKs;
+      bool ok = true;
+      int j = 0;
+      for (; j < nb && ok; j++) {
+        const int st = j % NST;
+        if (j >= NST) ok = mbar_wait(bar_free + st, (j / NST - 1) & 1, abort_flag);
+        if (!ok) break;
+        unsigned char* sb = smem + st * PL::kStage;
+        mbar_expect_tx(bar_full + st, 32768);
+        tma_load_3d(sb + PL::kA, &tmA, s0, j * BT, unit, bar_full + st);
+        tma_load_3d(sb + PL::kW, &tmW, s0, j * BT, unit, bar_full + st);
+        tma_load_3d(sb + PL::kX, tmX, 0, j * BT, unit, bar_full + st);
+        tma_load_3d(sb + PL::kX + 8192, tmX, 64, j * BT, unit, bar_full + st);
       }
-      umma_commit(bar_mma);
-      issued = true;
-    } else {
+      // drain: the copies of the last (up to) three blocks issued
       volatile int no_abort = 0;
-      mbar_wait(bar_x, 0, &no_abort);  // the copies still land in this CTA's shared memory
+      for (int u = max(0, j - NST); u < j; u++) mbar_wait(bar_full + u % NST, (u / NST) & 1, &no_abort);
     }
-  }
-  issued = __syncthreads_or(issued);
-  bool ok = issued && mbar_wait(bar_mma, 0, abort_flag);
-  ok = __syncthreads_and(ok);
-  if (ok) {
-    tc_fence_after();
-    // thread s holds TMEM lane s: its slot's rows of U_K (columns 0..127) and U_V (128..255)
-    const uint32_t lane_addr = tD + ((uint32_t)(warp * 32) << 16);
-    float* Us = U + ((size_t)unit * g.nb + j) * 2 * M * D;
-    float v[32];
-    for (int which = 0; which < 2; which++) {
-      float* row = Us + ((size_t)which * M + tid) * D;
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        tmem_ld32(lane_addr + which * 128 + c0, v);
-        tmem_wait_ld();
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, NS, 1, 0);  // A = X^T MN-major, B = C^T K-major
+      int issued = 0;
+      for (int j = 0; j < nb; j++) {
+        const int st = j % NST, b = j % NB;
+        bool ok = mbar_wait(bar_c_full + b, (j / NB) & 1, abort_flag);  // implies the carry freed buffer b
+        if (ok) ok = mbar_wait(bar_full + st, (j / NST) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dX = sdesc_sw128(smem_u32(smem + st * PL::kStage + PL::kX), 8192, 1024);
+        const uint64_t dH = sdesc_sw128(smem_u32(smem + PL::kC + b * 8192), 16, 1024);
+        const uint64_t dL = sdesc_sw128(smem_u32(smem + PL::kC + b * 8192 + 4096), 16, 1024);
 #pragma unroll
-        for (int q = 0; q < 8; q++)
-          *reinterpret_cast<float4*>(row + c0 + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int kk = 0; kk < 4; kk++) {  // 16 tokens per step
+          umma_bf16(tU + b * 32, dX + (uint64_t)((kk * 2048) >> 4), dH + (uint64_t)((kk * 32) >> 4), idesc, kk > 0);
+          umma_bf16(tU + b * 32, dX + (uint64_t)((kk * 2048) >> 4), dL + (uint64_t)((kk * 32) >> 4), idesc, 1);
+        }
+        umma_commit(bar_u_full + b);
+        umma_commit(bar_free + st);
+        issued++;
+      }
+      if (issued > 0) {
+        // every MMA issued must finish before tensor memory is freed
+        umma_commit(bar_drain);
+        volatile int no_abort = 0;
+        mbar_wait(bar_drain, 0, &no_abort);
       }
     }
-  } else if (tid == 0 && issued) {
-    // the MMAs may still be in flight after an abort: let them finish before freeing tensor memory
-    umma_commit(bar_mma);
-    volatile int no_abort = 0;
-    mbar_wait(bar_mma, 0, &no_abort);
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && tid == 0) report(status, PYR_ETIMEOUT);
-  if (warp == 0) {
+  if (warp == 9) {
     tc_fence_after();
-    tmem_dealloc(tD, 256);
+    tmem_dealloc(tU, 32 * NB);
   }
 }
 
@@ -296,21 +377,28 @@ cudaError_t launch_t(const Geo& g, int M, const void* Ks, const void* V, const f
   float* U = static_cast<float*>(ws);
   float* Dj = reinterpret_cast<float*>(static_cast<char*>(ws) + L.u_bytes);
   cudaError_t e;
-  if (sizeof(T) == 2 && D == 128 && M == 128 && g.b == 64) {
-    CUtensorMap mk, mv;
-    if (!tc::make_tmap_bf16_3d(&mk, Ks, D, g.N, g.B * g.Hkv) || !tc::make_tmap_bf16_3d(&mv, V, D, g.N, g.B * g.Hkv))
-      return cudaErrorInvalidValue;
-    e = cudaFuncSetAttribute(phba_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TcPlan::kBytes);
-    if (e != cudaSuccess) return e;
-    phba_chunk_tc_kernel<<<dim3(g.nb, g.B * g.Hkv), 128, TcPlan::kBytes, st>>>(mk, mv, A, W, U, Dj, status, g);
-  } else {
-    const size_t smem = sizeof(float) * ((size_t)g.b * kSlotGroup + (size_t)g.b * D);
-    auto ka = phba_chunk_kernel<T, D>;
-    e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ka<<<dim3(g.nb, g.B * g.Hkv), kThreads, smem, st>>>(static_cast<const T*>(Ks), static_cast<const T*>(V), A, W,
-                                                         M, U, Dj, g);
+  if constexpr (sizeof(T) == 2 && D == 128) {
+    if (M % 32 == 0 && g.b == 64) {
+      // one pass, no workspace
+      CUtensorMap ma, mw, mk, mv;
+      if (!tc::make_tmap_f32_3d(&ma, A, M, g.N, g.B * g.Hkv, 32, 64) ||
+          !tc::make_tmap_f32_3d(&mw, W, M, g.N, g.B * g.Hkv, 32, 64) ||
+          !tc::make_tmap_bf16_3d(&mk, Ks, D, g.N, g.B * g.Hkv) || !tc::make_tmap_bf16_3d(&mv, V, D, g.N, g.B * g.Hkv))
+        return cudaErrorInvalidValue;
+      auto kc = phba_carry_tc_kernel<T>;
+      e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CarryPlan::kBytes);
+      if (e != cudaSuccess) return e;
+      kc<<<dim3(2 * (M / 32), g.B * g.Hkv), CarryPlan::kThreads, CarryPlan::kBytes, st>>>(ma, mw, mk, mv, static_cast<T*>(PK),
+                                                                           static_cast<T*>(PV), M, status, g);
+      return cudaGetLastError();
+    }
   }
+  const size_t smem = sizeof(float) * ((size_t)g.b * kSlotGroup + (size_t)g.b * D);
+  auto ka = phba_chunk_kernel<T, D>;
+  e = cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  ka<<<dim3(g.nb, g.B * g.Hkv), kThreads, smem, st>>>(static_cast<const T*>(Ks), static_cast<const T*>(V), A, W,
+                                                       M, U, Dj, g);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   phba_scan_kernel<T, D><<<dim3(ceil_div((int64_t)M * D, kThreads), g.B * g.Hkv), kThreads, 0, st>>>(

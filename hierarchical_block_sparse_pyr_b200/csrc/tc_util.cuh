@@ -212,5 +212,9 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // end read as zeros).
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, int inner, int rows, int heads, int box_rows = 64);
 
+// Host: 3-D TMA map over a [heads][rows][inner] fp32 tensor with a box of box_inner x box_rows x 1 and
+// no swizzle (rows past the end read as zeros).
+bool make_tmap_f32_3d(CUtensorMap* m, const void* base, int inner, int rows, int heads, int box_inner, int box_rows);
+
 }  // namespace tc
 }  // namespace pyr

@@ -257,10 +257,13 @@ PYR_API size_t phba_state_workspace_bytes(const pyr_shape* s, int M);
 
 /*
  * phba_state_build - the prefix states of every key block, computed
- * chunkwise as the summary describes (A.1.1): within each block, log-A sums
- * give every token's decay to the block end and the block's writes become
- * one decay-weighted matrix product; only the block-boundary states are
- * carried from block to block. fp32 arithmetic.
+ * chunkwise as the summary describes (A.1.1): within each block, every
+ * token's decay to the block end (the product of the later retentions; a
+ * log-A sum on the general path, a direct product on the bf16, d = 128,
+ * b = 64, M % 32 == 0 path) weights its write, and the block's writes
+ * become one decay-weighted matrix product; only the block-boundary states
+ * are carried from block to block. fp32 arithmetic. The bf16, d = 128,
+ * b = 64, M % 32 == 0 path does not touch the workspace.
  *   Ks        device, [B][Hkv][N][d] in s->dtype: the state branch's keys (the
  *             pages use un-rotated keys here; pass K when there is no rotation).
  *   V         device, [B][Hkv][N][d] in s->dtype.
