@@ -19,7 +19,12 @@
 //   (A operand in TMEM, at the same lanes as its accumulator); P_B goes to
 //   shared memory (a 128B-swizzled K-major operand) and feeds an SS MMA.
 // Routed attention only: dense attention (every block for both query blocks)
-// keeps the general kernel, whose union is then exactly one block list.
+// keeps the general kernel, whose union is then exactly one block list. With
+// PHBA prefix states (M > 0, a multiple of 64; PHBA summary 3.3 and A.1.3:
+// one softmax over tokens and state slots) each half's state tiles follow its
+// token tiles: every entry j >= 1 of its list brings the M-slot state stored
+// before block j (its own block's state for the diagonal, the aligned state
+// for a routed block) as M / 64 tiles with no mask; block 0 has no state.
 // Warp roles (as in the general kernel): warps 0..3 softmax, one thread per
 // (row of A, row of B) lane pair; warp 4 TMA producer of Q and of the step's
 // K tiles (one per half); warp 5 MMA issuer; warp 6 TMA producer of the step's
@@ -66,10 +71,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+template <bool kStates>  // PHBA state tiles after the token tiles (M > 0)
 __global__ void __launch_bounds__(kThreads, 2)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const int32_t* __restrict__ idx,
-                     __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* status, Geo g) {
+                     __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int* status, Geo g,
+                     const __grid_constant__ CUtensorMap tmPK, const __grid_constant__ CUtensorMap tmPV, int M) {
   using PL = PairPlan;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_align<1024>(smem_raw);
@@ -113,12 +120,27 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tS = tmem;        // S slot sb at column 64 sb; P_A over its first 32 columns
   const uint32_t tO = tmem + 128;  // O at columns 128..255
 
-  // tiles per half: the routed blocks, then the block itself
-  int T[2];
+  // tiles per half: the routed blocks, then the block itself, then (with states) M / 64 tiles of the
+  // state of every listed block j >= 1 (the list is ascending, so only its first entry can be block 0)
+  const int SPB = M / kKeys;
+  int T[2], Ttok[2], sfirst[2];
 #pragma unroll
-  for (int h = 0; h < 2; h++) T[h] = h < nq_here ? lists[4 * kTileListPitch + h] : 0;
+  for (int h = 0; h < 2; h++) {
+    Ttok[h] = h < nq_here ? lists[4 * kTileListPitch + h] : 0;
+    sfirst[h] = (Ttok[h] > 0 && lists[h * kTileListPitch] == 0) ? 1 : 0;
+    T[h] = Ttok[h] + (kStates ? (Ttok[h] - sfirst[h]) * SPB : 0);
+  }
   const int Tmax = max(T[0], T[1]);
-  auto block_of = [&](int h, int k) { return lists[h * kTileListPitch + k]; };
+  // tile k of half h: its first key row (in K / V, or in the [nb * M] state rows) and whether it is a state tile
+  auto tile_of = [&](int h, int k, int* key0) -> bool {
+    if (!kStates || k < Ttok[h]) {
+      *key0 = lists[h * kTileListPitch + k] * kKeys;
+      return false;
+    }
+    const int u = k - Ttok[h], e = sfirst[h] + u / SPB;
+    *key0 = lists[h * kTileListPitch + e] * M + (u % SPB) * kKeys;
+    return true;
+  };
 
   unsigned char* sQ = smem + PL::kQ;
   unsigned char* sK = smem + PL::kK;
@@ -149,9 +171,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_expect_tx(full, nt * 16384);
         for (int h = 0; h < 2; h++) {
           if (k >= T[h]) continue;
-          const int key0 = block_of(h, k) * kKeys;
-          for (int dh = 0; dh < 2; dh++)
-            tma_load_3d(ring + h * 16384 + dh * 8192, map, dh * 64, key0, unit, full);
+          int key0;
+          const bool state = tile_of(h, k, &key0);
+          const CUtensorMap* mp = state ? (is_k ? &tmPK : &tmPV) : map;
+          for (int dh = 0; dh < 2; dh++) tma_load_3d(ring + h * 16384 + dh * 8192, mp, dh * 64, key0, unit, full);
         }
       }
       // drain: wait (bounded) for every copy issued so far before the CTA may exit
@@ -234,12 +257,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     float s[kKeys];
     for (int k = 0; k < Tmax; k++) {
       const int sb = k & 1;
-      // this row's tile at step k: full (routed: every key < N), causal (its own block), or none
-      int md = 0, key0 = 0;
+      // this row's tile at step k: full (routed: every key < N), causal (its own block), state slots (all
+      // of them), or none
+      int md = 0, key0 = 0, lim = 0;
       if (row_ok && k < T[h]) {
-        const int j = block_of(h, k);
-        key0 = j * kKeys;
-        md = j == iq ? 2 : 1;
+        if (tile_of(h, k, &key0)) {
+          md = 1;
+          lim = kKeys;
+        } else {
+          md = key0 == iq * kKeys ? 2 : 1;
+          lim = md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1);
+        }
       }
       ok = warp_wait(bar_s_full + sb, (k >> 1) & 1, abort_flag);
       if (!ok) break;
@@ -247,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_ld32(tS_row + sb * 64, s);
       tmem_ld32(tS_row + sb * 64 + 32, s + 32);
       tmem_wait_ld();
-      const int lim = md == 0 ? 0 : (md == 1 ? min(kKeys, g.N - key0) : min(kKeys, p - key0 + 1));
       if (lim < kKeys) {
 #pragma unroll
         for (int c = 0; c < kKeys; c++) s[c] = c < lim ? s[c] : -INFINITY;
@@ -370,13 +397,14 @@ bool attn_pair_supported(const Geo& g) {
 }
 
 cudaError_t launch_attn_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                             const int32_t* idx, void* O, float* lse, int* status, cudaStream_t st) {
-  auto kern = attn_pair_kernel;
+                             const int32_t* idx, void* O, float* lse, int* status, cudaStream_t st,
+                             const CUtensorMap& mpk, const CUtensorMap& mpv, int M) {
+  auto kern = M > 0 ? attn_pair_kernel<true> : attn_pair_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairPlan::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((g.nqb + 1) / 2, g.B * g.Hkv);
-  kern<<<grid, kThreads, PairPlan::kBytes, st>>>(mq, mk, mv, idx, reinterpret_cast<__nv_bfloat16*>(O), lse,
-                                                 status, g);
+  kern<<<grid, kThreads, PairPlan::kBytes, st>>>(mq, mk, mv, idx, reinterpret_cast<__nv_bfloat16*>(O), lse, status, g,
+                                                 mpk, mpv, M);
   return cudaGetLastError();
 }
 

@@ -448,7 +448,8 @@ cudaError_t launch_cfg(const Geo& g, const CUtensorMap& mq, const CUtensorMap& m
 // two 64-row query blocks of one head per CTA, each over its own block list (attn_pair.cu)
 bool attn_pair_supported(const Geo& g);
 cudaError_t launch_attn_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                             const int32_t* idx, void* O, float* lse, int* status, cudaStream_t st);
+                             const int32_t* idx, void* O, float* lse, int* status, cudaStream_t st,
+                             const CUtensorMap& mpk, const CUtensorMap& mpv, int M);
 
 bool attn_tc_supported(const Geo& g) {
   if (g.dtype != PYR_BF16 || g.d != 128) return false;
@@ -476,7 +477,8 @@ cudaError_t launch_attn_tc(const Geo& g, const void* Q, const void* K, const voi
     mpv = mv;
   }
   const int rows = g.G * g.b;
-  if (!dense && M == 0 && attn_pair_supported(g)) return launch_attn_pair(g, mq, mk, mv, idx, O, lse, status, st);
+  if (!dense && attn_pair_supported(g))
+    return launch_attn_pair(g, mq, mk, mv, idx, O, lse, status, st, mpk, mpv, M);
   if (g.b == 64) {
     if (rows == 64) return launch_cfg<1, 2, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
     if (rows == 128) return launch_cfg<1, 1, 64, 2>(g, mq, mk, mv, idx, dense, O, lse, status, st, mpk, mpv, M);
