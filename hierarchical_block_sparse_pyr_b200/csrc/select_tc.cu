@@ -255,6 +255,9 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
   int nphase = 0;
   int32_t* out = idx + ((size_t)unit * g.nqb + qb) * g.topk;
 
+  // valid candidate slots of the level about to run: every start-level node begins before block i;
+  // below, every kept node's left child does, and the rank step counts the valid right children
+  int n_valid_next = nc;
   for (int l = g.s0; l >= 0 && ok; l--) {
     const bool start = (l == g.s0);
     // this thread's slot (rank phase: slot = tid) and its node; with at most 32 slots (M = 64,
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     constexpr bool kSplit = (MC == 64 && STACK);
     const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
     const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
-    const int n_valid = __syncthreads_count(slot_m >= 0);
+    const int n_valid = n_valid_next;
     // keep count, except at level 0 with the fallback on, where it can grow after scoring
     const int keep_lo = min(l > 0 ? g.cap / 2 : base, n_valid);
     int32_t* trow = o.trace ? sel_trace_row(o, g, unit, qb, l) : nullptr;
@@ -515,12 +518,14 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
       __syncthreads();
       keep = sel_fcf_keep(o, g, base, n_valid, sbr, *s_conf, &decision_margin);
     }
+    bool right_valid = false;
     if (my_rank >= 0) {
       if (my_rank < keep) {
         if (l > 0) {
           const int c1 = 2 * my_node + 1;
+          right_valid = c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i;
           cand[2 * my_rank] = 2 * my_node;
-          cand[2 * my_rank + 1] = (c1 < g.lvl_n[l - 1] && (c1 << (l - 1)) < i) ? c1 : -1;
+          cand[2 * my_rank + 1] = right_valid ? c1 : -1;
           if (rcg) psc[2 * my_rank] = psc[2 * my_rank + 1] = key_score(my_key);
         } else {
           kept[my_rank] = my_node;
@@ -531,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
       if (my_rank == keep) s_edge[1] = key_score(my_key);
     }
     if (trow && tid >= keep && tid < o.tw) trow[tid] = -1;
-    __syncthreads();
+    n_valid_next = keep + __syncthreads_count(right_valid);  // also the barrier before the next level
     if (tid == 0) {
       if (keep < n_valid && keep > 0) {
         const float mg = s_edge[0] - s_edge[1];
