@@ -173,6 +173,15 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
 #pragma unroll
     for (int k = 0; k < kPer; k++) goff[k] = a_chunk_off<MC, NT, STACK>(warp + 4 * k, lane);
   }
+  // separate hi / lo operands (one tile of MC rows): slot c = warp + 4k is row c, so its destination is
+  // a per-thread base + (k / 2) 8-row groups + one of two in-group offsets (row & 7 = warp + 4 (k & 1))
+  int ns_base = 0, ns_par0 = 0, ns_par1 = 0;
+  if (!STACK) {
+    const int q16 = lane & 15, c8 = q16 & 7;
+    ns_base = (lane >= 16 ? C::kAOp : 0) + (q16 >> 3) * (MC * 128);
+    ns_par0 = warp * 128 + ((c8 ^ warp) << 4);
+    ns_par1 = (warp + 4) * 128 + ((c8 ^ (warp + 4)) << 4);
+  }
   // start level s0: every node that begins before block i, node m in slot m
   int nc = min(g.lvl_n[g.s0], (i + (1 << g.s0) - 1) >> g.s0);
   {
@@ -185,10 +194,12 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
         if (c < nc && c != ms) cp_async16(sA + goff[k], src + (size_t)c * 256);
       }
     } else {
-      for (int x = tid; x < nc * 32; x += kThreads) {
-        const int c = x >> 5, q = x & 31;
-        if (c == ms) continue;
-        cp_async16(sA + a_chunk_off<MC, NT, STACK>(c, q), pu + (size_t)(g.lvl_off[g.s0] + c) * 256 + q * 8);
+      const __nv_bfloat16* src = pu + (size_t)g.lvl_off[g.s0] * 256 + lane * 8;
+#pragma unroll 4
+      for (int k = 0; k < MC / 4; k++) {
+        const int c = warp + 4 * k;
+        if (c >= nc) break;
+        if (c != ms) cp_async16(sA + ns_base + (k >> 1) * 1024 + ((k & 1) ? ns_par1 : ns_par0), src + (size_t)c * 256);
       }
     }
   }
@@ -298,15 +309,19 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
             cp_async16(sA + goff[k], src + (size_t)m * 256);
         }
       } else {
-        for (int x = tid; x < nc * 32; x += kThreads) {
-          const int c = x >> 5, q = x & 31;
+        const __nv_bfloat16* src = pu + (size_t)g.lvl_off[l] * 256 + lane * 8;
+        const uint4 strad = *reinterpret_cast<const uint4*>(ppair + l * 512 + lane * 16);
+#pragma unroll 4
+        for (int k = 0; k < MC / 4; k++) {
+          const int c = warp + 4 * k;
+          if (c >= nc) break;
           const int m = cand[c];
           if (m < 0) continue;
-          unsigned char* dst = sA + a_chunk_off<MC, NT, STACK>(c, q);
+          unsigned char* dst = sA + ns_base + (k >> 1) * 1024 + ((k & 1) ? ns_par1 : ns_par0);
           if (m == ms)
-            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ppair + l * 512 + q * 16);
+            *reinterpret_cast<uint4*>(dst) = strad;
           else
-            cp_async16(dst, pu + (size_t)(g.lvl_off[l] + m) * 256 + q * 8);
+            cp_async16(dst, src + (size_t)m * 256);
         }
       }
     }
