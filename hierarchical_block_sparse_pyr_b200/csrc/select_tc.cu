@@ -273,9 +273,11 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     const bool start = (l == g.s0);
     // this thread's slot (rank phase: slot = tid) and its node; with at most 32 slots (M = 64,
     // stacked rows) four threads share slot tid / 4 in the rank count
-    constexpr bool kSplit = (MC == 64 && STACK);
+    // stacked operands hold at most CPT = 32 or 64 slots: TPS = 4 or 2 threads share a slot in the rank
+    constexpr int TPS = STACK ? kThreads / C::CPT : 1;
+    constexpr bool kSplit = TPS > 1;
     const int slot_m = tid < nc ? (start ? tid : cand[tid]) : -1;
-    const int split_m = (kSplit && (tid >> 2) < nc) ? (start ? (tid >> 2) : cand[tid >> 2]) : -1;
+    const int split_m = (kSplit && tid / TPS < nc) ? (start ? tid / TPS : cand[tid / TPS]) : -1;
     const int n_valid = n_valid_next;
     // keep count, except at level 0 with the fallback on, where it can grow after scoring
     const int keep_lo = min(l > 0 ? g.cap / 2 : base, n_valid);
@@ -355,70 +357,76 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     // halves of every 64-column batch with one shuffle each, so that each holds hi + lo for 32
     // columns; each keeps an online max and sum over its columns, and the pair merges at the end
     const bool full = (rb == g.b);
-    if constexpr (kSplit) {
-      // M = 64 stacked rows: the 16-lane TMEM load hands thread t the hi row (lane t/4) and the lo
-      // row (lane t/4 + 8) of candidate warp*H + t/4 at the same two columns of every eight, so
-      // hi + lo is thread-local and four threads split the candidate's query rows
-      const int c = warp * C::H + (lane >> 2);
+    if constexpr (STACK && MC == 64) {
+      // M = 64 stacked rows: an M = 64 accumulator fills lanes 0-15 of each warp's TMEM sub-partition,
+      // 8 candidates' hi rows in lanes 0-7 and their lo rows in lanes 8-15. The 16-lane TMEM load hands
+      // thread t the hi row (lane t/4) and the lo row (lane t/4 + 8) of one candidate at the same two
+      // columns of every eight, so hi + lo is thread-local and four threads split the candidate's query
+      // rows. (The same load over the M = 128 stacked layout, two 16-lane groups per warp with the rows
+      // regrouped to match, measured slower at 64K than the 32-lane load with a shuffle: 1.386 -> 1.457 ms.)
       const int cb = 2 * (lane & 3);
-      float m2 = -INFINITY, s2 = 0.f;
-      if (ntiles > 0 && __any_sync(0xffffffffu, c < nc)) {  // warp-uniform
+      {
+        const int c = warp * C::H + (lane >> 2);
+        const uint32_t grp_addr = my_lane_addr;
+        float m2 = -INFINITY, s2 = 0.f;
+        if (ntiles > 0 && __any_sync(0xffffffffu, c < nc)) {  // warp-uniform
 #pragma unroll 1
-        for (int c0 = 0; c0 < R; c0 += 64) {
-          uint32_t r[32];
-          tmem_ld16x256b_x8(my_lane_addr + c0, r);
-          tmem_wait_ld();
-          float x[16];
-#pragma unroll
-          for (int k = 0; k < 8; k++) {
-            x[2 * k] = __uint_as_float(r[4 * k]) + __uint_as_float(r[4 * k + 2]);
-            x[2 * k + 1] = __uint_as_float(r[4 * k + 1]) + __uint_as_float(r[4 * k + 3]);
-          }
-          if (!full) {
-#pragma unroll
-            for (int k = 0; k < 16; k++) x[k] = ((c0 + 8 * (k >> 1) + cb + (k & 1)) % g.b) < rb ? x[k] : -INFINITY;
-          }
-          float a[6];
-#pragma unroll
-          for (int k = 0; k < 5; k++) a[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
-          a[5] = x[15];
-          const float bm = fmax3(fmax3(a[0], a[1], a[2]), a[3], fmaxf(a[4], a[5])) * sl2;
-          const float mn = fmaxf(m2, bm);
-          if (mn != -INFINITY) {
-            s2 *= ex2(m2 - mn);  // 0 on the first valid batch (m2 = -inf)
-            m2 = mn;
-            const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
-            float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          for (int c0 = 0; c0 < R; c0 += 64) {
+            uint32_t r[32];
+            tmem_ld16x256b_x8(grp_addr + c0, r);
+            tmem_wait_ld();
+            float x[16];
 #pragma unroll
             for (int k = 0; k < 8; k++) {
-              const float2 y = __ffma2_rn(make_float2(x[2 * k], x[2 * k + 1]), scl, off);
-              acc[k & 1] = __fadd2_rn(acc[k & 1], make_float2(ex2(y.x), ex2(y.y)));
+              x[2 * k] = __uint_as_float(r[4 * k]) + __uint_as_float(r[4 * k + 2]);
+              x[2 * k + 1] = __uint_as_float(r[4 * k + 1]) + __uint_as_float(r[4 * k + 3]);
             }
-            const float2 sum = __fadd2_rn(acc[0], acc[1]);
-            s2 += sum.x + sum.y;
+            if (!full) {
+#pragma unroll
+              for (int k = 0; k < 16; k++) x[k] = ((c0 + 8 * (k >> 1) + cb + (k & 1)) % g.b) < rb ? x[k] : -INFINITY;
+            }
+            float a[6];
+#pragma unroll
+            for (int k = 0; k < 5; k++) a[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+            a[5] = x[15];
+            const float bm = fmax3(fmax3(a[0], a[1], a[2]), a[3], fmaxf(a[4], a[5])) * sl2;
+            const float mn = fmaxf(m2, bm);
+            if (mn != -INFINITY) {
+              s2 *= ex2(m2 - mn);  // 0 on the first valid batch (m2 = -inf)
+              m2 = mn;
+              const float2 scl = make_float2(sl2, sl2), off = make_float2(-m2, -m2);
+              float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+              for (int k = 0; k < 8; k++) {
+                const float2 y = __ffma2_rn(make_float2(x[2 * k], x[2 * k + 1]), scl, off);
+                acc[k & 1] = __fadd2_rn(acc[k & 1], make_float2(ex2(y.x), ex2(y.y)));
+              }
+              const float2 sum = __fadd2_rn(acc[0], acc[1]);
+              s2 += sum.x + sum.y;
+            }
           }
         }
-      }
-      // merge the four threads of the candidate
+        // merge the four threads of the candidate
 #pragma unroll
-      for (int sh = 1; sh <= 2; sh <<= 1) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m2, sh), so = __shfl_xor_sync(0xffffffffu, s2, sh);
-        const float M = fmaxf(m2, mo);
-        s2 = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
-        m2 = M;
-      }
-      if ((lane & 3) == 0 && c < nc) {
-        const int m = start ? c : cand[c];
-        unsigned long long key = 0ull;  // empty slots rank below every node
-        if (m >= 0) {
-          const int j0 = m << l;
-          const int j1 = min(min((m + 1) << l, g.nb), i);
-          const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
-          float sc = (m2 + __log2f(s2)) * 0.6931471805599453f + __logf(nval);
-          if (rcg && !start) sc = fmaf(o.rcg_lambda, psc[c], sc);
-          key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
+        for (int sh = 1; sh <= 2; sh <<= 1) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m2, sh), so = __shfl_xor_sync(0xffffffffu, s2, sh);
+          const float M = fmaxf(m2, mo);
+          s2 = (m2 == -INFINITY ? 0.f : s2 * ex2(m2 - M)) + (mo == -INFINITY ? 0.f : so * ex2(mo - M));
+          m2 = M;
         }
-        keys[c] = key;
+        if ((lane & 3) == 0 && c < nc) {
+          const int m = start ? c : cand[c];
+          unsigned long long key = 0ull;  // empty slots rank below every node
+          if (m >= 0) {
+            const int j0 = m << l;
+            const int j1 = min(min((m + 1) << l, g.nb), i);
+            const float nval = (float)(min((int64_t)j1 * g.b, (int64_t)g.N) - (int64_t)j0 * g.b);
+            float sc = (m2 + __log2f(s2)) * 0.6931471805599453f + __logf(nval);
+            if (rcg && !start) sc = fmaf(o.rcg_lambda, psc[c], sc);
+            key = ((unsigned long long)float_order_key(sc) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)m);
+          }
+          keys[c] = key;
+        }
       }
     } else
 #pragma unroll 1
@@ -491,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     }  // scored level
     tc_fence_before();
     const int nc8 = (nc + 7) & ~7;
-    if (tid >= nc && tid < (kSplit ? 32 : nc8)) keys[tid] = 0ull;  // zero pad for the 8-wide reads
+    if (tid >= nc && tid < (kSplit ? C::CPT : nc8)) keys[tid] = 0ull;  // zero pad for the 8-wide reads
     __syncthreads();
     // ---- keep the best: rank = number of strictly larger keys (keys are distinct: they hold the
     // node index); a kept node of rank r puts its children (those that exist and start before
@@ -499,16 +507,20 @@ __global__ void __launch_bounds__(kThreads, SelCfg<MC, NT, STACK>::kMinBlocks)
     int my_rank = -1, my_node = -1;
     unsigned long long my_key = 0ull;
     if (kSplit) {
-      // slot tid / 4: each of its four threads counts the larger keys among 8 of the 32
-      const int sl = tid >> 2, part = tid & 3;
+      // slot tid / TPS: each of its TPS threads counts the larger keys among CPT / TPS of the CPT
+      constexpr int KPP = C::CPT / TPS;
+      const int sl = tid / TPS, part = tid % TPS;
       const unsigned long long k_sl = keys[sl];
-      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys) + part * 4;
-      const ulonglong2 a0 = k2[0], a1 = k2[1], a2 = k2[2], a3 = k2[3];
-      int rank = split_m >= 0 ? (a0.x > k_sl) + (a0.y > k_sl) + (a1.x > k_sl) + (a1.y > k_sl) +
-                                    (a2.x > k_sl) + (a2.y > k_sl) + (a3.x > k_sl) + (a3.y > k_sl)
-                              : 0;
-      rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-      rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+      const ulonglong2* k2 = reinterpret_cast<const ulonglong2*>(keys) + part * (KPP / 2);
+      int rank = 0;
+#pragma unroll
+      for (int u = 0; u < KPP / 2; u++) {
+        const ulonglong2 a = k2[u];
+        rank += (a.x > k_sl) + (a.y > k_sl);
+      }
+      if (split_m < 0) rank = 0;
+#pragma unroll
+      for (int sh = 1; sh < TPS; sh <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, sh);
       if (split_m >= 0 && part == 0) {
         my_rank = rank;
         my_node = split_m;
