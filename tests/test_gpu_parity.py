@@ -55,6 +55,10 @@ CASES = [
               dtype=BF16, seed=31, n_needle=6),
     W0.scaled(name="cap100_separate", B=1, Hq=4, Hkv=2, N=16384, Nq=16384, d=128, b=64, topk=40, cap=100,
               dtype=BF16, seed=32, n_needle=6),
+    # long route lists for the paired-block MHA attention (up to 101 entries per query block) and the
+    # separate hi / lo selection layout
+    W0.scaled(name="mha_topk100", B=1, Hq=2, Hkv=2, N=12288 + 40, Nq=12288 + 40, d=128, b=64, topk=100, cap=128,
+              dtype=BF16, seed=34, n_needle=6),
 ]
 
 

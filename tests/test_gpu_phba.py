@@ -36,6 +36,9 @@ CASES = [
                dtype=BF16, seed=72), 128, False),
     (W0.scaled(name="phba_tc_b128", B=1, Hq=2, Hkv=2, N=4173, Nq=4173, d=128, b=128, topk=4, cap=8, dtype=BF16,
                seed=73), 64, False),
+    # the largest state: eight 32-slot tiles in the one-pass build, four state tiles per block in attention
+    (W0.scaled(name="phba_tc_mha_m256", B=1, Hq=2, Hkv=2, N=2048 + 64 + 17, Nq=2048 + 64 + 17, d=128, b=64, topk=5,
+               cap=10, dtype=BF16, seed=77), 256, False),
     # CUDA-core path: fp32, a separate state query, M not a multiple of 64
     (W0.scaled(name="phba_simt_f32", B=1, Hq=4, Hkv=2, N=1000, Nq=1000, d=64, b=32, topk=5, cap=10, dtype=F32,
                seed=74), 5, True),
