@@ -37,7 +37,8 @@ LIB_PATH = os.path.join(_PKG, "lib", "libpyr.so")
 PYR_OK, PYR_EINVAL, PYR_EUNSUPPORTED, PYR_ECUDA, PYR_ETIMEOUT, PYR_EBADIDX = range(6)
 PYR_F32, PYR_BF16 = 0, 1
 
-ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_pyramid_elems", "pyr_build", "pyr_update",
+ABI_SYMBOLS = ("pyr_num_levels", "pyr_num_nodes", "pyr_num_qblocks", "pyr_pyramid_elems", "pyr_build", "pyr_means",
+               "pyr_update",
                "pyr_select", "pyr_select_ex", "pyr_select_trace_levels", "pyr_select_trace_width", "bsa_forward",
                "dense_forward", "bsa_forward_host", "pyr_host_workspace_bytes", "bsa_route_invert", "bsa_backward",
                "bsa_backward_noalloc", "pyr_selftest_wait", "pyr_strerror", "phba_state_elems",
@@ -80,6 +81,8 @@ def _load_lib():
     lib.pyr_pyramid_elems.restype = ctypes.c_size_t
     lib.pyr_build.argtypes = [sp, vp, vp, vp, vp]
     lib.pyr_build.restype = ctypes.c_int
+    lib.pyr_means.argtypes = [sp, vp, vp, vp, vp]
+    lib.pyr_means.restype = ctypes.c_int
     lib.pyr_update.argtypes = [sp, vp, vp, ctypes.c_int, vp, vp]
     lib.pyr_update.restype = ctypes.c_int
     lib.pyr_select.argtypes = [sp, vp, vp, vp, vp, vp, vp]
@@ -188,6 +191,12 @@ def _check(rc, what):
 def pyr_build(s: PyrShape, K, pyr, status=None, stream=None):
     _check(_L().pyr_build(ctypes.byref(s), _dev(K, "K"), _dev(pyr, "pyr"), _dev(status, "status", True),
                           _stream(stream)), "pyr_build")
+
+
+def pyr_means(s: PyrShape, pyr, means, status=None, stream=None):
+    """fp32 node means [B, Hkv, P, d] (means, written) from a pyramid's (hi, lo) pairs."""
+    _check(_L().pyr_means(ctypes.byref(s), _dev(pyr, "pyr"), _dev(means, "means"), _dev(status, "status", True),
+                          _stream(stream)), "pyr_means")
 
 
 def pyr_update(s: PyrShape, K, pyr, from_pos: int, status=None, stream=None):
@@ -367,10 +376,11 @@ def run_backward(s: PyrShape, Q, K, V, dO, fwd: "Buffers", bwd: BackwardBuffers,
     return bwd
 
 
-def pyramid_means(pyr: torch.Tensor) -> torch.Tensor:
-    """fp32 node means [..., P, d] from the (hi, lo) pair storage [..., P, 2, d]."""
-    p = pyr.float()
-    return p[..., 0, :] + p[..., 1, :]
+def pyramid_means(s: PyrShape, pyr: torch.Tensor, stream=None) -> torch.Tensor:
+    """Allocate and fill the fp32 node means [B, Hkv, P, d] of a pyramid (pyr_means)."""
+    means = torch.empty((s.B, s.Hkv, num_nodes(s), s.d), dtype=torch.float32, device=pyr.device)
+    pyr_means(s, pyr, means, stream=stream)
+    return means
 
 
 def run(s: PyrShape, Q, K, V, buf: Buffers, stream=None, with_gap=True):

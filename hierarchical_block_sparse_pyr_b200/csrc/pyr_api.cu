@@ -136,6 +136,16 @@ int pyr_build(const pyr_shape* s, const void* K, void* pyr, int* dev_status, voi
   return launch_status(pyr::launch_pyramid(g, K, static_cast<__nv_bfloat16*>(pyr), dev_status, (cudaStream_t)stream));
 }
 
+int pyr_means(const pyr_shape* s, const void* pyr, float* means, int* dev_status, void* stream) {
+  Geo g;
+  int rc = make_geo(s, &g);
+  if (rc) return rc;
+  if (!pyr || !means || !aligned16(pyr) || (reinterpret_cast<uintptr_t>(means) & 3)) return PYR_EINVAL;
+  (void)dev_status;
+  return launch_status(
+      pyr::launch_pyramid_means(g, static_cast<const __nv_bfloat16*>(pyr), means, (cudaStream_t)stream));
+}
+
 int pyr_update(const pyr_shape* s, const void* K, void* pyr, int from_pos, int* dev_status, void* stream) {
   Geo g;
   int rc = make_geo(s, &g);

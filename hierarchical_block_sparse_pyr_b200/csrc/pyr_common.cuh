@@ -82,6 +82,8 @@ bool current_context_id(unsigned long long* id);
 cudaError_t launch_pyramid(const Geo& g, const void* K, __nv_bfloat16* pyr, int* status, cudaStream_t st);
 cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* pyr, int from_pos, int* status,
                                   cudaStream_t st);
+// fp32 node means (hi + lo) of a pyramid, [B * Hkv][P][d]
+cudaError_t launch_pyramid_means(const Geo& g, const __nv_bfloat16* pyr, float* means, cudaStream_t st);
 bool attn_decode_supported(const Geo& g);
 bool attn_decode_warp_supported(const Geo& g);  // one warp per 64-key tile, G <= 8
 cudaError_t launch_attn_decode_warp(const Geo& g, const void* Q, const void* K, const void* V, const int32_t* idx,

@@ -16,6 +16,8 @@
 //                     launched as a programmatic dependent of the chunk kernel,
 //                     so its CTAs are resident before the chunk kernel ends and
 //                     wait (griddepcontrol.wait) for the chunk kernel's writes.
+#include <algorithm>
+
 #include "pyr_common.cuh"
 
 namespace pyr {
@@ -274,6 +276,46 @@ cudaError_t launch_pyramid_update(const Geo& g, const void* K, __nv_bfloat16* py
                                                                    j_first);
   else
     pyr_update_kernel<float><<<g.B * g.Hkv, 128, 0, st>>>(reinterpret_cast<const float*>(K), pyr, g, j_first);
+  return cudaGetLastError();
+}
+
+namespace {
+
+// means[n][e] = hi + lo for every node n of every unit: a streaming pass, 8 elements per thread
+__global__ void __launch_bounds__(256) pyr_means_kernel(const __nv_bfloat16* __restrict__ pyr,
+                                                         float* __restrict__ means, int64_t nodes, int d) {
+  const int64_t per_node = d / 8;  // 8-element groups per node
+  const int64_t total = nodes * per_node;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < total; x += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = x / per_node, e8 = (x - n * per_node) * 8;
+    const uint4 hv = *reinterpret_cast<const uint4*>(pyr + (n * 2) * d + e8);
+    const uint4 lv = *reinterpret_cast<const uint4*>(pyr + (n * 2 + 1) * d + e8);
+    const uint32_t h[4] = {hv.x, hv.y, hv.z, hv.w}, lo[4] = {lv.x, lv.y, lv.z, lv.w};
+    float out[8];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      out[2 * k] = __uint_as_float(h[k] << 16) + __uint_as_float(lo[k] << 16);
+      out[2 * k + 1] = __uint_as_float(h[k] & 0xFFFF0000u) + __uint_as_float(lo[k] & 0xFFFF0000u);
+    }
+    float* dst = means + n * d + e8;
+    if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      reinterpret_cast<float4*>(dst)[0] = make_float4(out[0], out[1], out[2], out[3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(out[4], out[5], out[6], out[7]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; k++) dst[k] = out[k];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pyramid_means(const Geo& g, const __nv_bfloat16* pyr, float* means, cudaStream_t st) {
+  const int64_t nodes = (int64_t)g.B * g.Hkv * g.P;
+  const int64_t groups = nodes * (g.d / 8);
+  const int blocks = (int)std::min<int64_t>((groups + 255) / 256, 148 * 16);
+  if (blocks <= 0) return cudaSuccess;
+  pyr_means_kernel<<<blocks, 256, 0, st>>>(pyr, means, nodes, g.d);
   return cudaGetLastError();
 }
 

@@ -123,6 +123,17 @@ PYR_API size_t pyr_pyramid_elems(const pyr_shape* s);
 PYR_API int pyr_build(const pyr_shape* s, const void* K, void* pyr, int* dev_status, void* stream);
 
 /*
+ * pyr_means - the fp32 node means of a pyramid: means[u][n][e] = hi + lo of
+ * node n's pair, for a caller that wants the pyramid as plain fp32 centroids
+ * (PHBA A.1.2) rather than the (hi, lo) storage the walk reads.
+ *   pyr   device, as written by pyr_build / pyr_update for the same shape.
+ *   means device, [B][Hkv][P][d] fp32 (written), 4-byte aligned.
+ * Enqueued on the stream like the other calls; returns PYR_OK or a
+ * host-side error (nothing is written on error).
+ */
+PYR_API int pyr_means(const pyr_shape* s, const void* pyr, float* means, int* dev_status, void* stream);
+
+/*
  * pyr_update - bring a pyramid up to date after the keys at positions
  * >= from_pos (0 <= from_pos < N) were rewritten, with the shape unchanged;
  * for example a decode step that writes its new key into the last slot. Only

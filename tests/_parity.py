@@ -56,7 +56,7 @@ def run_gpu(w, Q, K, V, idx=None, dense=False, opts=None, with_trace=False):
         use = buf.idx if idx is None else torch.as_tensor(np.ascontiguousarray(idx), dtype=torch.int32).cuda()
         P.bsa_forward(s, Qd, Kd, Vd, use, buf.O, buf.lse, buf.status)
     torch.cuda.synchronize()
-    out = dict(pyr=P.pyramid_means(buf.pyr).cpu(), idx=buf.idx.cpu(), gap=buf.gap.cpu(), O=buf.O.float().cpu(),
+    out = dict(pyr=P.pyramid_means(s, buf.pyr).cpu(), idx=buf.idx.cpu(), gap=buf.gap.cpu(), O=buf.O.float().cpu(),
                lse=buf.lse.cpu(), status=int(buf.status.item()))
     if trace is not None:
         out["trace"] = trace.reshape(w.B * w.Hkv, trace.shape[2], trace.shape[3], trace.shape[4]).cpu()

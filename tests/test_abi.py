@@ -87,6 +87,8 @@ def test_host_validation_rejects_null_and_misaligned_pointers():
     assert lib.bsa_forward(ctypes.byref(s), 16, 16, 16, None, 16, None, None, None) == P.PYR_EINVAL
     assert lib.dense_forward(ctypes.byref(s), 16, 16, 16, 8, None, None, None) == P.PYR_EINVAL
     assert lib.pyr_build(None, 16, 16, None, None) == P.PYR_EINVAL
+    assert lib.pyr_means(ctypes.byref(s), None, 16, None, None) == P.PYR_EINVAL  # no pyramid
+    assert lib.pyr_means(ctypes.byref(s), 16, 18, None, None) == P.PYR_EINVAL    # means not 4-byte aligned
     for code in range(6):
         assert isinstance(P.strerror(code), str) and P.strerror(code)
 

@@ -148,8 +148,8 @@ def test_pyr_update_matches_a_rebuild_and_the_oracle(case):
     P.pyr_build(s, Kd, fresh.pyr, fresh.status)
     torch.cuda.synchronize()
     assert int(buf.status.item()) == 0
-    upd = P.pyramid_means(buf.pyr).cpu().double().numpy()
-    reb = P.pyramid_means(fresh.pyr).cpu().double().numpy()
+    upd = P.pyramid_means(s, buf.pyr).cpu().double().numpy()
+    reb = P.pyramid_means(s, fresh.pyr).cpu().double().numpy()
     pyr_o = oracle.pyramid(w, K2, list(range(w.B * w.Hkv)))
     check_pyramid(upd.reshape(pyr_o.shape), pyr_o)
     assert np.abs(upd - reb).max() <= 2e-5 * (1 + np.abs(reb).max())
