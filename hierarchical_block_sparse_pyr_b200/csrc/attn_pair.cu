@@ -26,7 +26,8 @@
 // before block j (its own block's state for the diagonal, the aligned state
 // for a routed block) as M / 64 tiles with no mask; block 0 has no state.
 // Warp roles (as in the general kernel): warps 0..3 softmax, one thread per
-// (row of A, row of B) lane pair; warp 4 TMA producer of Q and of the step's
+// row (lanes 0..15 of warp w: rows 16w .. 16w + 15 of A; lanes 16..31: the
+// same rows of B); warp 4 TMA producer of Q and of the step's
 // K tiles (one per half); warp 5 MMA issuer; warp 6 TMA producer of the step's
 // V tiles. Every mbarrier wait is bounded; a wait that runs out aborts the CTA
 // (PYR_ETIMEOUT), which still drains its copies and MMAs and frees its tensor
