@@ -9,8 +9,9 @@
 // head), TPC threads per candidate (TPC = 128 / cap slots: 2 for cap <= 64,
 // 1 for cap <= 128), each taking d / TPC elements of the node mean from its
 // (hi, lo) pair in fp32 and of all G query rows (held in shared memory,
-// pre-scaled by log2(e) / sqrt(d)). Per level: one pass of 16-byte loads and
-// FMAs, a shuffle between the candidate's threads, the LogSumExp over the G
+// pre-scaled by log2(e) / sqrt(d)). Per level: the thread's 16-byte loads of
+// the candidate's (hi, lo) row, all issued before the first is used (one memory
+// round trip), FMAs, a shuffle between the candidate's threads, the LogSumExp over the G
 // rows, a rank count over packed keys (ties to the lower node index), and
 // the kept node of rank r writes its children to slots 2r, 2r+1. The node
 // that straddles the query block uses the exact mean of its part before the
@@ -124,11 +125,18 @@ __global__ void __launch_bounds__(kThreads) select_decode_kernel(const T* __rest
         const __nv_bfloat16* row = pu + (size_t)(g.lvl_off[l] + m) * 2 * D;
         const uint4* hi4 = reinterpret_cast<const uint4*>(row + e0);
         const uint4* lo4 = reinterpret_cast<const uint4*>(row + D + e0);
-#pragma unroll 2
+        // every 16-byte load of this thread's share first: one memory round trip per level
+        uint4 hv[DPT / 8], lv[DPT / 8];
+#pragma unroll
+        for (int v = 0; v < DPT / 8; v++) {
+          hv[v] = __ldg(hi4 + v);
+          lv[v] = __ldg(lo4 + v);
+        }
+#pragma unroll
         for (int v = 0; v < DPT / 8; v++) {
           float hf[8], lf[8], kv[8];
-          bf16x8_to_f32(hi4[v], hf);
-          bf16x8_to_f32(lo4[v], lf);
+          bf16x8_to_f32(hv[v], hf);
+          bf16x8_to_f32(lv[v], lf);
 #pragma unroll
           for (int k = 0; k < 8; k++) kv[k] = hf[k] + lf[k];
           const int e = e0 + v * 8;
