@@ -679,6 +679,16 @@ cudaError_t launch_dkdv(const Geo& g, const CUtensorMap& mq, const CUtensorMap& 
 
 }  // namespace
 
+// 64-row MHA blocks (backward_pair.cu): products transposed so that one block's own list fills M = 128
+bool backward_pair_supported(const Geo& g);
+cudaError_t launch_backward_dq_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk,
+                                    const CUtensorMap& mv, const CUtensorMap& mdo, const float* lse,
+                                    const float* delta, const int32_t* idx, void* dQ, int* status, cudaStream_t st);
+cudaError_t launch_backward_dkdv_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk,
+                                      const CUtensorMap& mv, const CUtensorMap& mdo, const float* lse,
+                                      const float* delta, const int32_t* offset, const int32_t* rho, void* dK,
+                                      void* dV, int* status, cudaStream_t st);
+
 bool backward_tc_supported(const Geo& g) {
   if (g.dtype != PYR_BF16 || g.d != 128) return false;
   if (g.b != 64 && g.b != 128) return false;
@@ -694,6 +704,8 @@ cudaError_t launch_backward_dq_tc(const Geo& g, const void* Q, const void* K, co
   if (!make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq) || !make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv) ||
       !make_tmap_bf16_3d(&mv, V, g.d, g.N, g.B * g.Hkv) || !make_tmap_bf16_3d(&mdo, dO, g.d, g.Nq, g.B * g.Hq))
     return cudaErrorInvalidValue;
+  if (backward_pair_supported(g))
+    return launch_backward_dq_pair(g, mq, mk, mv, mdo, lse, delta, idx, dQ, status, st);
   const int rows = g.G * g.b;
   if (g.b == 64) {
     if (rows == 64) return launch_dq<2, 64>(g, mq, mk, mv, mdo, lse, delta, idx, dQ, status, st);
@@ -712,6 +724,8 @@ cudaError_t launch_backward_dkdv_tc(const Geo& g, const void* Q, const void* K, 
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq) || !tc::make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv) ||
       !tc::make_tmap_bf16_3d(&mv, V, g.d, g.N, g.B * g.Hkv) || !tc::make_tmap_bf16_3d(&mdo, dO, g.d, g.Nq, g.B * g.Hq))
     return cudaErrorInvalidValue;
+  if (backward_pair_supported(g))
+    return launch_backward_dkdv_pair(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
   if (g.b == 64) return launch_dkdv<64>(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
   return launch_dkdv<128>(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
 }

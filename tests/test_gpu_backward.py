@@ -32,6 +32,9 @@ CASES = [
               seed=43),
     W0.scaled(name="bf16_b128", B=1, Hq=2, Hkv=2, N=2048 + 40, Nq=2048 + 40, d=128, b=128, topk=4, cap=8, dtype=BF16,
               seed=44),
+    # 64-row MHA blocks (the paired-list kernels): ragged tail, odd and even list lengths, two batches
+    W0.scaled(name="bf16_mha_ragged", B=2, Hq=2, Hkv=2, N=2000, Nq=2000, d=128, b=64, topk=7, cap=14, dtype=BF16,
+              seed=46),
     W0.scaled(name="f32_b16_d128", B=1, Hq=2, Hkv=1, N=333, Nq=333, d=128, b=16, topk=5, cap=10, dtype=F32, seed=45),
 ]
 
