@@ -12,7 +12,8 @@
 //                        = total; rho's unused tail = -1
 //   route_scatter_kernel one thread per idx row: pos = --offset[u][j]; after
 //                        it offset[u][j] is the start of j's range
-//   route_sort_kernel    one thread per (unit, key block): insertion sort
+//   route_sort_kernel    one CTA per (key block, unit): rank by counting, or a
+//                        bitmap of the range's query blocks for long ranges
 //
 // Gradients (the SIMT path: fp32 on the CUDA cores, every dtype and shape the
 // library takes). P is recomputed from the saved log-sum-exp as A.1.4 states;
@@ -111,21 +112,62 @@ __global__ void route_scatter_kernel(const int32_t* __restrict__ idx, int32_t* o
   }
 }
 
-__global__ void route_sort_kernel(const int32_t* __restrict__ offset, int32_t* rho, Geo g) {
-  const int64_t n = (int64_t)g.B * g.Hkv * g.nb;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const int u = (int)(e / g.nb), j = (int)(e % g.nb);
-    const int32_t* off = offset + (int64_t)u * (g.nb + 1);
-    int32_t* r = rho + (int64_t)u * g.nqb * g.topk;
-    const int a = off[j], z = off[j + 1];
-    for (int x = a + 1; x < z; x++) {
-      const int v = r[x];
-      int y = x - 1;
-      while (y >= a && r[y] > v) {
-        r[y + 1] = r[y];
-        y--;
-      }
-      r[y + 1] = v;
+// One CTA per (key block j, unit) puts j's range in ascending order. The
+// entries of a range are distinct query blocks (a row routes a block at most
+// once). Up to kSortThreads entries: each thread ranks its entry by counting
+// the smaller ones. Longer ranges: a bitmap over the query blocks, then each
+// thread emits the set bits of its run of words after a block-wide prefix
+// count. Either way the work is linear in the range (plus nqb / 32 words).
+constexpr int kSortThreads = 128;
+
+__global__ void __launch_bounds__(kSortThreads) route_sort_kernel(const int32_t* __restrict__ offset, int32_t* rho,
+                                                                 Geo g) {
+  extern __shared__ uint32_t bits[];  // ceil(nqb / 32) words
+  __shared__ int32_t vals[kSortThreads];
+  __shared__ int warp_tot[kSortThreads / 32];
+  const int u = blockIdx.y, j = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int32_t* off = offset + (int64_t)u * (g.nb + 1);
+  int32_t* r = rho + (int64_t)u * g.nqb * g.topk;
+  const int a = off[j], n = off[j + 1] - a;
+  if (n <= 1) return;
+  if (n <= kSortThreads) {
+    const int v = t < n ? r[a + t] : 0;
+    vals[t] = v;
+    __syncthreads();  // every entry is read before any is written
+    if (t < n) {
+      int rank = 0;
+      for (int k = 0; k < n; k++) rank += vals[k] < v;
+      r[a + rank] = v;
+    }
+    return;
+  }
+  const int words = (g.nqb + 31) >> 5;
+  for (int w = t; w < words; w += kSortThreads) bits[w] = 0;
+  __syncthreads();
+  for (int k = t; k < n; k += kSortThreads) {
+    const int v = r[a + k];
+    atomicOr(&bits[v >> 5], 1u << (v & 31));
+  }
+  __syncthreads();
+  const int per = (words + kSortThreads - 1) / kSortThreads;
+  const int w0 = min(words, t * per), w1 = min(words, w0 + per);
+  int cnt = 0;
+  for (int w = w0; w < w1; w++) cnt += __popc(bits[w]);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int pos = a + incl - cnt;
+  for (int w = 0; w < warp; w++) pos += warp_tot[w];
+  for (int w = w0; w < w1; w++) {
+    uint32_t m = bits[w];
+    while (m) {
+      r[pos++] = (w << 5) + __ffs(m) - 1;
+      m &= m - 1;
     }
   }
 }
@@ -311,7 +353,14 @@ cudaError_t launch_route_invert(const Geo& g, const int32_t* idx, int32_t* offse
   route_count_kernel<<<grid_for(rows, kEntryThreads), kEntryThreads, 0, st>>>(idx, offset, status, g);
   route_scan_kernel<<<g.B * g.Hkv, kScanThreads, 0, st>>>(offset, rho, g);
   route_scatter_kernel<<<grid_for(rows, kEntryThreads), kEntryThreads, 0, st>>>(idx, offset, rho, g);
-  route_sort_kernel<<<grid_for((int64_t)g.B * g.Hkv * g.nb, kEntryThreads), kEntryThreads, 0, st>>>(offset, rho, g);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t bitmap = sizeof(uint32_t) * (size_t)((g.nqb + 31) / 32);
+  if (bitmap > 48 * 1024) {
+    e = cudaFuncSetAttribute(route_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bitmap);
+    if (e != cudaSuccess) return e;
+  }
+  route_sort_kernel<<<dim3(g.nb, g.B * g.Hkv), kSortThreads, bitmap, st>>>(offset, rho, g);
   return cudaGetLastError();
 }
 

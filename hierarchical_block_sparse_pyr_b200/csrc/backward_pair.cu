@@ -8,34 +8,47 @@
 // their lists (the general kernels of backward_tc.cu) pays a full step for
 // every union entry, even where only one half attends it. These kernels put
 // on the M side of every MMA 128 rows that ONE block's own list supplies, two
-// list entries at a time, and transpose the products to match, so no union is
+// list entries per step, and transpose the products to match, so no union is
 // formed:
 //
-// bwd_dq_pair_kernel: one CTA per (query block i, unit). Its key tiles (the
-// accepted routes of row i, ascending, then block i itself) are taken two at a
-// time, 128 keys per step:
+// bwd_dq_pair_kernel, per query block i: its key tiles (the accepted routes of
+// row i, ascending, then block i itself), 128 keys per step:
 //   S^T = K2 Q^T,  dP^T = V2 dO^T      (M = 128 keys, N = 64 rows, K = d)
 //   one thread per key: P^T = exp(S^T / sqrt(d) - lse), dS^T = P^T (dP^T - D),
 //   bf16, written to shared memory over the V tiles (dP^T no longer needs them)
 //   dQ^T += K2^T dS^T                   (M = d, N = 64 rows, K = 128 keys)
 //
-// bwd_dkdv_pair_kernel: one CTA per (key block j, unit). The query blocks that
-// attend j (j itself, causal, then the block-major list offset/rho, all > j)
-// are taken two at a time, 128 rows per step:
+// bwd_dkdv_pair_kernel, per key block j: the query blocks that attend j (j
+// itself, causal, then the block-major list offset/rho, all > j), 128 rows
+// per step:
 //   S = Q2 K^T,  dP = dO2 V^T          (M = 128 rows, N = 64 keys, K = d)
-//   one thread per row: P, then dS = P (dP - D), bf16, through one buffer
+//   one thread per row: P and dS = P (dP - D), bf16, into shared memory
 //   dV^T += dO2^T P,  dK^T += Q2^T dS  (M = d, N = 64 keys, K = 128 rows)
 //
 // An odd list pads its last step with a second copy of its last block whose
 // half is masked to zero (the operands stay finite, so 0 * operand = 0).
 // Operands transposed for the second product are read from the same
-// shared-memory tiles as MN-major descriptors. Each CTA holds 256 tensor-memory
-// columns and at most 112 KB of shared memory, so two CTAs share an SM and
-// one's loads and softmax run under the other's MMAs. Warps 0-3: one thread
-// per tensor-memory lane; warp 4: TMA producer; warp 5: MMA issuer. Every wait
-// is bounded; an abort drains in-flight copies and MMAs and frees tensor
-// memory.
+// shared-memory tiles through MN-major descriptors.
+//
+// Both kernels are persistent, one CTA per SM, and software-pipelined across
+// steps and blocks: two stages of the streamed operands (K2/V2, or Q2/dO2),
+// two stages of the per-block operands, two S/dP buffers and two accumulators
+// in tensor memory (512 columns). Step u's S and dP are issued while step
+// u-1's gradient MMAs wait for its softmax, so the softmax of u-1 runs under
+// the S and dP of u, and a block's epilogue under the next block's steps. dQ
+// CTAs walk query blocks blockIdx.x + k gridDim.x (every list holds at most
+// topk + 1 tiles). dK/dV lists range from one block to every later query
+// block (a block that every query routes to), so dK/dV CTAs take key blocks
+// from an atomic work counter, the long lists first, and the longest list
+// starts at the beginning. Warps 0-3: one thread per tensor-memory lane;
+// warp 4: producer (route lists, TMA); warps 5, 6, 7: MMA issuers of S, dP and
+// the products that consume the softmax. A thread issues one MMA about every
+// 65 cycles (measured), while an N = 64 MMA runs in about 32, so a single
+// issuer would leave the tensor pipe idle half the time. Every wait is
+// bounded; an abort drains in-flight copies and MMAs and frees tensor memory.
 #include <cudaTypedefs.h>
+
+#include <algorithm>
 
 #include "pyr_common.cuh"
 #include "tc_util.cuh"
@@ -52,36 +65,49 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Shared memory is laid out from the dynamic window's start, which the
 // kernels require to be 1024-byte aligned (the 128-byte swizzle atoms are
 // 1024 bytes); they check it and report PYR_EINVAL otherwise.
+// dQ: one persistent CTA per SM walks its query blocks w = blockIdx.x + k gridDim.x.
 struct DqPairPlan {
-  static constexpr int kQ = 0;          // [2 d-halves][64 rows][128 B]
-  static constexpr int kDO = 16384;     // same
-  static constexpr int kK = 32768;      // [2 d-halves][128 keys][128 B]
-  static constexpr int kV = 65536;      // same; dS^T [128 keys][64 rows] bf16 over its first 16 KB
-  static constexpr int kRow = 98304;    // lse * log2(e) [64], D [64] of the block's rows
-  static constexpr int kBar = kRow + 512;
-  static constexpr int kNumBars = 7;
+  static constexpr int kStages = 3;     // K2/V2 stages
+  static constexpr int kQ = 0;          // {Q, dO} of the current block: [2 d-halves][64 rows][128 B] each
+  static constexpr int kKV = 32768;     // kStages x {K2, V2}: [2 d-halves][128 keys][128 B] each;
+                                        //   dS^T [128 keys][64 rows] bf16 over the first 16 KB of V2
+  static constexpr int kRow = kKV + kStages * 65536;  // 2 blocks x {lse * log2(e) [64], D [64]}
+  static constexpr int kInfo = kRow + 1024;           // kStages x StepInfo
+  static constexpr int kBar = kInfo + 64;
+  static constexpr int kNumBars = 25;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag
-  static constexpr int kList = kMisc + 16;          // route compaction scratch
-  static constexpr int kBytes = kList + kTileListScratch * 4;
-  static constexpr int kThreads = 6 * 32;
-  static constexpr int kTmemCols = 256;  // S^T 0..63, dP^T 64..127, dQ^T 128..191
+  static constexpr int kList = kMisc + 16;          // the producer's route list
+  static constexpr int kBytes = kList + kTileListPitch * 4;
+  static constexpr int kThreads = 8 * 32;
+  static constexpr int kTmemCols = 512;  // S^T, dP^T of 2 steps at 128 s (+64); dQ^T of 2 blocks at 256 + 64 b
 };
 
-struct KvPairPlan {
-  static constexpr int kK = 0;        // [2 d-halves][64 keys][128 B]
-  static constexpr int kV = 16384;    // same
-  static constexpr int kQ = 32768;    // [2 d-halves][128 rows][128 B]
-  static constexpr int kDO = 65536;   // same
-  static constexpr int kPS = 98304;   // P, then dS: [128 rows][64 keys] bf16
-  static constexpr int kBar = 114688;
-  static constexpr int kNumBars = 9;
-  static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 16;
-  static constexpr int kThreads = 6 * 32;
-  static constexpr int kTmemCols = 256;  // S 0..63, dP 64..127, dV^T 128..191, dK^T 192..255
+// One step (two blocks on the M side), written by the producer before the step's copies.
+struct StepInfo {
+  int a, b;   // the two blocks: key blocks (dQ) or query blocks (dK, dV)
+  int flags;  // kFirst / kLast (of the query block), kEnd (of the CTA), own / padding tiles
+  int w;      // work item: unit * nqb + query block
 };
-static_assert(2 * (KvPairPlan::kBytes + 1024) <= 228 * 1024, "two dK/dV CTAs per SM");
-static_assert(2 * (DqPairPlan::kBytes + 1024) <= 228 * 1024, "two dQ CTAs per SM");
+constexpr int kFirst = 1, kLast = 2, kEnd = 4, kOwnA = 8, kOwnB = 16, kPadB = 32;
+
+// dK, dV: one persistent CTA per SM takes key blocks from a work counter, long lists first.
+struct KvPairPlan {
+  static constexpr int kKV = 0;        // 2 stages x {K, V}: [2 d-halves][64 keys][128 B] each
+  static constexpr int kQ = 65536;     // 2 stages x {Q2, dO2}: [2 d-halves][128 rows][128 B] each
+  static constexpr int kP = 196608;    // P  [128 rows][64 keys] bf16, MN-major operand
+  static constexpr int kDS = 212992;   // dS [128 rows][64 keys] bf16, MN-major operand
+  static constexpr int kInfo = 229376;  // 2 stages x StepInfo
+  static constexpr int kBar = kInfo + 64;
+  static constexpr int kNumBars = 23;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag, first work item
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kThreads = 8 * 32;
+  static constexpr int kTmemCols = 512;  // S, dP of 2 steps at 128 s (+64); dV^T, dK^T of 2 blocks at 256 + 128 b (+64)
+};
+// Key blocks whose lists hold more query blocks than this are scheduled first.
+constexpr int kLongList = 64;
+static_assert(KvPairPlan::kBytes <= 227 * 1024, "dK/dV shared memory");
+static_assert(DqPairPlan::kBytes <= 227 * 1024, "dQ shared memory");
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const bool ok = mbar_wait(bar, parity, abort_flag);
@@ -114,55 +140,59 @@ __device__ __forceinline__ uint64_t mnmajor(uint32_t base, int kk, uint32_t chun
 
 // ---------------------------------------------------------------------------- dQ
 
-__global__ void __launch_bounds__(DqPairPlan::kThreads, 2)
+__global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
     bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                        const float* __restrict__ lse, const float* __restrict__ delta,
                        const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ dQ, int* status, Geo g) {
   using PL = DqPairPlan;
+  constexpr int NS = PL::kStages;
   extern __shared__ __align__(1024) unsigned char smem[];
   if (smem_u32(smem) & 1023) {
     if (threadIdx.x == 0) report(status, PYR_EINVAL);
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
-  uint64_t* bar_q = bars;         // Q, dO landed (and the rows' lse, D written)
-  uint64_t* bar_kv = bars + 1;    // a step's K and V tiles landed
-  uint64_t* bar_s = bars + 2;     // S^T, dP^T of the step in tensor memory
-  uint64_t* bar_p = bars + 3;     // dS^T of the step written (4 warps)
-  uint64_t* bar_free = bars + 4;  // the step's dQ MMAs done: K, V and dS^T reusable
-  uint64_t* bar_dq = bars + 5;    // every dQ MMA done
-  uint64_t* bar_drain = bars + 6;
+  uint64_t* q_full = bars;              // a block's Q, dO landed
+  uint64_t* q_free = bars + 1;          // the block's last S^T, dP^T MMAs done (2 issuers)
+  uint64_t* row_full = bars + 2;        // [2] a block's lse, D written
+  uint64_t* row_free = bars + 4;        // [2] ... read (4 warps)
+  uint64_t* kv_full = bars + 6;         // [NS] a step's K2, V2 landed, its StepInfo written
+  uint64_t* kv_free = kv_full + NS;     // [NS] the step's dQ MMAs done: K2, V2 and dS^T reusable
+  uint64_t* s_full = kv_free + NS;      // [2] S^T, dP^T of a step in tensor memory (2 issuers)
+  uint64_t* s_free = s_full + 2;        // [2] ... read into registers (4 warps)
+  uint64_t* p_full = s_free + 2;        // [2] dS^T of a step written (4 warps)
+  uint64_t* dq_full = p_full + 2;       // [2] a block's dQ^T complete
+  uint64_t* dq_free = dq_full + 2;      // [2] ... read into registers (4 warps)
+  uint64_t* bar_drain = dq_free + 2;   // [3] each issuer's MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
+  StepInfo* info = reinterpret_cast<StepInfo*>(smem + PL::kInfo);
   int* list = reinterpret_cast<int*>(smem + PL::kList);
-  unsigned char* sQ = smem + PL::kQ;
-  unsigned char* sDO = smem + PL::kDO;
-  unsigned char* sK = smem + PL::kK;
-  unsigned char* sV = smem + PL::kV;
-  float* s_row = reinterpret_cast<float*>(smem + PL::kRow);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.y;  // (batch, kv head) = (batch, query head): one query head per kv head
-  const int iq = g.i0 + blockIdx.x;
-  const int p0 = iq * 64 - g.q_offset;  // first row of the block (q_offset = 0 here)
-  const int rows = min(64, g.Nq - p0);
+  const int total = g.nqb * g.B * g.Hkv;  // work items: (unit, query block)
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    mbar_init(bar_kv, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 4);
-    mbar_init(bar_free, 1);
-    mbar_init(bar_dq, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_free, 2);
+    for (int s = 0; s < 2; s++) {
+      mbar_init(row_full + s, 1);
+      mbar_init(row_free + s, 4);
+      mbar_init(s_full + s, 2);
+      mbar_init(s_free + s, 4);
+      mbar_init(p_full + s, 4);
+      mbar_init(dq_full + s, 1);
+      mbar_init(dq_free + s, 4);
+    }
+    for (int s = 0; s < NS; s++) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_free + s, 1);
+    }
+    for (int k = 0; k < 3; k++) mbar_init(bar_drain + k, 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
-  // the block's key tiles: accepted routes, ascending, then block iq (ends with a CTA barrier)
-  compact_routes(idx + ((size_t)unit * g.nqb + blockIdx.x) * g.topk, g.topk, iq, 1, list, status);
-  const int T = list[4 * kTileListPitch];
-  const int steps = (T + 1) >> 1;
   if (warp == 5) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
@@ -171,72 +201,153 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 64, tDQ = tmem + 128;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
-    for (int e = lane; e < 64; e += 32) {
-      const bool in = e < rows;
-      const size_t row = (size_t)unit * g.Nq + p0 + e;
-      s_row[e] = in ? lse[row] * kLog2e : 0.f;
-      s_row[64 + e] = in ? delta[row] : 0.f;
-    }
-    __syncwarp();
-    if (lane == 0) {
-      mbar_expect_tx(bar_q, 32768);
-      for (int h = 0; h < 2; h++) {
-        tma_load_3d(sQ + h * 8192, &tmQ, h * 64, p0, unit, bar_q);
-        tma_load_3d(sDO + h * 8192, &tmDO, h * 64, p0, unit, bar_q);
+    int u = 0, nq = 0;  // steps and blocks whose copies were issued
+    bool ok = true;
+    for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
+      const int unit = w / g.nqb, iq = g.i0 + w % g.nqb;
+      const int p0 = iq * 64 - g.q_offset, rows = min(64, g.Nq - p0);
+      const int rs = nq & 1;
+      if (nq >= 2) {
+        bool f = true;
+        if (lane == 0) f = mbar_wait(row_free + rs, ((nq >> 1) - 1) & 1, abort_flag);
+        ok = __shfl_sync(0xffffffffu, f, 0);
+        if (!ok) break;
       }
-      int u = 0;
-      for (; u < steps; u++) {
-        if (u > 0 && !mbar_wait(bar_free, (u - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_kv, 65536);
-        for (int c = 0; c < 2; c++) {
-          const int key0 = list[min(2 * u + c, T - 1)] * 64;
-          for (int h = 0; h < 2; h++) {
-            tma_load_3d(sK + h * 16384 + c * 8192, &tmK, h * 64, key0, unit, bar_kv);
-            tma_load_3d(sV + h * 16384 + c * 8192, &tmV, h * 64, key0, unit, bar_kv);
+      // key tiles: accepted routes, ascending, then block iq
+      const int T = compact_route_row(idx + (size_t)w * g.topk, g.topk, iq, list, status);
+      float* s_row = reinterpret_cast<float*>(smem + PL::kRow + rs * 512);
+      for (int e = lane; e < 64; e += 32) {
+        const bool in = e < rows;
+        const size_t row = (size_t)unit * g.Nq + p0 + e;
+        s_row[e] = in ? lse[row] * kLog2e : 0.f;
+        s_row[64 + e] = in ? delta[row] : 0.f;
+      }
+      __syncwarp();
+      const int steps = (T + 1) >> 1;
+      const bool last_w = w + (int)gridDim.x >= total;
+      if (lane == 0) {
+        mbar_arrive(row_full + rs);
+        for (int t = 0; t < steps; t++, u++) {
+          const int s = u % NS;
+          if (u >= NS && !mbar_wait(kv_free + s, ((u / NS) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int ta = 2 * t, tb = 2 * t + 1;
+          StepInfo si;
+          si.a = list[ta];
+          si.b = list[min(tb, T - 1)];
+          si.w = w;
+          si.flags = (t == 0 ? kFirst : 0) | (t == steps - 1 ? kLast : 0) | (t == steps - 1 && last_w ? kEnd : 0) |
+                     (ta == T - 1 ? kOwnA : 0) | (tb == T - 1 ? kOwnB : 0) | (tb >= T ? kPadB : 0);
+          info[s] = si;
+          unsigned char* skv = smem + PL::kKV + s * 65536;
+          mbar_expect_tx(kv_full + s, 65536);
+          for (int c = 0; c < 2; c++) {
+            const int key0 = (c ? si.b : si.a) * 64;
+            for (int h = 0; h < 2; h++) {
+              tma_load_3d(skv + h * 16384 + c * 8192, &tmK, h * 64, key0, unit, kv_full + s);
+              tma_load_3d(skv + 32768 + h * 16384 + c * 8192, &tmV, h * 64, key0, unit, kv_full + s);
+            }
+          }
+          if (t == 0) {
+            // Q, dO after the first step's tiles: the previous block's last S^T, dP^T must be done
+            if (nq >= 1 && !mbar_wait(q_free, (nq - 1) & 1, abort_flag)) {
+              ok = false;
+              u++;
+              break;
+            }
+            mbar_expect_tx(q_full, 32768);
+            for (int h = 0; h < 2; h++) {
+              tma_load_3d(smem + PL::kQ + h * 8192, &tmQ, h * 64, p0, unit, q_full);
+              tma_load_3d(smem + PL::kQ + 16384 + h * 8192, &tmDO, h * 64, p0, unit, q_full);
+            }
+            nq++;
           }
         }
       }
-      // copies still in flight land before the CTA can exit
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      nq = __shfl_sync(0xffffffffu, nq, 0);
+    }
+    // copies still in flight land before the CTA can exit
+    if (lane == 0) {
       volatile int no_abort = 0;
-      mbar_wait(bar_q, 0, &no_abort);
-      if (u > 0) mbar_wait(bar_kv, (u - 1) & 1, &no_abort);
+      for (int v = max(0, u - NS); v < u; v++) mbar_wait(kv_full + (v % NS), (v / NS) & 1, &no_abort);
+      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 5 || warp == 6) {
+    // ------------------------------------------------------------ S^T (warp 5) and dP^T (warp 6) issuers
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // keys x rows, both K-major
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, 64, 1, 1);  // d x rows, both MN-major
-      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
-      int issued = 0;
-      for (int u = 0; u < steps && ok; u++) {
-        ok = mbar_wait(bar_kv, u & 1, abort_flag);
-        if (!ok) break;
+      const bool is_s = warp == 5;
+      const uint32_t a0 = smem_u32(smem), aB = a0 + PL::kQ + (is_s ? 0 : 16384);  // Q or dO
+      int issued = 0, u = 0, n = 0;
+      while (true) {
+        const int s = u % NS;
+        if (!mbar_wait(kv_full + s, (u / NS) & 1, abort_flag)) break;
+        const int flags = info[s].flags;
+        if ((flags & kFirst) && !mbar_wait(q_full, n & 1, abort_flag)) break;
+        if (u >= 2 && !mbar_wait(s_free + (u & 1), ((u >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
+        const uint32_t aA = a0 + PL::kKV + s * 65536 + (is_s ? 0 : 32768);  // K2 or V2
+        const uint32_t tD = tmem + (u & 1) * 128 + (is_s ? 0 : 64);
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++) umma_bf16(tS, kmajor(aK, kk, 16384), kmajor(aQ, kk, 8192), idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++) umma_bf16(tP, kmajor(aV, kk, 16384), kmajor(aDO, kk, 8192), idesc_s, kk > 0);
-        umma_commit(bar_s);
+        for (int kk = 0; kk < 8; kk++) umma_bf16(tD, kmajor(aA, kk, 16384), kmajor(aB, kk, 8192), idesc_s, kk > 0);
+        umma_commit(s_full + (u & 1));
         issued++;
-        ok = mbar_wait(bar_p, u & 1, abort_flag);
-        if (!ok) break;
+        if (flags & kLast) {
+          umma_commit(q_free);
+          n++;
+        }
+        if (flags & kEnd) break;
+        u++;
+      }
+      if (issued > 0) {
+        umma_commit(bar_drain + warp - 5);
+        volatile int no_abort = 0;
+        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 7) {
+    // ------------------------------------------------------------ dQ issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_q = idesc_bf16_f32(128, 64, 1, 1);  // d x rows, both MN-major
+      const uint32_t a0 = smem_u32(smem);
+      int issued = 0, u = 0, n = 0;
+      while (true) {
+        const int s = u % NS, b = n & 1;
+        // the step's StepInfo (its stage is refilled only after this thread's kv_free commit)
+        if (!mbar_wait(kv_full + s, (u / NS) & 1, abort_flag)) break;
+        const int flags = info[s].flags;
+        if (!mbar_wait(p_full + (u & 1), (u >> 1) & 1, abort_flag)) break;
+        if ((flags & kFirst) && n >= 2 && !mbar_wait(dq_free + b, ((n >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
+        // dQ^T of the block += K2^T dS^T of the step
+        const uint32_t aK = a0 + PL::kKV + s * 65536, aDS = aK + 32768;
+        const uint32_t tDQ = tmem + 256 + b * 64;
 #pragma unroll
         for (int kk = 0; kk < 8; kk++)
-          umma_bf16(tDQ, mnmajor(aK, kk, 16384), mnmajor(aV, kk, 8192), idesc_q, (u > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar_free);
+          umma_bf16(tDQ, mnmajor(aK, kk, 16384), mnmajor(aDS, kk, 8192), idesc_q,
+                    ((flags & kFirst) && kk == 0) ? 0u : 1u);
+        umma_commit(kv_free + s);
+        issued++;
+        if (flags & kLast) {
+          umma_commit(dq_full + b);
+          n++;
+        }
+        if (flags & kEnd) break;
+        u++;
       }
-      if (ok) umma_commit(bar_dq);
       if (issued > 0) {
-        umma_commit(bar_drain);
+        umma_commit(bar_drain + 2);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain, 0, &no_abort);
+        mbar_wait(bar_drain + 2, 0, &no_abort);
       }
     }
     __syncwarp();
@@ -245,32 +356,41 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 2)
     const int r = warp * 32 + lane;  // key r % 64 of the step's tile r / 64
     const int half = r >> 6, kr = r & 63;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sl2 = rsqrtf((float)g.d) * kLog2e;
-    bool ok = warp_wait(bar_q, 0, abort_flag);  // the rows' lse and D
-    for (int u = 0; u < steps && ok; u++) {
-      const int t = 2 * u + half;
-      const int x = list[min(t, T - 1)] * 64 + kr;  // this thread's key position
-      // rows that attend the key: [c_lo, c_hi); none in a padding half or past the keys;
-      // in block iq itself (the last tile) only rows at or after the key
-      const int c_lo = t == T - 1 ? kr : 0;
-      const int c_hi = (t < T && x < g.N) ? rows : 0;
-      ok = warp_wait(bar_s, u & 1, abort_flag);
-      if (!ok) break;
+    const float sl2 = rsqrtf((float)g.d) * kLog2e, scale = rsqrtf((float)g.d);
+    int u = 0, n = 0;
+    while (true) {
+      const int s = u % NS, b = n & 1;
+      if (!warp_wait(kv_full + s, (u / NS) & 1, abort_flag)) break;  // the step's StepInfo
+      const StepInfo si = info[s];
+      if ((si.flags & kFirst) && !warp_wait(row_full + b, (n >> 1) & 1, abort_flag)) break;  // lse, D
+      if (!warp_wait(s_full + (u & 1), (u >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      float s[64], dp[64];
-      tmem_ld32(tS + lane_base, s);
-      tmem_ld32(tS + lane_base + 32, s + 32);
-      tmem_ld32(tP + lane_base, dp);
-      tmem_ld32(tP + lane_base + 32, dp + 32);
+      float sv[64], dp[64];
+      const uint32_t tS = tmem + (u & 1) * 128 + lane_base;
+      tmem_ld32(tS, sv);
+      tmem_ld32(tS + 32, sv + 32);
+      tmem_ld32(tS + 64, dp);
+      tmem_ld32(tS + 96, dp + 32);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free + (u & 1));
+      const int unit = si.w / g.nqb;
+      const int p0 = (g.i0 + si.w % g.nqb) * 64 - g.q_offset, rows = min(64, g.Nq - p0);
+      const int x = (half ? si.b : si.a) * 64 + kr;  // this thread's key position
+      // rows that attend the key: [c_lo, c_hi); none in a padding half or past the keys; in
+      // the block's own tile only rows at or after the key
+      const int c_lo = (si.flags & (half ? kOwnB : kOwnA)) ? kr : 0;
+      const int c_hi = ((half && (si.flags & kPadB)) || x >= g.N) ? 0 : rows;
+      const float* s_row = reinterpret_cast<const float*>(smem + PL::kRow + b * 512);
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 64; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(s_row + c);
         const float4 d4 = *reinterpret_cast<const float4*>(s_row + 64 + c);
-        const float2 y0 = __ffma2_rn(make_float2(s[c], s[c + 1]), make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
+        const float2 y0 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
         const float2 y1 =
-            __ffma2_rn(make_float2(s[c + 2], s[c + 3]), make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
+            __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), make_float2(sl2, sl2), make_float2(-l4.z, -l4.w));
         const float e0 = (c >= c_lo && c < c_hi) ? ex2(y0.x) : 0.f;
         const float e1 = (c + 1 >= c_lo && c + 1 < c_hi) ? ex2(y0.y) : 0.f;
         const float e2 = (c + 2 >= c_lo && c + 2 < c_hi) ? ex2(y1.x) : 0.f;
@@ -278,26 +398,32 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 2)
         pk[c / 2] = pack_bf16(e0 * (dp[c] - d4.x), e1 * (dp[c + 1] - d4.y));
         pk[c / 2 + 1] = pack_bf16(e2 * (dp[c + 2] - d4.z), e3 * (dp[c + 3] - d4.w));
       }
-      // dS^T over the V tiles: the step's dP^T MMAs (committed with bar_s) have read them
-      store_row_sw128(sV, r, pk);
+      // dS^T over the V tiles: the step's dP^T MMAs (committed with s_full) have read them
+      store_row_sw128(smem + PL::kKV + s * 65536 + 32768, r, pk);
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p);
-    }
-    if (ok) ok = warp_wait(bar_dq, 0, abort_flag);
-    if (ok) {
-      tc_fence_after();
-      float o[64];
-      tmem_ld32(tDQ + lane_base, o);
-      tmem_ld32(tDQ + lane_base + 32, o + 32);
-      tmem_wait_ld();
-      const float scale = rsqrtf((float)g.d);
-      // lane r of dQ^T is feature r: column c is row p0 + c
-      __nv_bfloat16* dst = dQ + ((size_t)unit * g.Nq + p0) * 128 + r;
+      if (lane == 0) mbar_arrive(p_full + (u & 1));
+      if (si.flags & kLast) {
+        if (lane == 0) mbar_arrive(row_free + b);  // the block's lse and D are read
+        if (!warp_wait(dq_full + b, (n >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        float o[64];
+        const uint32_t tDQ = tmem + 256 + b * 64 + lane_base;
+        tmem_ld32(tDQ, o);
+        tmem_ld32(tDQ + 32, o + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dq_free + b);
+        // lane r of dQ^T is feature r: column c is row p0 + c
+        __nv_bfloat16* dst = dQ + ((size_t)unit * g.Nq + p0) * 128 + r;
 #pragma unroll
-      for (int c = 0; c < 64; c++)
-        if (c < rows) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
+        for (int c = 0; c < 64; c++)
+          if (c < rows) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
+        n++;
+      }
+      if (si.flags & kEnd) break;
+      u++;
     }
   }
 
@@ -313,12 +439,38 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 2)
 
 // ---------------------------------------------------------------------------- dK, dV
 
-__global__ void __launch_bounds__(KvPairPlan::kThreads, 2)
+// Work order of the dK/dV kernel: items (unit * nb + key block) whose list is
+// longer than kLongList go to `list` first (any order: each item's result does
+// not depend on when it runs); ctr[0] counts them, ctr[1] is the work counter.
+__global__ void bwd_long_items_kernel(const int32_t* __restrict__ offset, int* ctr, int* list, Geo g) {
+  const int total = g.nb * g.B * g.Hkv;
+  for (int w = blockIdx.x * blockDim.x + threadIdx.x; w < total; w += gridDim.x * blockDim.x) {
+    const int32_t* off = offset + (size_t)(w / g.nb) * (g.nb + 1) + w % g.nb;
+    if (off[1] - off[0] + 1 > kLongList) list[atomicAdd(ctr, 1)] = w;
+  }
+}
+
+// The next work item of the calling CTA, or -1: long items first, then the
+// others in index order.
+__device__ __forceinline__ int grab_item(int* ctr, const int* list, const int32_t* __restrict__ offset, const Geo& g) {
+  const int total = g.nb * g.B * g.Hkv, nlong = ctr[0];
+  for (;;) {
+    const int t = atomicAdd(ctr + 1, 1);
+    if (t < nlong) return list[t];
+    const int w = t - nlong;
+    if (w >= total) return -1;
+    const int32_t* off = offset + (size_t)(w / g.nb) * (g.nb + 1) + w % g.nb;
+    if (off[1] - off[0] + 1 <= kLongList) return w;
+  }
+}
+
+__global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
     bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                          const float* __restrict__ lse, const float* __restrict__ delta,
-                         const int32_t* __restrict__ offset, const int32_t* __restrict__ rho,
-                         __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV, int* status, Geo g) {
+                         const int32_t* __restrict__ offset, const int32_t* __restrict__ rho, int* ctr,
+                         const int* long_list, __nv_bfloat16* __restrict__ dK, __nv_bfloat16* __restrict__ dV,
+                         int* status, Geo g) {
   using PL = KvPairPlan;
   extern __shared__ __align__(1024) unsigned char smem[];
   if (smem_u32(smem) & 1023) {
@@ -326,46 +478,45 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 2)
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
-  uint64_t* bar_kv = bars;        // the block's K and V landed
-  uint64_t* bar_ld = bars + 1;    // a step's Q2, dO2 landed
-  uint64_t* bar_s = bars + 2;     // S, dP of the step in tensor memory
-  uint64_t* bar_p = bars + 3;     // P written (4 warps)
-  uint64_t* bar_pv = bars + 4;    // the step's dV MMAs done: the buffer takes dS
-  uint64_t* bar_ds = bars + 5;    // dS written (4 warps)
-  uint64_t* bar_free = bars + 6;  // the step's dK MMAs done: Q2, dO2 and the buffer reusable
-  uint64_t* bar_done = bars + 7;  // every MMA done
-  uint64_t* bar_drain = bars + 8;
+  uint64_t* kv_full = bars;        // [2] a key block's K, V landed
+  uint64_t* kv_free = bars + 2;    // [2] its last S, dP MMAs done (2 issuers)
+  uint64_t* ld_full = bars + 4;    // [2] a step's Q2, dO2 landed, its StepInfo written
+  uint64_t* ld_free = bars + 6;    // [2] the step's dK MMAs done: Q2, dO2 reusable
+  uint64_t* s_full = bars + 8;     // [2] S, dP of a step in tensor memory (2 issuers)
+  uint64_t* s_free = bars + 10;    // [2] ... read into registers (4 warps)
+  uint64_t* acc_full = bars + 12;  // [2] a key block's dV^T, dK^T complete
+  uint64_t* acc_free = bars + 14;  // [2] ... read into registers (4 warps)
+  uint64_t* p_full = bars + 16;    // P written (4 warps)
+  uint64_t* p_free = bars + 17;    // the dV MMAs that read P done
+  uint64_t* ds_full = bars + 18;   // dS written (4 warps)
+  uint64_t* ds_free = bars + 19;   // the dK MMAs that read dS done
+  uint64_t* bar_drain = bars + 20;  // [3] each issuer's MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
-  unsigned char* sK = smem + PL::kK;
-  unsigned char* sV = smem + PL::kV;
-  unsigned char* sQ = smem + PL::kQ;
-  unsigned char* sDO = smem + PL::kDO;
-  unsigned char* sPS = smem + PL::kPS;
+  int* first_item = reinterpret_cast<int*>(smem + PL::kMisc + 8);
+  StepInfo* info = reinterpret_cast<StepInfo*>(smem + PL::kInfo);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.y;
-  const int j = blockIdx.x;  // key block
-  const int x0 = j * 64;
-  // query blocks attending j: j itself (entry 0), then rho[offset[j] ..) (all > j, ascending)
-  const int32_t* off_u = offset + (size_t)unit * (g.nb + 1);
-  const int32_t* vis = rho + (size_t)unit * g.nqb * g.topk + off_u[j];
-  const int T = 1 + off_u[j + 1] - off_u[j];
-  const int steps = (T + 1) >> 1;
-  auto qblock = [&](int t) { return t == 0 ? j : vis[t - 1]; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_kv, 1);
-    mbar_init(bar_ld, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 4);
-    mbar_init(bar_pv, 1);
-    mbar_init(bar_ds, 4);
-    mbar_init(bar_free, 1);
-    mbar_init(bar_done, 1);
-    mbar_init(bar_drain, 1);
+    for (int s = 0; s < 2; s++) {
+      mbar_init(kv_full + s, 1);
+      mbar_init(kv_free + s, 2);
+      mbar_init(ld_full + s, 1);
+      mbar_init(ld_free + s, 1);
+      mbar_init(s_full + s, 2);
+      mbar_init(s_free + s, 4);
+      mbar_init(acc_full + s, 1);
+      mbar_init(acc_free + s, 4);
+    }
+    mbar_init(p_full, 4);
+    mbar_init(p_free, 1);
+    mbar_init(ds_full, 4);
+    mbar_init(ds_free, 1);
+    for (int k = 0; k < 3; k++) mbar_init(bar_drain + k, 1);
     fence_mbar_init();
     *abort_flag = 0;
+    *first_item = grab_item(ctr, long_list, offset, g);
   }
   if (warp == 5) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
@@ -375,139 +526,218 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tP = tmem + 64, tDV = tmem + 128, tDK = tmem + 192;
+  const bool has_work = *first_item >= 0;
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_expect_tx(bar_kv, 32768);
-      for (int h = 0; h < 2; h++) {
-        tma_load_3d(sK + h * 8192, &tmK, h * 64, x0, unit, bar_kv);
-        tma_load_3d(sV + h * 8192, &tmV, h * 64, x0, unit, bar_kv);
-      }
-      int u = 0;
-      for (; u < steps; u++) {
-        if (u > 0 && !mbar_wait(bar_free, (u - 1) & 1, abort_flag)) break;
-        mbar_expect_tx(bar_ld, 65536);
-        for (int c = 0; c < 2; c++) {
-          const int row0 = qblock(min(2 * u + c, T - 1)) * 64;
-          for (int h = 0; h < 2; h++) {
-            tma_load_3d(sQ + h * 16384 + c * 8192, &tmQ, h * 64, row0, unit, bar_ld);
-            tma_load_3d(sDO + h * 16384 + c * 8192, &tmDO, h * 64, row0, unit, bar_ld);
+      int u = 0, n = 0;  // steps and key blocks whose copies were issued
+      bool ok = true;
+      int item = *first_item;
+      while (item >= 0 && ok) {
+        const int next = grab_item(ctr, long_list, offset, g);
+        const int unit = item / g.nb, j = item % g.nb;
+        const int32_t* off = offset + (size_t)unit * (g.nb + 1) + j;
+        const int32_t* vis = rho + (size_t)unit * g.nqb * g.topk + off[0];
+        const int T = 1 + off[1] - off[0];  // j itself, then the query blocks that route to j
+        const int ks = n & 1;
+        if (n >= 2 && !(ok = mbar_wait(kv_free + ks, ((n >> 1) - 1) & 1, abort_flag))) break;
+        unsigned char* skv = smem + PL::kKV + ks * 32768;
+        mbar_expect_tx(kv_full + ks, 32768);
+        for (int h = 0; h < 2; h++) {
+          tma_load_3d(skv + h * 8192, &tmK, h * 64, j * 64, unit, kv_full + ks);
+          tma_load_3d(skv + 16384 + h * 8192, &tmV, h * 64, j * 64, unit, kv_full + ks);
+        }
+        n++;
+        const int steps = (T + 1) >> 1;
+        for (int t = 0; t < steps; t++, u++) {
+          const int s = u & 1;
+          if (u >= 2 && !(ok = mbar_wait(ld_free + s, ((u >> 1) - 1) & 1, abort_flag))) break;
+          const int ta = 2 * t, tb = 2 * t + 1;
+          StepInfo si;
+          si.a = ta == 0 ? j : vis[ta - 1];
+          si.b = tb < T ? vis[tb - 1] : si.a;
+          si.w = item;
+          si.flags = (t == 0 ? kFirst : 0) | (t == steps - 1 ? kLast : 0) | (t == steps - 1 && next < 0 ? kEnd : 0) |
+                     (ta == 0 ? kOwnA : 0) | (tb >= T ? kPadB : 0);
+          info[s] = si;
+          unsigned char* sq = smem + PL::kQ + s * 65536;
+          mbar_expect_tx(ld_full + s, 65536);
+          for (int c = 0; c < 2; c++) {
+            const int row0 = (c ? si.b : si.a) * 64;
+            for (int h = 0; h < 2; h++) {
+              tma_load_3d(sq + h * 16384 + c * 8192, &tmQ, h * 64, row0, unit, ld_full + s);
+              tma_load_3d(sq + 32768 + h * 16384 + c * 8192, &tmDO, h * 64, row0, unit, ld_full + s);
+            }
           }
         }
+        item = next;
       }
+      // copies still in flight land before the CTA can exit
       volatile int no_abort = 0;
-      mbar_wait(bar_kv, 0, &no_abort);
-      if (u > 0) mbar_wait(bar_ld, (u - 1) & 1, &no_abort);
+      for (int v = max(0, u - 2); v < u; v++) mbar_wait(ld_full + (v & 1), (v >> 1) & 1, &no_abort);
+      for (int m = max(0, n - 2); m < n; m++) mbar_wait(kv_full + (m & 1), (m >> 1) & 1, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == 5 || warp == 6) {
+    // ------------------------------------------------------------ S (warp 5) and dP (warp 6) issuers
+    if (lane == 0 && has_work) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // rows x keys, both K-major
-      constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, 1, 1);  // d x keys, both MN-major
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO);
-      const uint32_t aPS = smem_u32(sPS);
-      bool ok = mbar_wait(bar_kv, 0, abort_flag);
-      int issued = 0;
-      for (int u = 0; u < steps && ok; u++) {
-        ok = mbar_wait(bar_ld, u & 1, abort_flag);
-        if (!ok) break;
+      const bool is_s = warp == 5;
+      const uint32_t a0 = smem_u32(smem);
+      int issued = 0, u = 0, n = 0;
+      while (true) {
+        const int s = u & 1, ks = n & 1;
+        if (!mbar_wait(ld_full + s, (u >> 1) & 1, abort_flag)) break;
+        const int flags = info[s].flags;
+        if ((flags & kFirst) && !mbar_wait(kv_full + ks, (n >> 1) & 1, abort_flag)) break;
+        if (u >= 2 && !mbar_wait(s_free + s, ((u >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
+        const uint32_t aA = a0 + PL::kQ + s * 65536 + (is_s ? 0 : 32768);   // Q2 or dO2
+        const uint32_t aB = a0 + PL::kKV + ks * 32768 + (is_s ? 0 : 16384);  // K or V
+        const uint32_t tD = tmem + s * 128 + (is_s ? 0 : 64);
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++) umma_bf16(tS, kmajor(aQ, kk, 16384), kmajor(aK, kk, 8192), idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++) umma_bf16(tP, kmajor(aDO, kk, 16384), kmajor(aV, kk, 8192), idesc_s, kk > 0);
-        umma_commit(bar_s);
+        for (int kk = 0; kk < 8; kk++) umma_bf16(tD, kmajor(aA, kk, 16384), kmajor(aB, kk, 8192), idesc_s, kk > 0);
+        umma_commit(s_full + s);
         issued++;
-        ok = mbar_wait(bar_p, u & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          umma_bf16(tDV, mnmajor(aDO, kk, 16384), mnmajor(aPS, kk, 8192), idesc_g, (u > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar_pv);
-        ok = mbar_wait(bar_ds, u & 1, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          umma_bf16(tDK, mnmajor(aQ, kk, 16384), mnmajor(aPS, kk, 8192), idesc_g, (u > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar_free);
+        if (flags & kLast) {
+          umma_commit(kv_free + ks);
+          n++;
+        }
+        if (flags & kEnd) break;
+        u++;
       }
-      if (ok) umma_commit(bar_done);
       if (issued > 0) {
-        umma_commit(bar_drain);
+        umma_commit(bar_drain + warp - 5);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain, 0, &no_abort);
+        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp == 7) {
+    // ------------------------------------------------------------ dV, dK issuer
+    if (lane == 0 && has_work) {
+      constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, 1, 1);  // d x keys, both MN-major
+      const uint32_t a0 = smem_u32(smem);
+      int issued = 0, u = 0, n = 0;
+      while (true) {
+        const int s = u & 1, b = n & 1;
+        // the step's StepInfo (its stage is refilled only after this thread's ld_free commit)
+        if (!mbar_wait(ld_full + s, (u >> 1) & 1, abort_flag)) break;
+        const int flags = info[s].flags;
+        if (!mbar_wait(p_full, u & 1, abort_flag)) break;
+        if ((flags & kFirst) && n >= 2 && !mbar_wait(acc_free + b, ((n >> 1) - 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        // dV^T, dK^T of the key block += dO2^T P, Q2^T dS of the step
+        const uint32_t aQ = a0 + PL::kQ + s * 65536, aDO = aQ + 32768;
+        const uint32_t tDV = tmem + 256 + b * 128, tDK = tDV + 64;
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)
+          umma_bf16(tDV, mnmajor(aDO, kk, 16384), mnmajor(a0 + PL::kP, kk, 8192), idesc_g,
+                    ((flags & kFirst) && kk == 0) ? 0u : 1u);
+        umma_commit(p_free);
+        if (!mbar_wait(ds_full, u & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++)
+          umma_bf16(tDK, mnmajor(aQ, kk, 16384), mnmajor(a0 + PL::kDS, kk, 8192), idesc_g,
+                    ((flags & kFirst) && kk == 0) ? 0u : 1u);
+        umma_commit(ds_free);
+        // Q2, dO2 reusable: this step's S and dP were complete before its softmax wrote P
+        umma_commit(ld_free + s);
+        issued++;
+        if (flags & kLast) {
+          umma_commit(acc_full + b);
+          n++;
+        }
+        if (flags & kEnd) break;
+        u++;
+      }
+      if (issued > 0) {
+        umma_commit(bar_drain + 2);
+        volatile int no_abort = 0;
+        mbar_wait(bar_drain + 2, 0, &no_abort);
+      }
+    }
+    __syncwarp();
+  } else if (has_work) {
     // ------------------------------------------------------------ one thread per row (lane)
     const int r = warp * 32 + lane;  // row r % 64 of the step's query block r / 64
     const int half = r >> 6, rr = r & 63;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sl2 = rsqrtf((float)g.d) * kLog2e;
-    const int keys = min(64, g.N - x0);
-    bool ok = true;
-    for (int u = 0; u < steps && ok; u++) {
-      const int t = 2 * u + half;
-      const int p = qblock(min(t, T - 1)) * 64 + rr;  // this thread's row position
-      const bool in = t < T && p < g.Nq;
-      // keys the row attends: [0, c_hi); in block j itself (entry 0) only keys up to the row
-      const int c_hi = in ? (t == 0 ? min(keys, rr + 1) : keys) : 0;
+    const float sl2 = rsqrtf((float)g.d) * kLog2e, scale = rsqrtf((float)g.d);
+    int u = 0, n = 0;
+    while (true) {
+      const int s = u & 1, b = n & 1;
+      if (!warp_wait(ld_full + s, (u >> 1) & 1, abort_flag)) break;  // the step's StepInfo
+      const StepInfo si = info[s];
+      const int unit = si.w / g.nb, x0 = (si.w % g.nb) * 64, keys = min(64, g.N - x0);
+      const int p = (half ? si.b : si.a) * 64 + rr;  // this thread's row position
+      // keys the row attends: [0, c_hi); none in a padding half or past the rows; in the key
+      // block's own query block only keys up to the row
+      const bool in = !(half && (si.flags & kPadB)) && p < g.Nq;
+      const int c_hi = in ? ((!half && (si.flags & kOwnA)) ? min(keys, rr + 1) : keys) : 0;
       const size_t row = (size_t)unit * g.Nq + min(p, g.Nq - 1);
       const float lse2 = lse[row] * kLog2e, D = delta[row];
-      ok = warp_wait(bar_s, u & 1, abort_flag);
-      if (!ok) break;
+      if (!warp_wait(s_full + s, (u >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      float s[64], dp[64];
-      tmem_ld32(tS + lane_base, s);
-      tmem_ld32(tS + lane_base + 32, s + 32);
-      tmem_ld32(tP + lane_base, dp);
-      tmem_ld32(tP + lane_base + 32, dp + 32);
+      float sv[64], dp[64];
+      const uint32_t tS = tmem + s * 128 + lane_base;
+      tmem_ld32(tS, sv);
+      tmem_ld32(tS + 32, sv + 32);
+      tmem_ld32(tS + 64, dp);
+      tmem_ld32(tS + 96, dp + 32);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free + s);
       uint32_t pk[32], dk[32];
       const float2 scl = make_float2(sl2, sl2), offs = make_float2(-lse2, -lse2), dd = make_float2(-D, -D);
 #pragma unroll
       for (int c = 0; c < 32; c++) {
-        const float2 y = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), scl, offs);
+        const float2 y = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), scl, offs);
         const float e0 = 2 * c < c_hi ? ex2(y.x) : 0.f, e1 = 2 * c + 1 < c_hi ? ex2(y.y) : 0.f;
         const float2 z = __fadd2_rn(make_float2(dp[2 * c], dp[2 * c + 1]), dd);
         pk[c] = pack_bf16(e0, e1);
         dk[c] = pack_bf16(e0 * z.x, e1 * z.y);
       }
-      // the buffer is free: bar_s was committed after the previous step's dK MMAs
-      store_row_sw128(sPS, r, pk);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p);
-      ok = warp_wait(bar_pv, u & 1, abort_flag);  // dV has read P
-      if (!ok) break;
-      store_row_sw128(sPS, r, dk);
+      if (u >= 1 && !warp_wait(p_free, (u - 1) & 1, abort_flag)) break;  // the previous dV MMAs read P
+      store_row_sw128(smem + PL::kP, r, pk);
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_ds);
-    }
-    if (ok) ok = warp_wait(bar_done, 0, abort_flag);
-    if (ok) {
-      tc_fence_after();
-      const float scale = rsqrtf((float)g.d);
-      float o[64];
-      for (int which = 0; which < 2; which++) {
-        tmem_ld32((which ? tDK : tDV) + lane_base, o);
-        tmem_ld32((which ? tDK : tDV) + lane_base + 32, o + 32);
-        tmem_wait_ld();
-        const float sc = which ? scale : 1.f;
+      if (lane == 0) mbar_arrive(p_full);
+      if (u >= 1 && !warp_wait(ds_free, (u - 1) & 1, abort_flag)) break;  // the previous dK MMAs read dS
+      store_row_sw128(smem + PL::kDS, r, dk);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ds_full);
+      if (si.flags & kLast) {
+        if (!warp_wait(acc_full + b, (n >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
         // lane r of dV^T / dK^T is feature r: column c is key x0 + c
-        __nv_bfloat16* dst = (which ? dK : dV) + ((size_t)unit * g.N + x0) * 128 + r;
+        const uint32_t tDV = tmem + 256 + b * 128 + lane_base;
+        float o[64];
+        tmem_ld32(tDV, o);
+        tmem_ld32(tDV + 32, o + 32);
+        tmem_wait_ld();
+        __nv_bfloat16* dst = dV + ((size_t)unit * g.N + x0) * 128 + r;
 #pragma unroll
         for (int c = 0; c < 64; c++)
-          if (c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * sc);
+          if (c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c]);
+        tmem_ld32(tDV + 64, o);
+        tmem_ld32(tDV + 96, o + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_free + b);
+        dst = dK + ((size_t)unit * g.N + x0) * 128 + r;
+#pragma unroll
+        for (int c = 0; c < 64; c++)
+          if (c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
+        n++;
       }
+      if (si.flags & kEnd) break;
+      u++;
     }
   }
 
@@ -533,8 +763,11 @@ cudaError_t launch_backward_dq_pair(const Geo& g, const CUtensorMap& mq, const C
   cudaError_t e = cudaFuncSetAttribute(bwd_dq_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DqPairPlan::kBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(g.nqb, g.B * g.Hkv);
-  bwd_dq_pair_kernel<<<grid, DqPairPlan::kThreads, DqPairPlan::kBytes, st>>>(
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int total = g.nqb * g.B * g.Hkv;  // persistent: one CTA per SM walks its share of the query blocks
+  bwd_dq_pair_kernel<<<std::min(total, sms), DqPairPlan::kThreads, DqPairPlan::kBytes, st>>>(
       mq, mk, mv, mdo, lse, delta, idx, reinterpret_cast<__nv_bfloat16*>(dQ), status, g);
   return cudaGetLastError();
 }
@@ -542,13 +775,22 @@ cudaError_t launch_backward_dq_pair(const Geo& g, const CUtensorMap& mq, const C
 cudaError_t launch_backward_dkdv_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk,
                                       const CUtensorMap& mv, const CUtensorMap& mdo, const float* lse,
                                       const float* delta, const int32_t* offset, const int32_t* rho, void* dK,
-                                      void* dV, int* status, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       KvPairPlan::kBytes);
+                                      void* dV, void* scratch, int* status, cudaStream_t st) {
+  // scratch (>= 8 + 4 * items bytes, free until this kernel ends): the work counters, then the long items
+  int* ctr = static_cast<int*>(scratch);
+  int* list = ctr + 2;
+  const int total = g.nb * g.B * g.Hkv;
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 2 * sizeof(int), st);
   if (e != cudaSuccess) return e;
-  dim3 grid(g.nb, g.B * g.Hkv);
-  bwd_dkdv_pair_kernel<<<grid, KvPairPlan::kThreads, KvPairPlan::kBytes, st>>>(
-      mq, mk, mv, mdo, lse, delta, offset, rho, reinterpret_cast<__nv_bfloat16*>(dK),
+  bwd_long_items_kernel<<<std::min((total + 255) / 256, 1024), 256, 0, st>>>(offset, ctr, list, g);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_dkdv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, KvPairPlan::kBytes);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  bwd_dkdv_pair_kernel<<<std::min(total, sms), KvPairPlan::kThreads, KvPairPlan::kBytes, st>>>(
+      mq, mk, mv, mdo, lse, delta, offset, rho, ctr, list, reinterpret_cast<__nv_bfloat16*>(dK),
       reinterpret_cast<__nv_bfloat16*>(dV), status, g);
   return cudaGetLastError();
 }

@@ -687,7 +687,7 @@ cudaError_t launch_backward_dq_pair(const Geo& g, const CUtensorMap& mq, const C
 cudaError_t launch_backward_dkdv_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk,
                                       const CUtensorMap& mv, const CUtensorMap& mdo, const float* lse,
                                       const float* delta, const int32_t* offset, const int32_t* rho, void* dK,
-                                      void* dV, int* status, cudaStream_t st);
+                                      void* dV, void* scratch, int* status, cudaStream_t st);
 
 bool backward_tc_supported(const Geo& g) {
   if (g.dtype != PYR_BF16 || g.d != 128) return false;
@@ -719,13 +719,13 @@ cudaError_t launch_backward_dq_tc(const Geo& g, const void* Q, const void* K, co
 namespace pyr {
 cudaError_t launch_backward_dkdv_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
                                     const float* lse, const float* delta, const int32_t* offset, const int32_t* rho,
-                                    void* dK, void* dV, int* status, cudaStream_t st) {
+                                    void* dK, void* dV, void* scratch, int* status, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mdo;
   if (!tc::make_tmap_bf16_3d(&mq, Q, g.d, g.Nq, g.B * g.Hq) || !tc::make_tmap_bf16_3d(&mk, K, g.d, g.N, g.B * g.Hkv) ||
       !tc::make_tmap_bf16_3d(&mv, V, g.d, g.N, g.B * g.Hkv) || !tc::make_tmap_bf16_3d(&mdo, dO, g.d, g.Nq, g.B * g.Hq))
     return cudaErrorInvalidValue;
   if (backward_pair_supported(g))
-    return launch_backward_dkdv_pair(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
+    return launch_backward_dkdv_pair(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, scratch, status, st);
   if (g.b == 64) return launch_dkdv<64>(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
   return launch_dkdv<128>(g, mq, mk, mv, mdo, lse, delta, offset, rho, dK, dV, status, st);
 }

@@ -306,9 +306,10 @@ int bsa_backward(const pyr_shape* s, const void* Q, const void* K, const void* V
   if (pyr::backward_tc_supported(g)) {
     cudaError_t e = pyr::launch_backward_simt(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV,
                                               pyr::kBwdDelta, st);
-    if (e == cudaSuccess) e = pyr::launch_backward_dq_tc(g, Q, K, V, dO, lse, delta, idx, dQ, dev_status, st);
+    // dK, dV first: until the dQ kernel writes it, dQ serves the dK/dV kernel as its work-list scratch
     if (e == cudaSuccess)
-      e = pyr::launch_backward_dkdv_tc(g, Q, K, V, dO, lse, delta, offset, rho, dK, dV, dev_status, st);
+      e = pyr::launch_backward_dkdv_tc(g, Q, K, V, dO, lse, delta, offset, rho, dK, dV, dQ, dev_status, st);
+    if (e == cudaSuccess) e = pyr::launch_backward_dq_tc(g, Q, K, V, dO, lse, delta, idx, dQ, dev_status, st);
     return launch_status(e);
   }
   return launch_status(pyr::launch_backward_simt(g, Q, K, V, O, lse, dO, idx, offset, rho, delta, dQ, dK, dV,

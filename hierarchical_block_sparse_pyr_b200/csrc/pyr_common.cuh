@@ -113,9 +113,11 @@ cudaError_t launch_backward_simt(const Geo& g, const void* Q, const void* K, con
                                  const int32_t* rho, float* delta, void* dQ, void* dK, void* dV, int parts,
                                  cudaStream_t st);
 bool backward_tc_supported(const Geo& g);
+// scratch: device memory of at least 8 + 4 * B * Hkv * nb bytes that no other operand uses and that
+// nothing reads until this launch ends (bsa_backward passes dQ, written afterwards)
 cudaError_t launch_backward_dkdv_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
                                     const float* lse, const float* delta, const int32_t* offset, const int32_t* rho,
-                                    void* dK, void* dV, int* status, cudaStream_t st);
+                                    void* dK, void* dV, void* scratch, int* status, cudaStream_t st);
 cudaError_t launch_backward_dq_tc(const Geo& g, const void* Q, const void* K, const void* V, const void* dO,
                                   const float* lse, const float* delta, const int32_t* idx, void* dQ, int* status,
                                   cudaStream_t st);

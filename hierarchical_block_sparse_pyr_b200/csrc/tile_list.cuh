@@ -33,6 +33,36 @@ __device__ __forceinline__ int lower_bound_smem(const int* a, int n, int v) {
   return lo;
 }
 
+// Warp-level compaction of one idx row (query block iq, in slot order, by the
+// rule above) into L: the accepted routes, ascending, then iq itself. Returns
+// the length on every lane; L is complete (and visible to the warp) on return.
+__device__ inline int compact_route_row(const int32_t* __restrict__ row, int topk, int iq, int* L, int* status) {
+  const int lane = threadIdx.x & 31;
+  int base = 0, pmax = -1;
+  for (int k0 = 0; k0 < topk; k0 += 32) {
+    const int k = k0 + lane;
+    const int j = k < topk ? row[k] : -1;
+    const bool in_range = j >= 0 && j < iq;
+    int incl = in_range ? j : -1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl = max(incl, y);
+    }
+    int before = __shfl_up_sync(0xffffffffu, incl, 1);
+    before = max(lane == 0 ? -1 : before, pmax);
+    const bool acc = in_range && j > before;
+    if (j >= 0 && !acc) report(status, PYR_EBADIDX);
+    const unsigned m = __ballot_sync(0xffffffffu, acc);
+    if (acc) L[base + __popc(m & ((1u << lane) - 1u))] = j;
+    base += __popc(m);
+    pmax = max(pmax, __shfl_sync(0xffffffffu, incl, 31));
+  }
+  if (lane == 0) L[base] = iq;
+  __syncwarp();
+  return base + 1;
+}
+
 // Compaction of the routes of nq (1..2) consecutive query blocks, one warp per
 // block: list q (at scratch + q * kTileListPitch) holds row q's accepted routes,
 // ascending, then the block's own index; its length is at
@@ -41,36 +71,10 @@ __device__ __forceinline__ int lower_bound_smem(const int* a, int n, int v) {
 __device__ inline void compact_routes(const int32_t* __restrict__ rows, int topk, int i_first, int nq, int* scratch,
                                       int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int* cnt = scratch + 4 * kTileListPitch;
   if (warp < nq) {
-    // compact the accepted routes of row `warp`, then append its own block
-    const int iq = i_first + warp;
-    const int32_t* row = rows + (size_t)warp * topk;
-    int* L = scratch + warp * kTileListPitch;
-    int base = 0, pmax = -1;
-    for (int k0 = 0; k0 < topk; k0 += 32) {
-      const int k = k0 + lane;
-      const int j = k < topk ? row[k] : -1;
-      const bool in_range = j >= 0 && j < iq;
-      int incl = in_range ? j : -1;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl = max(incl, y);
-      }
-      int before = __shfl_up_sync(0xffffffffu, incl, 1);
-      before = max(lane == 0 ? -1 : before, pmax);
-      const bool acc = in_range && j > before;
-      if (j >= 0 && !acc) report(status, PYR_EBADIDX);
-      const unsigned m = __ballot_sync(0xffffffffu, acc);
-      if (acc) L[base + __popc(m & ((1u << lane) - 1u))] = j;
-      base += __popc(m);
-      pmax = max(pmax, __shfl_sync(0xffffffffu, incl, 31));
-    }
-    if (lane == 0) {
-      L[base] = iq;
-      cnt[warp] = base + 1;
-    }
+    const int n = compact_route_row(rows + (size_t)warp * topk, topk, i_first + warp,
+                                    scratch + warp * kTileListPitch, status);
+    if (lane == 0) scratch[4 * kTileListPitch + warp] = n;
   }
   __syncthreads();
 }
