@@ -41,9 +41,9 @@
 // block (a block that every query routes to), so dK/dV CTAs take key blocks
 // from an atomic work counter, the long lists first, and the longest list
 // starts at the beginning. Warps 0-3: one thread per tensor-memory lane;
-// warp 4: producer (route lists, TMA); warps 5, 6, 7: MMA issuers of S, dP and
-// the products that consume the softmax. A thread issues one MMA about every
-// 65 cycles (measured), while an N = 64 MMA runs in about 32, so a single
+// warp 4: producer (route lists, TMA); warps 5, 6, 7: MMA issuers (dQ: S, dP,
+// dQ; dK/dV: S and dP, dV, dK). A thread issues one MMA about every 65
+// cycles (measured), while an N = 64 MMA runs in about 32, so a single
 // issuer would leave the tensor pipe idle half the time. Every wait is
 // bounded; an abort drains in-flight copies and MMAs and frees tensor memory.
 #include <cudaTypedefs.h>
@@ -98,7 +98,7 @@ struct KvPairPlan {
   static constexpr int kDS = 212992;   // dS [128 rows][64 keys] bf16, MN-major operand
   static constexpr int kInfo = 229376;  // 2 stages x StepInfo
   static constexpr int kBar = kInfo + 64;
-  static constexpr int kNumBars = 23;
+  static constexpr int kNumBars = 24;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag, first work item
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kThreads = 8 * 32;
@@ -206,9 +206,27 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
     // ------------------------------------------------------------ producer
     int u = 0, nq = 0;  // steps and blocks whose copies were issued
     bool ok = true;
+    // a block's idx row and its rows' lse and D, loaded one block ahead into registers
+    int nidx[4];
+    float nl[2], nd[2];
+    auto fetch = [&](int w) {
+      if (w >= total) return;
+      const int32_t* row = idx + (size_t)w * g.topk;
+#pragma unroll
+      for (int c = 0; c < 4; c++) nidx[c] = 32 * c + lane < g.topk ? row[32 * c + lane] : -1;
+      const int unit = w / g.nqb, p0 = (g.i0 + w % g.nqb) * 64 - g.q_offset, rows = min(64, g.Nq - p0);
+#pragma unroll
+      for (int h = 0; h < 2; h++) {
+        const int e = lane + 32 * h;
+        const size_t r = (size_t)unit * g.Nq + p0 + min(e, rows - 1);
+        nl[h] = e < rows ? lse[r] * kLog2e : 0.f;
+        nd[h] = e < rows ? delta[r] : 0.f;
+      }
+    };
+    fetch(blockIdx.x);
     for (int w = blockIdx.x; w < total && ok; w += gridDim.x) {
       const int unit = w / g.nqb, iq = g.i0 + w % g.nqb;
-      const int p0 = iq * 64 - g.q_offset, rows = min(64, g.Nq - p0);
+      const int p0 = iq * 64 - g.q_offset;
       const int rs = nq & 1;
       if (nq >= 2) {
         bool f = true;
@@ -217,15 +235,14 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
         if (!ok) break;
       }
       // key tiles: accepted routes, ascending, then block iq
-      const int T = compact_route_row(idx + (size_t)w * g.topk, g.topk, iq, list, status);
+      const int T = compact_route_row_with([&](int c) { return nidx[c]; }, g.topk, iq, list, status);
       float* s_row = reinterpret_cast<float*>(smem + PL::kRow + rs * 512);
-      for (int e = lane; e < 64; e += 32) {
-        const bool in = e < rows;
-        const size_t row = (size_t)unit * g.Nq + p0 + e;
-        s_row[e] = in ? lse[row] * kLog2e : 0.f;
-        s_row[64 + e] = in ? delta[row] : 0.f;
-      }
+      s_row[lane] = nl[0];
+      s_row[lane + 32] = nl[1];
+      s_row[64 + lane] = nd[0];
+      s_row[96 + lane] = nd[1];
       __syncwarp();
+      fetch(w + (int)gridDim.x);  // in flight while this block's copies are issued
       const int steps = (T + 1) >> 1;
       const bool last_w = w + (int)gridDim.x >= total;
       if (lane == 0) {
@@ -479,12 +496,12 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PL::kBar);
   uint64_t* kv_full = bars;        // [2] a key block's K, V landed
-  uint64_t* kv_free = bars + 2;    // [2] its last S, dP MMAs done (2 issuers)
+  uint64_t* kv_free = bars + 2;    // [2] its last S, dP MMAs done
   uint64_t* ld_full = bars + 4;    // [2] a step's Q2, dO2 landed, its StepInfo written
-  uint64_t* ld_free = bars + 6;    // [2] the step's dK MMAs done: Q2, dO2 reusable
-  uint64_t* s_full = bars + 8;     // [2] S, dP of a step in tensor memory (2 issuers)
+  uint64_t* ld_free = bars + 6;    // [2] the step's dV and dK MMAs done (2 issuers): Q2, dO2 reusable
+  uint64_t* s_full = bars + 8;     // [2] S, dP of a step in tensor memory
   uint64_t* s_free = bars + 10;    // [2] ... read into registers (4 warps)
-  uint64_t* acc_full = bars + 12;  // [2] a key block's dV^T, dK^T complete
+  uint64_t* acc_full = bars + 12;  // [2] a key block's dV^T, dK^T complete (2 issuers)
   uint64_t* acc_free = bars + 14;  // [2] ... read into registers (4 warps)
   uint64_t* p_full = bars + 16;    // P written (4 warps)
   uint64_t* p_free = bars + 17;    // the dV MMAs that read P done
@@ -501,12 +518,12 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; s++) {
       mbar_init(kv_full + s, 1);
-      mbar_init(kv_free + s, 2);
+      mbar_init(kv_free + s, 1);
       mbar_init(ld_full + s, 1);
-      mbar_init(ld_free + s, 1);
-      mbar_init(s_full + s, 2);
+      mbar_init(ld_free + s, 2);
+      mbar_init(s_full + s, 1);
       mbar_init(s_free + s, 4);
-      mbar_init(acc_full + s, 1);
+      mbar_init(acc_full + s, 2);
       mbar_init(acc_free + s, 4);
     }
     mbar_init(p_full, 4);
@@ -579,11 +596,10 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
       for (int m = max(0, n - 2); m < n; m++) mbar_wait(kv_full + (m & 1), (m >> 1) & 1, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5 || warp == 6) {
-    // ------------------------------------------------------------ S (warp 5) and dP (warp 6) issuers
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ S, dP issuer
     if (lane == 0 && has_work) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // rows x keys, both K-major
-      const bool is_s = warp == 5;
       const uint32_t a0 = smem_u32(smem);
       int issued = 0, u = 0, n = 0;
       while (true) {
@@ -593,11 +609,13 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
         if ((flags & kFirst) && !mbar_wait(kv_full + ks, (n >> 1) & 1, abort_flag)) break;
         if (u >= 2 && !mbar_wait(s_free + s, ((u >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t aA = a0 + PL::kQ + s * 65536 + (is_s ? 0 : 32768);   // Q2 or dO2
-        const uint32_t aB = a0 + PL::kKV + ks * 32768 + (is_s ? 0 : 16384);  // K or V
-        const uint32_t tD = tmem + s * 128 + (is_s ? 0 : 64);
+        const uint32_t aQ = a0 + PL::kQ + s * 65536, aDO = aQ + 32768;
+        const uint32_t aK = a0 + PL::kKV + ks * 32768, aV = aK + 16384;
+        const uint32_t tS = tmem + s * 128, tP = tS + 64;
 #pragma unroll
-        for (int kk = 0; kk < 8; kk++) umma_bf16(tD, kmajor(aA, kk, 16384), kmajor(aB, kk, 8192), idesc_s, kk > 0);
+        for (int kk = 0; kk < 8; kk++) umma_bf16(tS, kmajor(aQ, kk, 16384), kmajor(aK, kk, 8192), idesc_s, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; kk++) umma_bf16(tP, kmajor(aDO, kk, 16384), kmajor(aV, kk, 8192), idesc_s, kk > 0);
         umma_commit(s_full + s);
         issued++;
         if (flags & kLast) {
@@ -608,42 +626,38 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
         u++;
       }
       if (issued > 0) {
-        umma_commit(bar_drain + warp - 5);
+        umma_commit(bar_drain);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
+        mbar_wait(bar_drain, 0, &no_abort);
       }
     }
     __syncwarp();
-  } else if (warp == 7) {
-    // ------------------------------------------------------------ dV, dK issuer
+  } else if (warp == 6 || warp == 7) {
+    // ------------------------------------------------------------ dV (warp 6) and dK (warp 7) issuers
     if (lane == 0 && has_work) {
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, 1, 1);  // d x keys, both MN-major
-      const uint32_t a0 = smem_u32(smem);
+      const bool is_v = warp == 6;
+      uint64_t* in_full = is_v ? p_full : ds_full;    // P or dS written
+      uint64_t* in_free = is_v ? p_free : ds_free;    // ... read by this issuer's MMAs
+      const uint32_t a0 = smem_u32(smem), aB = a0 + (is_v ? PL::kP : PL::kDS);
       int issued = 0, u = 0, n = 0;
       while (true) {
         const int s = u & 1, b = n & 1;
         // the step's StepInfo (its stage is refilled only after this thread's ld_free commit)
         if (!mbar_wait(ld_full + s, (u >> 1) & 1, abort_flag)) break;
         const int flags = info[s].flags;
-        if (!mbar_wait(p_full, u & 1, abort_flag)) break;
+        if (!mbar_wait(in_full, u & 1, abort_flag)) break;
         if ((flags & kFirst) && n >= 2 && !mbar_wait(acc_free + b, ((n >> 1) - 1) & 1, abort_flag)) break;
         tc_fence_after();
-        // dV^T, dK^T of the key block += dO2^T P, Q2^T dS of the step
-        const uint32_t aQ = a0 + PL::kQ + s * 65536, aDO = aQ + 32768;
-        const uint32_t tDV = tmem + 256 + b * 128, tDK = tDV + 64;
+        // dV^T += dO2^T P, or dK^T += Q2^T dS, of the key block
+        const uint32_t aA = a0 + PL::kQ + s * 65536 + (is_v ? 32768 : 0);
+        const uint32_t tD = tmem + 256 + b * 128 + (is_v ? 0 : 64);
 #pragma unroll
         for (int kk = 0; kk < 8; kk++)
-          umma_bf16(tDV, mnmajor(aDO, kk, 16384), mnmajor(a0 + PL::kP, kk, 8192), idesc_g,
-                    ((flags & kFirst) && kk == 0) ? 0u : 1u);
-        umma_commit(p_free);
-        if (!mbar_wait(ds_full, u & 1, abort_flag)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; kk++)
-          umma_bf16(tDK, mnmajor(aQ, kk, 16384), mnmajor(a0 + PL::kDS, kk, 8192), idesc_g,
-                    ((flags & kFirst) && kk == 0) ? 0u : 1u);
-        umma_commit(ds_free);
-        // Q2, dO2 reusable: this step's S and dP were complete before its softmax wrote P
+          umma_bf16(tD, mnmajor(aA, kk, 16384), mnmajor(aB, kk, 8192), idesc_g, ((flags & kFirst) && kk == 0) ? 0u : 1u);
+        umma_commit(in_free);
+        // Q2, dO2 reusable once both issuers are done: this step's S and dP were complete
+        // before its softmax wrote P
         umma_commit(ld_free + s);
         issued++;
         if (flags & kLast) {
@@ -654,9 +668,9 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
         u++;
       }
       if (issued > 0) {
-        umma_commit(bar_drain + 2);
+        umma_commit(bar_drain + warp - 5);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain + 2, 0, &no_abort);
+        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
       }
     }
     __syncwarp();
@@ -754,7 +768,8 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
 }  // namespace
 
 bool backward_pair_supported(const Geo& g) {
-  return g.dtype == PYR_BF16 && g.d == 128 && g.b == 64 && g.G == 1 && g.q_offset == 0 && g.Nq == g.N;
+  return g.dtype == PYR_BF16 && g.d == 128 && g.b == 64 && g.G == 1 && g.q_offset == 0 && g.Nq == g.N &&
+         g.topk <= 128;
 }
 
 cudaError_t launch_backward_dq_pair(const Geo& g, const CUtensorMap& mq, const CUtensorMap& mk,

@@ -34,14 +34,18 @@ __device__ __forceinline__ int lower_bound_smem(const int* a, int n, int v) {
 }
 
 // Warp-level compaction of one idx row (query block iq, in slot order, by the
-// rule above) into L: the accepted routes, ascending, then iq itself. Returns
-// the length on every lane; L is complete (and visible to the warp) on return.
-__device__ inline int compact_route_row(const int32_t* __restrict__ row, int topk, int iq, int* L, int* status) {
+// rule above) into L: the accepted routes, ascending, then iq itself. Lane l
+// reads slot 32 c + l as get(c) (topk <= 128: at most 4 chunks). Returns the
+// length on every lane; L is complete (and visible to the warp) on return.
+template <typename Get>
+__device__ inline int compact_route_row_with(Get get, int topk, int iq, int* L, int* status) {
   const int lane = threadIdx.x & 31;
   int base = 0, pmax = -1;
-  for (int k0 = 0; k0 < topk; k0 += 32) {
-    const int k = k0 + lane;
-    const int j = k < topk ? row[k] : -1;
+#pragma unroll
+  for (int c = 0; c < 4; c++) {
+    const int k0 = 32 * c;
+    if (k0 >= topk) break;
+    const int j = k0 + lane < topk ? get(c) : -1;
     const bool in_range = j >= 0 && j < iq;
     int incl = in_range ? j : -1;
 #pragma unroll
@@ -61,6 +65,12 @@ __device__ inline int compact_route_row(const int32_t* __restrict__ row, int top
   if (lane == 0) L[base] = iq;
   __syncwarp();
   return base + 1;
+}
+
+// The same, reading the row from global memory.
+__device__ inline int compact_route_row(const int32_t* __restrict__ row, int topk, int iq, int* L, int* status) {
+  const int lane = threadIdx.x & 31;
+  return compact_route_row_with([&](int c) { return row[32 * c + lane]; }, topk, iq, L, status);
 }
 
 // Compaction of the routes of nq (1..2) consecutive query blocks, one warp per
