@@ -15,15 +15,17 @@
 //                       back into tensor memory over the S tile it came from;
 //                       epilogue;
 //   warp 4*MT           TMA producer of Q (once) and of the K tiles (64 keys);
-//   warp 4*MT+1         MMA issuer: S = Q K^T into TMEM (two S buffers),
-//                       O += P V with P read from TMEM, V from shared memory;
-//   warp 4*MT+2         TMA producer of the V tiles.
+//   warp 4*MT+1         MMA issuer of S = Q K^T into TMEM (two S buffers);
+//   warp 4*MT+2         TMA producer of the V tiles;
+//   warp 4*MT+3         MMA issuer of O += P V, P read from TMEM, V from
+//                       shared memory.
+// One thread issues an MMA about every 65 cycles, while an M = 128, N = 64
+// MMA runs in about 32, so the two products get an issuing thread each.
 // K and V have separate rings: a K tile is released as soon as its QK MMA has
 // finished, so the next K loads run one tile ahead of the late PV use of V.
-// tcgen05 MMAs of one thread execute in issue order and a commit covers every
-// earlier MMA, so S buffer reuse needs no extra barrier: QK of tile t+2 is
-// issued after PV of tile t, and the softmax of tile t+2 starts only once the
-// commit of QK t+2 (hence PV t) has landed.
+// S buffer reuse: QK of tile t+2 writes the S slot that holds P of tile t, so
+// its issuer first waits for the commit of PV t (bar_s_free); the softmax of
+// tile t+2 starts only once the commit of QK t+2 (hence PV t) has landed.
 // The K/V tile list is the union of the query blocks' routed blocks and their
 // diagonal blocks, ascending; each entry carries a mode per query block
 // (skip / full / causal). With PHBA prefix states (M > 0; PHBA summary 3.3 and
@@ -57,12 +59,12 @@ struct Plan {
   static constexpr int kKV = kQ + MT * 32768;          // K ring: NS x [2][64][128 B], then V ring
   static constexpr int kV = kKV + NS * 16384;
   static constexpr int kBar = kV + NS * 16384;         // mbarriers
-  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 3;
+  static constexpr int kNumBars = 1 + 4 * NS + 2 + 2 + 3 + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;    // tmem slot, abort flag, tile count
   static constexpr int kTiles = kMisc + 16;            // tile entries: (block << 4) | modes
   static constexpr int kEnd = kTiles + kMaxTiles * 4;
   static constexpr int kBytes = kEnd + 1024;           // + alignment slack
-  static constexpr int kThreads = (4 * MT + 3) * 32;
+  static constexpr int kThreads = (4 * MT + 4) * 32;
   static constexpr int kTmemCols = MT == 1 ? 256 : 512;
   static constexpr int kMinBlocks = kBytes <= 113 * 1024 ? 2 : 1;
 };
@@ -100,6 +102,8 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
   uint64_t* bar_o = bar_p_full + 2;
   uint64_t* bar_drain = bar_o + 1;
   uint64_t* bar_done = bar_drain + 1;  // every MMA of the CTA finished (one phase)
+  uint64_t* bar_drain2 = bar_done + 1;  // the P.V issuer's MMAs finished
+  uint64_t* bar_s_free = bar_drain2 + 1;  // [2] the P.V MMAs that read P from an S slot done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
   int* tiles = reinterpret_cast<int*>(smem + PL::kTiles);
@@ -127,6 +131,9 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     mbar_init(bar_o, 1);
     mbar_init(bar_drain, 1);
     mbar_init(bar_done, 1);
+    mbar_init(bar_drain2, 1);
+    mbar_init(bar_s_free, 1);
+    mbar_init(bar_s_free + 1, 1);
     fence_mbar_init();
     *abort_flag = 0;
   }
@@ -223,58 +230,71 @@ __global__ void __launch_bounds__(Plan<MT, NS>::kThreads, Plan<MT, NS>::kMinBloc
     }
     __syncwarp();
   } else if (warp == softmax_warps + 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ Q.K^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kKeys, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
       // operand descriptors: the base of each operand once; a stage and a K step add offsets to the
       // start-address field (16-byte units, no carry: shared addresses stay below 2^18 bytes)
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024), dK = sdesc_sw128(smem_u32(sK), 16, 1024);
-      const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       int issued = 0;
-      for (int t = 0; t <= T && ok; t++) {
-        if (t < T) {
-          const int s = t % NS, sb = t & 1;
-          ok = mbar_wait(bar_k_full + s, (t / NS) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dKs = dK + (uint64_t)(s * (16384 >> 4));
+      for (int t = 0; t < T && ok; t++) {
+        const int s = t % NS, sb = t & 1;
+        ok = mbar_wait(bar_k_full + s, (t / NS) & 1, abort_flag);
+        // S slot sb held P of tile t - 2 until that tile's P.V MMAs were done
+        if (ok && t >= 2) ok = mbar_wait(bar_s_free + sb, ((t >> 1) - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dKs = dK + (uint64_t)(s * (16384 >> 4));
 #pragma unroll
-          for (int mt = 0; mt < MT; mt++)
+        for (int mt = 0; mt < MT; mt++)
 #pragma unroll
-            for (int kk = 0; kk < 8; kk++)
-              umma_bf16(tS + (mt * 2 + sb) * 64, dQ + (uint64_t)((mt * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
-                        dKs + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
-          umma_commit(bar_s_full + sb);
-          umma_commit(bar_k_free + s);
-          issued++;
-        }
-        if (t >= 1) {
-          const int u = t - 1, s = u % NS, pb = u & 1;
-          ok = mbar_wait(bar_p_full + pb, (u >> 1) & 1, abort_flag);
-          if (ok) ok = mbar_wait(bar_v_full + s, (u / NS) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t dVs = dV + (uint64_t)(s * (16384 >> 4));
-          const uint32_t acc0 = u > 0 ? 1u : 0u;
-#pragma unroll
-          for (int mt = 0; mt < MT; mt++)
-#pragma unroll
-            for (int kk = 0; kk < 4; kk++)
-              umma_bf16_ts(tO + mt * 128, tS + (mt * 2 + pb) * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), idesc_pv,
-                           kk > 0 ? 1u : acc0);
-          umma_commit(bar_v_free + s);
-          umma_commit(bar_o);
-          issued++;
-        }
+          for (int kk = 0; kk < 8; kk++)
+            umma_bf16(tS + (mt * 2 + sb) * 64, dQ + (uint64_t)((mt * 32768 + (kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                      dKs + (uint64_t)(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+        umma_commit(bar_s_full + sb);
+        umma_commit(bar_k_free + s);
+        issued++;
       }
-      if (ok) umma_commit(bar_done);  // after the last P.V: the epilogue may read O
       if (issued > 0) {
         // every MMA issued so far must finish before the CTA frees its tensor memory
         umma_commit(bar_drain);
         volatile int no_abort = 0;
         mbar_wait(bar_drain, 0, &no_abort);
+      }
+    }
+    __syncwarp();
+  } else if (warp == softmax_warps + 3) {
+    // ------------------------------------------------------------ P.V issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);
+      bool ok = true;
+      int issued = 0;
+      for (int u = 0; u < T && ok; u++) {
+        const int s = u % NS, pb = u & 1;
+        ok = mbar_wait(bar_p_full + pb, (u >> 1) & 1, abort_flag);
+        if (ok) ok = mbar_wait(bar_v_full + s, (u / NS) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dVs = dV + (uint64_t)(s * (16384 >> 4));
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++)
+#pragma unroll
+          for (int kk = 0; kk < 4; kk++)
+            umma_bf16_ts(tO + mt * 128, tS + (mt * 2 + pb) * 64 + kk * 8, dVs + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                         kk > 0 ? 1u : acc0);
+        umma_commit(bar_v_free + s);
+        umma_commit(bar_o);
+        umma_commit(bar_s_free + pb);
+        issued++;
+      }
+      if (ok) umma_commit(bar_done);  // after the last P.V: the epilogue may read O
+      if (issued > 0) {
+        umma_commit(bar_drain2);
+        volatile int no_abort = 0;
+        mbar_wait(bar_drain2, 0, &no_abort);
       }
     }
     __syncwarp();
