@@ -18,7 +18,8 @@
 // Gradients (the SIMT path: fp32 on the CUDA cores, every dtype and shape the
 // library takes). P is recomputed from the saved log-sum-exp as A.1.4 states;
 // D_t = dO_t . O_t is computed once per row into the caller's workspace.
-//   bwd_delta_kernel  one warp per query row: D_t
+//   bwd_delta_kernel  one warp per query row: D_t (bf16 rows of 128: the
+//                     vectorised bwd_delta_bf16_d128_kernel)
 //   bwd_dq_kernel     one warp per query row: walks the row's routed blocks
 //                     and its own block, dQ_t = sum_k dS_tk k_k / sqrt(d)
 //   bwd_dkdv_kernel   one warp per key: walks the query blocks that route to
@@ -26,6 +27,8 @@
 //                     own block, dK_k = sum_t dS_tk q_t / sqrt(d),
 //                     dV_k = sum_t P_tk dO_t over the G heads of the group
 // No atomics touch the gradients: every output element has one owner.
+#include <algorithm>
+
 #include "pyr_common.cuh"
 
 namespace pyr {
@@ -217,6 +220,50 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) bwd_delta_kernel(const T* _
   if (lane == 0) delta[row] = a;
 }
 
+// D_t for bf16 rows of 128: 16 lanes per row (16 bytes of O and of dO each),
+// and each warp has 8 rows (4 per half-warp) of loads in flight per iteration.
+__device__ __forceinline__ float dot_bf16x8(uint4 a, uint4 b) {
+  const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&b);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; i++) {
+    const float2 u = __bfloat1622float2(x[i]), v = __bfloat1622float2(y[i]);
+    s = fmaf(u.x, v.x, s);
+    s = fmaf(u.y, v.y, s);
+  }
+  return s;
+}
+
+__global__ void __launch_bounds__(256) bwd_delta_bf16_d128_kernel(const __nv_bfloat16* __restrict__ O,
+                                                                  const __nv_bfloat16* __restrict__ dO,
+                                                                  float* __restrict__ delta, int64_t rows) {
+  const int lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
+  const int64_t warp_id = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r0 = warp_id * 8; r0 < rows; r0 += nwarps * 8) {  // the same trip count for the whole warp
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      const int64_t r = r0 + half * 4 + k;
+      a[k] = b[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows) {
+        a[k] = __ldg(reinterpret_cast<const uint4*>(O + r * 128) + sub);
+        b[k] = __ldg(reinterpret_cast<const uint4*>(dO + r * 128) + sub);
+      }
+    }
+    float s[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) s[k] = dot_bf16x8(a[k], b[k]);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1)
+#pragma unroll
+      for (int k = 0; k < 4; k++) s[k] += __shfl_xor_sync(0xffffffffu, s[k], o);
+    const int64_t r = r0 + half * 4 + sub;
+    if (sub < 4 && r < rows) delta[r] = sub == 0 ? s[0] : sub == 1 ? s[1] : sub == 2 ? s[2] : s[3];
+  }
+}
+
 template <typename T, int DPL>
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
     bwd_dq_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V, const T* __restrict__ dO,
@@ -333,8 +380,13 @@ cudaError_t launch_grads(const Geo& g, const void* Q, const void* K, const void*
   const T* k = static_cast<const T*>(K);
   const T* v = static_cast<const T*>(V);
   const T* d = static_cast<const T*>(dO);
-  if (parts & kBwdDelta)
+  if ((parts & kBwdDelta) && sizeof(T) == 2 && g.d == 128) {
+    const unsigned grid = (unsigned)std::min<int64_t>((rows + 63) / 64, 148 * 16);  // 8 warps x 8 rows per CTA pass
+    bwd_delta_bf16_d128_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(O),
+                                                     reinterpret_cast<const __nv_bfloat16*>(dO), delta, rows);
+  } else if (parts & kBwdDelta) {
     bwd_delta_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(static_cast<const T*>(O), d, delta, g);
+  }
   if (parts & kBwdDq)
     bwd_dq_kernel<T, DPL><<<rgrid, kWarpsPerCta * 32, 0, st>>>(q, k, v, d, lse, delta, idx, static_cast<T*>(dQ), g);
   if (parts & kBwdDkdv)

@@ -40,9 +40,11 @@
 // topk + 1 tiles). dK/dV lists range from one block to every later query
 // block (a block that every query routes to), so dK/dV CTAs take key blocks
 // from an atomic work counter, the long lists first, and the longest list
-// starts at the beginning. Warps 0-3: one thread per tensor-memory lane;
-// warp 4: producer (route lists, TMA); warps 5, 6, 7: MMA issuers (dQ: S, dP,
-// dQ; dK/dV: S and dP, dV, dK). A thread issues one MMA about every 65
+// starts at the beginning. Warps 0-7: softmax, warps w and w + 4 on
+// tensor-memory lanes 32 (w % 4) .. + 31 with 32 columns each (two warps per
+// scheduler, so one's tensor-memory loads overlap the other's math); warp 8:
+// producer (route lists, TMA); warps 9, 10, 11: MMA issuers (dQ: S, dP, dQ;
+// dK/dV: S and dP, dV, dK). A thread issues one MMA about every 65
 // cycles (measured), while an N = 64 MMA runs in about 32, so a single
 // issuer would leave the tensor pipe idle half the time. Every wait is
 // bounded; an abort drains in-flight copies and MMAs and frees tensor memory.
@@ -78,7 +80,7 @@ struct DqPairPlan {
   static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag
   static constexpr int kList = kMisc + 16;          // the producer's route list
   static constexpr int kBytes = kList + kTileListPitch * 4;
-  static constexpr int kThreads = 8 * 32;
+  static constexpr int kThreads = 12 * 32;
   static constexpr int kTmemCols = 512;  // S^T, dP^T of 2 steps at 128 s (+64); dQ^T of 2 blocks at 256 + 64 b
 };
 
@@ -101,7 +103,7 @@ struct KvPairPlan {
   static constexpr int kNumBars = 24;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag, first work item
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kThreads = 8 * 32;
+  static constexpr int kThreads = 12 * 32;
   static constexpr int kTmemCols = 512;  // S, dP of 2 steps at 128 s (+64); dV^T, dK^T of 2 blocks at 256 + 128 b (+64)
 };
 // Key blocks whose lists hold more query blocks than this are scheduled first.
@@ -126,6 +128,15 @@ __device__ __forceinline__ void store_row_sw128(unsigned char* base, int r, cons
 #pragma unroll
   for (int c = 0; c < 8; c++)
     *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
+// Half h (chunks 4h .. 4h + 3, N elements 32h .. 32h + 31) of row r of such an operand.
+__device__ __forceinline__ void store_row_half_sw128(unsigned char* base, int r, int h, const uint32_t* v) {
+  unsigned char* row = base + r * 128;
+#pragma unroll
+  for (int c = 0; c < 4; c++)
+    *reinterpret_cast<uint4*>(row + (((4 * h + c) ^ (r & 7)) << 4)) =
+        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
 }
 
 // The four shared-memory descriptors of one K = 16 slice kk (0..7):
@@ -178,12 +189,12 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
     mbar_init(q_free, 2);
     for (int s = 0; s < 2; s++) {
       mbar_init(row_full + s, 1);
-      mbar_init(row_free + s, 4);
+      mbar_init(row_free + s, 8);
       mbar_init(s_full + s, 2);
-      mbar_init(s_free + s, 4);
-      mbar_init(p_full + s, 4);
+      mbar_init(s_free + s, 8);
+      mbar_init(p_full + s, 8);
       mbar_init(dq_full + s, 1);
-      mbar_init(dq_free + s, 4);
+      mbar_init(dq_free + s, 8);
     }
     for (int s = 0; s < NS; s++) {
       mbar_init(kv_full + s, 1);
@@ -193,7 +204,7 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
     fence_mbar_init();
     *abort_flag = 0;
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
   }
@@ -202,7 +213,7 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     int u = 0, nq = 0;  // steps and blocks whose copies were issued
     bool ok = true;
@@ -297,11 +308,11 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
       if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5 || warp == 6) {
-    // ------------------------------------------------------------ S^T (warp 5) and dP^T (warp 6) issuers
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------------------------------------ S^T (warp 9) and dP^T (warp 10) issuers
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // keys x rows, both K-major
-      const bool is_s = warp == 5;
+      const bool is_s = warp == 9;
       const uint32_t a0 = smem_u32(smem), aB = a0 + PL::kQ + (is_s ? 0 : 16384);  // Q or dO
       int issued = 0, u = 0, n = 0;
       while (true) {
@@ -325,13 +336,13 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
         u++;
       }
       if (issued > 0) {
-        umma_commit(bar_drain + warp - 5);
+        umma_commit(bar_drain + warp - 9);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
+        mbar_wait(bar_drain + warp - 9, 0, &no_abort);
       }
     }
     __syncwarp();
-  } else if (warp == 7) {
+  } else if (warp == 11) {
     // ------------------------------------------------------------ dQ issuer
     if (lane == 0) {
       constexpr uint32_t idesc_q = idesc_bf16_f32(128, 64, 1, 1);  // d x rows, both MN-major
@@ -369,10 +380,12 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ one thread per key (lane)
-    const int r = warp * 32 + lane;  // key r % 64 of the step's tile r / 64
+    // ------------------------------------------------------------ softmax: warps w and w + 4 share
+    // tensor-memory lanes 32 (w % 4) .. + 31 (one key each) and take columns (rows) 0-31 / 32-63
+    const int q4 = warp & 3, c0 = (warp >> 2) * 32;
+    const int r = q4 * 32 + lane;  // key r % 64 of the step's tile r / 64
     const int half = r >> 6, kr = r & 63;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const float sl2 = rsqrtf((float)g.d) * kLog2e, scale = rsqrtf((float)g.d);
     int u = 0, n = 0;
     while (true) {
@@ -382,12 +395,10 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
       if ((si.flags & kFirst) && !warp_wait(row_full + b, (n >> 1) & 1, abort_flag)) break;  // lse, D
       if (!warp_wait(s_full + (u & 1), (u >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      float sv[64], dp[64];
-      const uint32_t tS = tmem + (u & 1) * 128 + lane_base;
+      float sv[32], dp[32];
+      const uint32_t tS = tmem + (u & 1) * 128 + lane_base + c0;
       tmem_ld32(tS, sv);
-      tmem_ld32(tS + 32, sv + 32);
       tmem_ld32(tS + 64, dp);
-      tmem_ld32(tS + 96, dp + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -395,14 +406,14 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
       const int unit = si.w / g.nqb;
       const int p0 = (g.i0 + si.w % g.nqb) * 64 - g.q_offset, rows = min(64, g.Nq - p0);
       const int x = (half ? si.b : si.a) * 64 + kr;  // this thread's key position
-      // rows that attend the key: [c_lo, c_hi); none in a padding half or past the keys; in
-      // the block's own tile only rows at or after the key
-      const int c_lo = (si.flags & (half ? kOwnB : kOwnA)) ? kr : 0;
-      const int c_hi = ((half && (si.flags & kPadB)) || x >= g.N) ? 0 : rows;
-      const float* s_row = reinterpret_cast<const float*>(smem + PL::kRow + b * 512);
-      uint32_t pk[32];
+      // rows that attend the key: [c_lo, c_hi) (columns c0 + c); none in a padding half or past the
+      // keys; in the block's own tile only rows at or after the key
+      const int c_lo = ((si.flags & (half ? kOwnB : kOwnA)) ? kr : 0) - c0;
+      const int c_hi = (((half && (si.flags & kPadB)) || x >= g.N) ? 0 : rows) - c0;
+      const float* s_row = reinterpret_cast<const float*>(smem + PL::kRow + b * 512) + c0;
+      uint32_t pk[16];
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {
+      for (int c = 0; c < 32; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(s_row + c);
         const float4 d4 = *reinterpret_cast<const float4*>(s_row + 64 + c);
         const float2 y0 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), make_float2(sl2, sl2), make_float2(-l4.x, -l4.y));
@@ -416,7 +427,7 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
         pk[c / 2 + 1] = pack_bf16(e2 * (dp[c + 2] - d4.z), e3 * (dp[c + 3] - d4.w));
       }
       // dS^T over the V tiles: the step's dP^T MMAs (committed with s_full) have read them
-      store_row_sw128(smem + PL::kKV + s * 65536 + 32768, r, pk);
+      store_row_half_sw128(smem + PL::kKV + s * 65536 + 32768, r, c0 >> 5, pk);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full + (u & 1));
@@ -424,19 +435,17 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
         if (lane == 0) mbar_arrive(row_free + b);  // the block's lse and D are read
         if (!warp_wait(dq_full + b, (n >> 1) & 1, abort_flag)) break;
         tc_fence_after();
-        float o[64];
-        const uint32_t tDQ = tmem + 256 + b * 64 + lane_base;
-        tmem_ld32(tDQ, o);
-        tmem_ld32(tDQ + 32, o + 32);
+        float o[32];
+        tmem_ld32(tmem + 256 + b * 64 + lane_base + c0, o);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dq_free + b);
-        // lane r of dQ^T is feature r: column c is row p0 + c
-        __nv_bfloat16* dst = dQ + ((size_t)unit * g.Nq + p0) * 128 + r;
+        // lane r of dQ^T is feature r: column c0 + c is row p0 + c0 + c
+        __nv_bfloat16* dst = dQ + ((size_t)unit * g.Nq + p0 + c0) * 128 + r;
 #pragma unroll
-        for (int c = 0; c < 64; c++)
-          if (c < rows) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
+        for (int c = 0; c < 32; c++)
+          if (c0 + c < rows) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
         n++;
       }
       if (si.flags & kEnd) break;
@@ -448,7 +457,7 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) report(status, PYR_ETIMEOUT);
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, PL::kTmemCols);
   }
@@ -522,20 +531,20 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
       mbar_init(ld_full + s, 1);
       mbar_init(ld_free + s, 2);
       mbar_init(s_full + s, 1);
-      mbar_init(s_free + s, 4);
+      mbar_init(s_free + s, 8);
       mbar_init(acc_full + s, 2);
-      mbar_init(acc_free + s, 4);
+      mbar_init(acc_free + s, 8);
     }
-    mbar_init(p_full, 4);
+    mbar_init(p_full, 8);
     mbar_init(p_free, 1);
-    mbar_init(ds_full, 4);
+    mbar_init(ds_full, 8);
     mbar_init(ds_free, 1);
     for (int k = 0; k < 3; k++) mbar_init(bar_drain + k, 1);
     fence_mbar_init();
     *abort_flag = 0;
     *first_item = grab_item(ctr, long_list, offset, g);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_slot, PL::kTmemCols);
     tmem_relinquish();
   }
@@ -545,7 +554,7 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const bool has_work = *first_item >= 0;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int u = 0, n = 0;  // steps and key blocks whose copies were issued
@@ -596,7 +605,7 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
       for (int m = max(0, n - 2); m < n; m++) mbar_wait(kv_full + (m & 1), (m >> 1) & 1, &no_abort);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ S, dP issuer
     if (lane == 0 && has_work) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);  // rows x keys, both K-major
@@ -632,11 +641,11 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 6 || warp == 7) {
-    // ------------------------------------------------------------ dV (warp 6) and dK (warp 7) issuers
+  } else if (warp == 10 || warp == 11) {
+    // ------------------------------------------------------------ dV (warp 10) and dK (warp 11) issuers
     if (lane == 0 && has_work) {
       constexpr uint32_t idesc_g = idesc_bf16_f32(128, 64, 1, 1);  // d x keys, both MN-major
-      const bool is_v = warp == 6;
+      const bool is_v = warp == 10;
       uint64_t* in_full = is_v ? p_full : ds_full;    // P or dS written
       uint64_t* in_free = is_v ? p_free : ds_free;    // ... read by this issuer's MMAs
       const uint32_t a0 = smem_u32(smem), aB = a0 + (is_v ? PL::kP : PL::kDS);
@@ -668,17 +677,19 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
         u++;
       }
       if (issued > 0) {
-        umma_commit(bar_drain + warp - 5);
+        umma_commit(bar_drain + warp - 9);
         volatile int no_abort = 0;
-        mbar_wait(bar_drain + warp - 5, 0, &no_abort);
+        mbar_wait(bar_drain + warp - 9, 0, &no_abort);
       }
     }
     __syncwarp();
   } else if (has_work) {
-    // ------------------------------------------------------------ one thread per row (lane)
-    const int r = warp * 32 + lane;  // row r % 64 of the step's query block r / 64
+    // ------------------------------------------------------------ softmax: warps w and w + 4 share
+    // tensor-memory lanes 32 (w % 4) .. + 31 (one row each) and take columns (keys) 0-31 / 32-63
+    const int q4 = warp & 3, c0 = (warp >> 2) * 32;
+    const int r = q4 * 32 + lane;  // row r % 64 of the step's query block r / 64
     const int half = r >> 6, rr = r & 63;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const float sl2 = rsqrtf((float)g.d) * kLog2e, scale = rsqrtf((float)g.d);
     int u = 0, n = 0;
     while (true) {
@@ -687,28 +698,26 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
       const StepInfo si = info[s];
       const int unit = si.w / g.nb, x0 = (si.w % g.nb) * 64, keys = min(64, g.N - x0);
       const int p = (half ? si.b : si.a) * 64 + rr;  // this thread's row position
-      // keys the row attends: [0, c_hi); none in a padding half or past the rows; in the key
-      // block's own query block only keys up to the row
+      // keys the row attends: [0, c_hi) (columns c0 + c); none in a padding half or past the rows;
+      // in the key block's own query block only keys up to the row
       const bool in = !(half && (si.flags & kPadB)) && p < g.Nq;
-      const int c_hi = in ? ((!half && (si.flags & kOwnA)) ? min(keys, rr + 1) : keys) : 0;
+      const int c_hi = (in ? ((!half && (si.flags & kOwnA)) ? min(keys, rr + 1) : keys) : 0) - c0;
       const size_t row = (size_t)unit * g.Nq + min(p, g.Nq - 1);
       const float lse2 = lse[row] * kLog2e, D = delta[row];
       if (!warp_wait(s_full + s, (u >> 1) & 1, abort_flag)) break;
       tc_fence_after();
-      float sv[64], dp[64];
-      const uint32_t tS = tmem + s * 128 + lane_base;
+      float sv[32], dp[32];
+      const uint32_t tS = tmem + s * 128 + lane_base + c0;
       tmem_ld32(tS, sv);
-      tmem_ld32(tS + 32, sv + 32);
       tmem_ld32(tS + 64, dp);
-      tmem_ld32(tS + 96, dp + 32);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free + s);
-      uint32_t pk[32], dk[32];
+      uint32_t pk[16], dk[16];
       const float2 scl = make_float2(sl2, sl2), offs = make_float2(-lse2, -lse2), dd = make_float2(-D, -D);
 #pragma unroll
-      for (int c = 0; c < 32; c++) {
+      for (int c = 0; c < 16; c++) {
         const float2 y = __ffma2_rn(make_float2(sv[2 * c], sv[2 * c + 1]), scl, offs);
         const float e0 = 2 * c < c_hi ? ex2(y.x) : 0.f, e1 = 2 * c + 1 < c_hi ? ex2(y.y) : 0.f;
         const float2 z = __fadd2_rn(make_float2(dp[2 * c], dp[2 * c + 1]), dd);
@@ -716,38 +725,36 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
         dk[c] = pack_bf16(e0 * z.x, e1 * z.y);
       }
       if (u >= 1 && !warp_wait(p_free, (u - 1) & 1, abort_flag)) break;  // the previous dV MMAs read P
-      store_row_sw128(smem + PL::kP, r, pk);
+      store_row_half_sw128(smem + PL::kP, r, c0 >> 5, pk);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
       if (u >= 1 && !warp_wait(ds_free, (u - 1) & 1, abort_flag)) break;  // the previous dK MMAs read dS
-      store_row_sw128(smem + PL::kDS, r, dk);
+      store_row_half_sw128(smem + PL::kDS, r, c0 >> 5, dk);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(ds_full);
       if (si.flags & kLast) {
         if (!warp_wait(acc_full + b, (n >> 1) & 1, abort_flag)) break;
         tc_fence_after();
-        // lane r of dV^T / dK^T is feature r: column c is key x0 + c
-        const uint32_t tDV = tmem + 256 + b * 128 + lane_base;
-        float o[64];
+        // lane r of dV^T / dK^T is feature r: column c0 + c is key x0 + c0 + c
+        const uint32_t tDV = tmem + 256 + b * 128 + lane_base + c0;
+        float o[32];
         tmem_ld32(tDV, o);
-        tmem_ld32(tDV + 32, o + 32);
         tmem_wait_ld();
-        __nv_bfloat16* dst = dV + ((size_t)unit * g.N + x0) * 128 + r;
+        __nv_bfloat16* dst = dV + ((size_t)unit * g.N + x0 + c0) * 128 + r;
 #pragma unroll
-        for (int c = 0; c < 64; c++)
-          if (c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c]);
+        for (int c = 0; c < 32; c++)
+          if (c0 + c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c]);
         tmem_ld32(tDV + 64, o);
-        tmem_ld32(tDV + 96, o + 32);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_free + b);
-        dst = dK + ((size_t)unit * g.N + x0) * 128 + r;
+        dst = dK + ((size_t)unit * g.N + x0 + c0) * 128 + r;
 #pragma unroll
-        for (int c = 0; c < 64; c++)
-          if (c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
+        for (int c = 0; c < 32; c++)
+          if (c0 + c < keys) dst[(size_t)c * 128] = __float2bfloat16_rn(o[c] * scale);
         n++;
       }
       if (si.flags & kEnd) break;
@@ -759,7 +766,7 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0) report(status, PYR_ETIMEOUT);
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, PL::kTmemCols);
   }
