@@ -35,6 +35,12 @@ CASES = [
     # 64-row MHA blocks (the paired-list kernels): ragged tail, odd and even list lengths, two batches
     W0.scaled(name="bf16_mha_ragged", B=2, Hq=2, Hkv=2, N=2000, Nq=2000, d=128, b=64, topk=7, cap=14, dtype=BF16,
               seed=46),
+    # key blocks that more than 64 query blocks attend (needles): the dK/dV work order puts them first
+    W0.scaled(name="bf16_mha_long_lists", B=1, Hq=2, Hkv=2, N=8192, Nq=8192, d=128, b=64, topk=24, cap=48,
+              dtype=BF16, seed=47, n_needle=4),
+    # one key block: a single step whose second half is padding
+    W0.scaled(name="bf16_mha_one_block", B=1, Hq=2, Hkv=2, N=64, Nq=64, d=128, b=64, topk=4, cap=8, dtype=BF16,
+              seed=48),
     W0.scaled(name="f32_b16_d128", B=1, Hq=2, Hkv=1, N=333, Nq=333, d=128, b=16, topk=5, cap=10, dtype=F32, seed=45),
 ]
 
@@ -83,6 +89,16 @@ def test_backward_small(w):
     gv = np.pad(g["dV"].reshape(w.B * w.Hkv, w.N, w.d), ((0, 0), (0, pad), (0, 0))).reshape(-1, w.b, w.d)
     _close(w, gk, dK, "dK")
     _close(w, gv, dV, "dV")
+
+
+def test_long_lists_case_has_long_lists():
+    # the needles of bf16_mha_long_lists are attended by more than 64 query blocks (oracle routes)
+    w = [c for c in CASES if c.name == "bf16_mha_long_lists"][0]
+    Q, K, V, _ = synth.generate(w)
+    idx = oracle.select_all(w, Q, K)[0]
+    nb = (w.N + w.b - 1) // w.b
+    longest = max(np.bincount(row[row >= 0], minlength=nb).max() for row in idx.reshape(w.B * w.Hkv, -1))
+    assert longest + 1 > 64
 
 
 def test_route_inversion_reports_bad_routes():
