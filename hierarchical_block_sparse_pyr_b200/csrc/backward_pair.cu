@@ -87,8 +87,8 @@ struct DqPairPlan {
 // One step (two blocks on the M side), written by the producer before the step's copies.
 struct StepInfo {
   int a, b;   // the two blocks: key blocks (dQ) or query blocks (dK, dV)
-  int flags;  // kFirst / kLast (of the query block), kEnd (of the CTA), own / padding tiles
-  int w;      // work item: unit * nqb + query block
+  int flags;  // kFirst / kLast (of the work item's list), kEnd (of the CTA), own / padding tiles
+  int w;      // work item: unit * nqb + query block (dQ) or unit * nb + key block (dK, dV)
 };
 constexpr int kFirst = 1, kLast = 2, kEnd = 4, kOwnA = 8, kOwnB = 16, kPadB = 32;
 
@@ -100,7 +100,7 @@ struct KvPairPlan {
   static constexpr int kDS = 212992;   // dS [128 rows][64 keys] bf16, MN-major operand
   static constexpr int kInfo = 229376;  // 2 stages x StepInfo
   static constexpr int kBar = kInfo + 64;
-  static constexpr int kNumBars = 24;
+  static constexpr int kNumBars = 23;
   static constexpr int kMisc = kBar + kNumBars * 8;  // tensor-memory base, abort flag, first work item
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kThreads = 12 * 32;
@@ -121,16 +121,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Row r of a [128][64] bf16 MN-major operand with 128-byte swizzle (row = the
-// K index, 64 contiguous N elements): 16-byte chunk c sits at chunk c ^ (r % 8).
-__device__ __forceinline__ void store_row_sw128(unsigned char* base, int r, const uint32_t* v) {
-  unsigned char* row = base + r * 128;
-#pragma unroll
-  for (int c = 0; c < 8; c++)
-    *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-}
-
-// Half h (chunks 4h .. 4h + 3, N elements 32h .. 32h + 31) of row r of such an operand.
+// Half h (16-byte chunks 4h .. 4h + 3, N elements 32h .. 32h + 31) of row r of a
+// [128][64] bf16 MN-major operand with 128-byte swizzle (row = the K index, 64
+// contiguous N elements): chunk c of a row sits at chunk c ^ (r % 8).
 __device__ __forceinline__ void store_row_half_sw128(unsigned char* base, int r, int h, const uint32_t* v) {
   unsigned char* row = base + r * 128;
 #pragma unroll
@@ -167,15 +160,15 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
   uint64_t* q_full = bars;              // a block's Q, dO landed
   uint64_t* q_free = bars + 1;          // the block's last S^T, dP^T MMAs done (2 issuers)
   uint64_t* row_full = bars + 2;        // [2] a block's lse, D written
-  uint64_t* row_free = bars + 4;        // [2] ... read (4 warps)
+  uint64_t* row_free = bars + 4;        // [2] ... read (8 softmax warps)
   uint64_t* kv_full = bars + 6;         // [NS] a step's K2, V2 landed, its StepInfo written
   uint64_t* kv_free = kv_full + NS;     // [NS] the step's dQ MMAs done: K2, V2 and dS^T reusable
   uint64_t* s_full = kv_free + NS;      // [2] S^T, dP^T of a step in tensor memory (2 issuers)
-  uint64_t* s_free = s_full + 2;        // [2] ... read into registers (4 warps)
-  uint64_t* p_full = s_free + 2;        // [2] dS^T of a step written (4 warps)
+  uint64_t* s_free = s_full + 2;        // [2] ... read into registers (8 softmax warps)
+  uint64_t* p_full = s_free + 2;        // [2] dS^T of a step written (8 softmax warps)
   uint64_t* dq_full = p_full + 2;       // [2] a block's dQ^T complete
-  uint64_t* dq_free = dq_full + 2;      // [2] ... read into registers (4 warps)
-  uint64_t* bar_drain = dq_free + 2;   // [3] each issuer's MMAs done
+  uint64_t* dq_free = dq_full + 2;      // [2] ... read into registers (8 softmax warps)
+  uint64_t* bar_drain = dq_free + 2;    // [3] each issuer's MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + PL::kMisc + 4);
   StepInfo* info = reinterpret_cast<StepInfo*>(smem + PL::kInfo);
@@ -509,12 +502,12 @@ __global__ void __launch_bounds__(KvPairPlan::kThreads, 1)
   uint64_t* ld_full = bars + 4;    // [2] a step's Q2, dO2 landed, its StepInfo written
   uint64_t* ld_free = bars + 6;    // [2] the step's dV and dK MMAs done (2 issuers): Q2, dO2 reusable
   uint64_t* s_full = bars + 8;     // [2] S, dP of a step in tensor memory
-  uint64_t* s_free = bars + 10;    // [2] ... read into registers (4 warps)
+  uint64_t* s_free = bars + 10;    // [2] ... read into registers (8 softmax warps)
   uint64_t* acc_full = bars + 12;  // [2] a key block's dV^T, dK^T complete (2 issuers)
-  uint64_t* acc_free = bars + 14;  // [2] ... read into registers (4 warps)
-  uint64_t* p_full = bars + 16;    // P written (4 warps)
+  uint64_t* acc_free = bars + 14;  // [2] ... read into registers (8 softmax warps)
+  uint64_t* p_full = bars + 16;    // P written (8 softmax warps)
   uint64_t* p_free = bars + 17;    // the dV MMAs that read P done
-  uint64_t* ds_full = bars + 18;   // dS written (4 warps)
+  uint64_t* ds_full = bars + 18;   // dS written (8 softmax warps)
   uint64_t* ds_free = bars + 19;   // the dK MMAs that read dS done
   uint64_t* bar_drain = bars + 20;  // [3] each issuer's MMAs done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + PL::kMisc);

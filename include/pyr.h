@@ -394,7 +394,10 @@ PYR_API int bsa_route_invert(const pyr_shape* s, const int32_t* idx, int32_t* of
  *   idx    device, as given to bsa_forward.
  *   offset, rho device, as written by bsa_route_invert from the same idx.
  *   delta  device, [B][Hq][Nq] fp32 workspace (overwritten with D_t).
- *   dQ     device, [B][Hq][Nq][d] in s->dtype (written).
+ *   dQ     device, [B][Hq][Nq][d] in s->dtype (written). Before the dQ
+ *          kernel writes it, its memory also holds the work list of the dK/dV
+ *          kernel (bf16, d = 128, b = 64, G = 1), so it must not overlap any
+ *          other argument.
  *   dK, dV device, [B][Hkv][N][d] in s->dtype (written, zero where no row
  *          attends).
  * Supported: whole-sequence prefill (q_offset == 0 and Nq == N); other
