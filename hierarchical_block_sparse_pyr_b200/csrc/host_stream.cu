@@ -22,6 +22,7 @@
 #include <map>
 #include <memory>
 #include <mutex>
+#include <vector>
 
 #include "pyr_common.cuh"
 
@@ -53,11 +54,51 @@ ChunkLayout layout_for(const pyr_shape* s, int64_t P, int64_t nqb, int upc, bool
   return c;
 }
 
-// Chunk size when the caller passes 0: about 16 chunks per call, so that the
-// last chunk (whose compute and copy-out are not hidden) is small.
-int auto_units(const pyr_shape* s) {
+// Chunk sizes when the caller passes 0. Every chunk costs a fixed overhead (its
+// copies and launches), and the last chunk's compute and copy-out are not
+// hidden, so the chunks shrink towards the end: chunks of `cap` units first,
+// then cap/2, ..., 2, 1, 1 (measured at 32K, 16 one-unit chunks take 8.7 ms
+// per step and 8 two-unit chunks 8.4 ms, against 7.6 ms for the copies alone).
+// cap: a quarter of the units, and at most 96 MiB of inputs per chunk.
+int auto_cap(const pyr_shape* s) {
   const int U = s->B * s->Hkv;
-  return U <= 16 ? 1 : (U + 15) / 16;
+  const size_t elt = s->dtype == PYR_F32 ? 4 : 2;
+  const size_t in_unit = (size_t)(s->Hq / s->Hkv) * s->Nq * s->d * elt + 2 * (size_t)s->N * s->d * elt;
+  const size_t by_bytes = (96u << 20) / (in_unit ? in_unit : 1);
+  size_t cap = (size_t)(U / 4);
+  if (cap > by_bytes) cap = by_bytes;
+  return cap < 1 ? 1 : (int)cap;
+}
+
+// The chunk sizes of a call (in order), summing to U: uniform chunks of upc
+// units (the last one possibly smaller), or with upc == 0 the shrinking
+// schedule above. Returns the largest chunk, which sizes the device slots.
+int chunk_schedule(const pyr_shape* s, int upc, std::vector<int>* sizes) {
+  const int U = s->B * s->Hkv;
+  sizes->clear();
+  if (upc > 0) {
+    if (upc > U) upc = U;
+    for (int u0 = 0; u0 < U; u0 += upc) sizes->push_back(U - u0 < upc ? U - u0 : upc);
+    return upc;
+  }
+  const int cap = auto_cap(s);
+  std::vector<int> tail = {1, 1};  // the end of the call, last chunk last
+  int sum = 2;
+  for (int n = 2; n < cap && sum + n <= U; n *= 2) {
+    tail.insert(tail.begin(), n);
+    sum += n;
+  }
+  if (sum > U) {  // too few units for the tail: one unit per chunk
+    sizes->assign(U, 1);
+    return 1;
+  }
+  const int rest = U - sum;
+  if (rest % cap) sizes->push_back(rest % cap);
+  for (int k = 0; k < rest / cap; k++) sizes->push_back(cap);
+  sizes->insert(sizes->end(), tail.begin(), tail.end());
+  int mx = 1;
+  for (int n : *sizes) mx = n > mx ? n : mx;
+  return mx;
 }
 
 // Two copy streams and the events that order the slots, made once per CUDA
@@ -111,9 +152,8 @@ int status_of(cudaError_t e) { return e == cudaSuccess ? PYR_OK : PYR_ECUDA; }
 extern "C" size_t pyr_host_workspace_bytes(const pyr_shape* s, int units_per_chunk, int with_lse) {
   if (units_per_chunk < 0 || pyr::validate_shape(s) != PYR_OK) return 0;
   const int64_t P = pyr_num_nodes(s), nqb = pyr_num_qblocks(s);
-  const int U = s->B * s->Hkv;
-  int upc = units_per_chunk ? units_per_chunk : auto_units(s);
-  if (upc > U) upc = U;
+  std::vector<int> sizes;
+  const int upc = chunk_schedule(s, units_per_chunk, &sizes);
   return layout_for(s, P, nqb, upc, with_lse != 0).total;
 }
 
@@ -124,9 +164,8 @@ extern "C" int bsa_forward_host(const pyr_shape* s, const void* Q, const void* K
   if (rc0 != PYR_OK) return rc0;
   const int64_t P = pyr_num_nodes(s), nqb = pyr_num_qblocks(s);
   if (!Q || !K || !V || !O || !workspace || ((uintptr_t)workspace & 15u) || units_per_chunk < 0) return PYR_EINVAL;
-  const int U = s->B * s->Hkv;
-  int upc = units_per_chunk ? units_per_chunk : auto_units(s);
-  if (upc > U) upc = U;
+  std::vector<int> sizes;
+  const int upc = chunk_schedule(s, units_per_chunk, &sizes);
   const ChunkLayout c = layout_for(s, P, nqb, upc, lse != nullptr);
   if (workspace_bytes < c.total) return PYR_EINVAL;
 
@@ -152,9 +191,9 @@ extern "C" int bsa_forward_host(const pyr_shape* s, const void* Q, const void* K
   if (e == cudaSuccess) e = cudaStreamWaitEvent(ds.d2h, ds.entry, 0);
   int rc = status_of(e);
 
-  const int nchunks = (U + upc - 1) / upc;
-  for (int ch = 0; ch < nchunks && rc == PYR_OK; ch++) {
-    const int u0 = ch * upc, n = U - u0 < upc ? U - u0 : upc;
+  const int nchunks = (int)sizes.size();
+  for (int ch = 0, u0 = 0; ch < nchunks && rc == PYR_OK; u0 += sizes[ch], ch++) {
+    const int n = sizes[ch];
     const int k = ch % kSlots;
     char* slot = base + k * c.slot;
     char *dq = slot, *dk = slot + c.q, *dv = dk + c.kv, *dout = dv + c.kv;

@@ -325,7 +325,10 @@ PYR_API int dense_forward(const pyr_shape* s, const void* Q, const void* K, cons
  * without device copies of them holds them.
  * The (batch, kv head) units are independent through all three steps, so
  * they stream through the device in chunks of `units_per_chunk` consecutive
- * units (0: about 16 chunks per call): chunk c is computed on `stream` while
+ * units (0: chunks that shrink towards the end of the call, from a quarter of
+ * the units with at most 96 MiB of inputs each down to 2, 1, 1, so that the
+ * per-chunk costs stay small and the last, unhidden chunk is one unit):
+ * chunk c is computed on `stream` while
  * chunk c + 1 is copied in and chunk c - 1's output copied out on two copy
  * streams the library keeps per device (made on the first call on a device,
  * held until the process exits). O and lse are bit-identical to the three

@@ -157,8 +157,13 @@ def test_host_entry_point_workspace_size():
     U = w.B * w.Hkv
     for upc, with_lse in ((1, False), (1, True), (3, True), (U, False)):
         assert P.host_workspace_bytes(s, upc, with_lse) == _ws_expected(w, upc, with_lse), (upc, with_lse)
-    # 0 picks about 16 chunks; more units per chunk than there are units means one chunk
-    assert P.host_workspace_bytes(s, 0) == _ws_expected(w, max(1, -(-U // 16)), False)
+    # 0 shrinks the chunks towards the end of the call; the largest, which sizes the slots, is a quarter
+    # of the units with at most 96 MiB of inputs (Q, K, V) per chunk: 4 of the 32K workload's 16 units
+    in_unit = (w.G * w.Nq + 2 * w.N) * w.d * 2
+    cap = max(1, min(U // 4, (96 << 20) // in_unit))
+    assert cap == 4
+    assert P.host_workspace_bytes(s, 0) == _ws_expected(w, cap, False)
+    # more units per chunk than there are units means one chunk
     assert P.host_workspace_bytes(s, 10 * U) == _ws_expected(w, U, False)
     assert P.host_workspace_bytes(s, -1) == 0
     bad = P.shape_of(w)
