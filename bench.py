@@ -146,6 +146,8 @@ def kernel_source(kernel, w):
     if kernel == "pyramid":
         return "pyramid.cu"
     if kernel == "select":
+        if w.decode:
+            return "select_decode.cu" if w.G <= 8 else "select.cu"  # the decode walk (G <= 8), else the SIMT walk
         return "select_tc.cu" if tc_select(w) else "select.cu"
     if w.decode:
         return "attn_decode_warp.cu" if w.G <= 8 else "attn_decode.cu"
