@@ -287,6 +287,16 @@ __global__ void __launch_bounds__(DqPairPlan::kThreads, 1)
               tma_load_3d(smem + PL::kQ + 16384 + h * 8192, &tmDO, h * 64, p0, unit, q_full);
             }
             nq++;
+            // the next block's Q and dO (first read here, so from DRAM) into L2: its load waits for
+            // this block's last S^T, dP^T and then stalls the next block's first step
+            if (!last_w) {
+              const int wn = w + (int)gridDim.x;
+              const int pn = (g.i0 + wn % g.nqb) * 64 - g.q_offset;
+              for (int h = 0; h < 2; h++) {
+                tma_prefetch_3d(&tmQ, h * 64, pn, wn / g.nqb);
+                tma_prefetch_3d(&tmDO, h * 64, pn, wn / g.nqb);
+              }
+            }
           }
         }
       }
